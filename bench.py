@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the R2L sidecar forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+
+A step is one full sidecar forward (in_proj → conv+SiLU → x_proj → dt_proj →
+reverse scan → out_proj → LayerNorm + gated residual) over one batch of the
+serving workload of "Bifocal Diffusion Language Models" (arXiv 2606.27732v1,
+§4.3 / Table 3: batch 8, prompt 4096; d_model 2048 per §4.1), with seeded
+synthetic hidden states and weights.  Every rank (one per GPU, launched by
+torchrun for N > 1) runs its own batch: sequences are independent, so the
+batch shards with no data-path collective (weak scaling).
+
+`value` is device time (CUDA events on the launching stream, max over ranks)
+with inputs resident in HBM; the per-step working set (~1.5 GB of activations
+and workspace) is far larger than the 126 MB L2, so no flush is needed.
+`e2e` is the same call with the hidden states copied from pinned host memory
+and the result copied back inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "R2L sidecar tokens/sec at B=8,L=4096,d=2048; scan HBM GB/s % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=2, help="workload 1..4 (2 = the headline)")
+    ap.add_argument("--general-a", action="store_true", help="force the general-A scan path")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "reverse_selective_ssm_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(stage, workload_tag):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
+        kv = {}
+        for line in open(f):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("stage") == stage and kv.get("workload") == workload_tag and \
+                kv.get("source_sha") == source_sha() and "dram_bytes_per_launch" in kv:
+            try:
+                return float(kv["dram_bytes_per_launch"])
+            except ValueError:
+                return None
+    return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.gpu = vis.split(",")[local_rank].strip() if vis else str(local_rank)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def algorithmic(case, stage):
+    """(bound, amount per launch, unit) for one stage on ``case`` (valid tokens only)."""
+    d, E, R, N = case.dims.d_model, case.dims.d_inner, case.dims.dt_rank, case.dims.d_state
+    T = case.valid_tokens
+    a = 2 if case.dtype.itemsize == 2 else 4
+    if stage == "in_proj":
+        return "tensor", 2.0 * T * d * 2 * E, "flop"
+    if stage == "x_proj":
+        return "tensor", 2.0 * T * E * (R + 2 * N), "flop"
+    if stage == "dt_proj":
+        return "tensor", 2.0 * T * R * E, "flop"
+    if stage == "out_proj":
+        return "tensor", 2.0 * T * E * d, "flop"
+    if stage == "conv":
+        return "hbm", float(T) * E * (a + a), "byte"
+    if stage == "scan":       # u, z, dt_raw read, y written (act) + B, C read (fp32)
+        return "hbm", float(T) * (E * 4 * a + 2 * N * 4), "byte"
+    if stage == "ln_residual":  # o read, h read, h written
+        return "hbm", float(T) * d * 3 * a, "byte"
+    raise KeyError(stage)
+
+
+def roofline_obj(case, stage, ms, peaks, peak_kind, workload_tag):
+    bound, amount, _ = algorithmic(case, stage)
+    if bound == "tensor":
+        achieved = amount / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        unit = "TFLOP/s"
+        peak_note = f"{peak_kind} cuBLAS bf16 sustained"
+    else:
+        achieved = amount / (ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        peak_note = f"{peak_kind} HBM copy"
+    return {"kernel": stage, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "peak_source": peak_note,
+            "algorithmic_per_launch": amount, "ms_per_launch": round(ms, 5),
+            "traffic": read_traffic(stage, workload_tag)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from reverse_selective_ssm_b200 import binding as bd
+    from reverse_selective_ssm_b200 import synthetic as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bd.load()
+    case = S.make_case(args.config)
+    flags = bd.R2L_FLAG_GENERAL_A if args.general_a else 0
+    dims = bd.dims_of(case.dims, case.dtype, flags)
+    h = case.h.to(dev)
+    wdev = [bd.weights_to_device(w, dev) for w in case.weights]
+    lengths = None if case.lengths is None else case.lengths.to(dev)
+    ws = bd.alloc_workspace(dims, case.B, case.L, dev)
+    stream = torch.cuda.current_stream()
+    hooks = len(wdev)
+    nst = len(bd.STAGES)
+
+    def step(events=None):
+        launches = 0
+        for k in range(hooks):
+            if events is not None:
+                launches += bd.sidecar_forward_profiled(h, wdev[k], dims, case.s[k], events[k], lengths, ws, stream)
+            else:
+                bd.sidecar_forward(h, wdev[k], dims, case.s[k], lengths, ws, stream)
+        return launches
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, fl = bd.get_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} flags {fl}")
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(hooks)]
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    # touch the events once so their handles exist before the timed region
+    for per_step in evs:
+        for per_hook in per_step:
+            for e in per_hook:
+                e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    launches = 0
+    for k in range(K):
+        launches += step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms_total = t0.elapsed_time(t1)
+    stage_ms = {s: 0.0 for s in bd.STAGES}
+    for k in range(K):
+        for hk in range(hooks):
+            e = evs[k][hk]
+            for i, s in enumerate(bd.STAGES):
+                stage_ms[s] += e[i].elapsed_time(e[i + 1])
+    per_launch = {s: v / (K * hooks) for s, v in stage_ms.items()}
+
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # ---- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_host = case.h.pin_memory()
+        out_host = torch.empty_like(h_host).pin_memory()
+        for _ in range(max(1, args.warmup // 2)):
+            h.copy_(h_host, non_blocking=True)
+            step()
+            out_host.copy_(h, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            h.copy_(h_host, non_blocking=True)
+            step()
+            out_host.copy_(h, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = h_host.numel() * h_host.element_size()
+        e2e = {"value": round(case.valid_tokens * world * K / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "api": "r2l_sidecar_forward via binding, pinned host hidden in/out"}
+
+    if rank != 0:
+        return None
+
+    peaks, peak_kind = load_peaks()
+    workload_tag = f"config{args.config}"
+    dom = max(per_launch, key=per_launch.get)
+    line = {
+        "metric": METRIC,
+        "value": round(case.valid_tokens * world * K / (ms_total * 1e-3), 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_total / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if case.dtype.itemsize == 2 else "f32",
+        "data": "synthetic (seeded N(0,1) hidden states, N(0,0.02) weights, A=-(1..16), D=1)",
+        "config": {"workload": case.name, "B": case.B, "L": case.L, "hooks": hooks,
+                   "d_model": case.dims.d_model, "d_inner": case.dims.d_inner,
+                   "d_state": case.dims.d_state, "dt_rank": case.dims.dt_rank,
+                   "valid_tokens_per_gpu": case.valid_tokens, "s": case.s if hooks > 1 else case.s[0],
+                   "l2": "inputs larger than L2 (~1.5 GB working set per step), no flush",
+                   "parallelism": f"dp{world}: one independent batch per GPU, no collective",
+                   "scan_path": "general-A" if args.general_a else "auto (power fast path when A=-(1..16))"},
+        "roofline": roofline_obj(case, dom, per_launch[dom], peaks, peak_kind, workload_tag),
+        "roofline_scan": roofline_obj(case, "scan", per_launch["scan"], peaks, peak_kind, workload_tag),
+        "stage_ms": {s: round(v, 5) for s, v in per_launch.items()},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+        "source_sha": source_sha(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case)
+    return line
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(case, sample_seqs=(0, 1)):
+    """The float64 oracle, as it stands, on a bounded sample of the workload."""
+    import oracle as O
+    from reverse_selective_ssm_b200 import synthetic as S
+    h = S.to_f64(case.h)
+    ws = [S.weights_f64(w) for w in case.weights]
+    t = time.perf_counter()
+    if len(ws) == 1:
+        O.sidecar_forward(h, ws[0], case.s[0], None, "bf16", list(sample_seqs))
+    else:
+        O.sidecar_stack(h, ws, case.s, None, "bf16", list(sample_seqs))
+    dt = time.perf_counter() - t
+    tokens = case.L * len(sample_seqs)
+    return {"value": round(tokens * len(ws) / dt / max(1, len(ws)), 2), "unit": "tokens/s",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"sequences {list(sample_seqs)} of the workload in full ({tokens} tokens), "
+                      f"numpy float64 oracle, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores, each step a bounded sample: the last
+    512 positions of one sequence (exact for those positions, since the output
+    at i depends on positions ≥ i only)."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle as O
+    from reverse_selective_ssm_b200 import synthetic as S
+    case = S.make_case(args.config)
+    h = S.to_f64(case.h)
+    ws = [S.weights_f64(w) for w in case.weights]
+    span = min(512, case.L)
+
+    def step(k):
+        b = k % case.B
+        n = case.L if case.lengths is None else int(case.lengths[b])
+        sub = h[b:b + 1, max(0, n - span):n]
+        if len(ws) == 1:
+            O.sidecar_forward(sub, ws[0], case.s[0], None, "bf16")
+        else:
+            O.sidecar_stack(sub, ws, case.s, None, "bf16")
+        return sub.shape[1]
+
+    for k in range(args.warmup):
+        step(k)
+    t = time.perf_counter()
+    tokens = 0
+    for k in range(args.steps):
+        tokens += step(k)
+    dt = time.perf_counter() - t
+    v = round(tokens / dt, 2)
+    sample = f"per step the last {span} positions of one sequence, numpy float64 oracle"
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": case.name, "B": case.B, "L": case.L, "hooks": len(ws)},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * r2l.h — C ABI of libr2l, the B200 (sm_100a) R2L sidecar forward.
+ *
+ * The operation is the reverse-direction Mamba stream of "Bifocal Diffusion
+ * Language Models: Asymmetric Bidirectional Context for Parallel Generation"
+ * (arXiv 2606.27732v1), §3.4 "R2LM Architecture", steps ❶–❹: for hidden
+ * states h ∈ R^{B×L×d},
+ *
+ *     h⁺ = h + tanh(s) · LN( flip( Mamba( flip(h) ) ) )
+ *
+ * where Mamba is the Mamba-1 selective-scan block (step ❷; d_state = 16,
+ * d_conv = 4, expand 2 per §4.1) and LN is a LayerNorm local to the stream
+ * (step ❸).  With flip applied per sequence to its valid prefix, the block
+ * runs from each sequence's last valid token to its first:
+ *
+ *     [x | z] = h·W_inᵀ
+ *     u_i     = SiLU(conv_b + Σ_{k=0..3} conv_w[:, 3-k] ⊙ x_{i+k})   (x_j = 0, j ≥ len)
+ *     [Δr | B | C]_i = u_i·W_xᵀ
+ *     Δ_i     = softplus(Δr_i·W_dtᵀ + dt_b)
+ *     H_i     = exp(Δ_i ⊗ A) ⊙ H_{i+1} + (Δ_i ⊙ u_i) ⊗ B_i,   H_len = 0,  A = -exp(A_log)
+ *     y_i     = (H_i·C_i + D ⊙ u_i) ⊙ SiLU(z_i)
+ *     o_i     = y_i·W_outᵀ
+ *     h_i    += tanh(s) · (γ ⊙ (o_i − mean) / sqrt(var + 1e-5) + β)      (0 ≤ i < len)
+ *
+ * Conventions (all entry points):
+ *   - Every pointer in a forward call is a DEVICE pointer owned by the caller,
+ *     except the r2l_dims / r2l_weights / r2l_debug_out structs themselves,
+ *     which are host memory read during the call only.  The library never
+ *     allocates, frees or synchronises on the forward path.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and runs asynchronously.  Errors found on the
+ *     host are returned as r2l_status before anything is enqueued; nothing is
+ *     thrown and nothing is printed.
+ *   - Matrices are row-major, nn.Linear convention W[out][in].
+ *   - The library holds no mutable global state; calls on different streams
+ *     with different workspaces may run concurrently.  Two calls that share a
+ *     workspace must be ordered by the caller.
+ */
+#ifndef R2L_H
+#define R2L_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define R2L_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define R2L_API __attribute__((visibility("default")))
+#else
+#define R2L_API
+#endif
+
+typedef enum {
+  R2L_OK = 0,
+  R2L_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad enum */
+  R2L_ERR_UNSUPPORTED = 2,   /* d_state != 16, d_conv != 4, or a size the kernels do not tile */
+  R2L_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+  R2L_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than r2l_workspace_size() */
+  R2L_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  R2L_ERR_DEVICE_CHECK = 6   /* r2l_get_device_status found a device-side flag */
+} r2l_status;
+
+typedef enum {
+  R2L_BF16 = 0,   /* bf16 activations and GEMM weights, fp32 accumulation and state */
+  R2L_FP32 = 1    /* fp32 everywhere, true fp32 arithmetic (no TF32) */
+} r2l_dtype;
+
+/* r2l_dims.flags */
+#define R2L_FLAG_GENERAL_A 0x1u   /* never take the A = -(1..16) power fast path of the scan */
+
+/* Device status bits, reported by r2l_get_device_status(). */
+#define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */
+
+typedef struct {
+  int d_model;       /* d: hidden width of the backbone                             */
+  int d_inner;       /* E: expanded width (2·d_model in the paper's setup)         */
+  int d_state;       /* N: SSM state size; must be 16                              */
+  int dt_rank;       /* R: rank of the Δ projection                                */
+  int d_conv;        /* W: depthwise conv width; must be 4                         */
+  r2l_dtype dtype;   /* activation / GEMM-weight storage type                      */
+  unsigned flags;    /* R2L_FLAG_* bits, 0 by default                              */
+} r2l_dims;
+
+/* One hook's parameters.  Device pointers, read-only, 16-byte aligned.
+ * "act" = bf16 for R2L_BF16, fp32 for R2L_FP32.                               */
+typedef struct {
+  const void  *in_proj_w;   /* act  [2E, d]   rows 0..E-1 produce x, rows E..2E-1 produce z */
+  const float *conv_w;      /* fp32 [E, W]    tap W-1 multiplies the current token          */
+  const float *conv_b;      /* fp32 [E]                                                      */
+  const void  *x_proj_w;    /* act  [R+2N, E] output rows ordered Δr | B | C                 */
+  const void  *dt_proj_w;   /* act  [E, R]                                                   */
+  const float *dt_proj_b;   /* fp32 [E]                                                      */
+  const float *A_log;       /* fp32 [E, N]    A = -exp(A_log)                                */
+  const float *D;           /* fp32 [E]                                                      */
+  const void  *out_proj_w;  /* act  [d, E]                                                   */
+  const float *ln_w;        /* fp32 [d]  LayerNorm γ; ln_w = ln_b = NULL: no LayerNorm       */
+  const float *ln_b;        /* fp32 [d]  LayerNorm β                                         */
+} r2l_weights;
+
+/* Optional intermediates for testing (device pointers, NULL = not wanted).
+ * Row b·L + i holds position i of sequence b; rows with i ≥ len_b hold
+ * unspecified values, except in hhat where they are not written.             */
+typedef struct {
+  void  *x;        /* act  [B·L, E]      in_proj, first half                  */
+  void  *z;        /* act  [B·L, E]      in_proj, second half                 */
+  void  *u;        /* act  [B·L, E]      conv + SiLU                          */
+  float *dbc;      /* fp32 [B·L, R+2N]   x_proj output Δr | B | C             */
+  void  *y;        /* act  [B·L, E]      scan output after the SiLU(z) gate   */
+  void  *o;        /* act  [B·L, d]      out_proj output                      */
+  float *hhat;     /* fp32 [B·L, d]      LayerNorm output (pre-gate)          */
+} r2l_debug_out;
+
+/* ABI version of the loaded library (R2L_ABI_VERSION at build time). */
+R2L_API int r2l_abi_version(void);
+
+/* Human-readable name of a status code; never NULL, static storage. */
+R2L_API const char *r2l_status_string(r2l_status status);
+
+/* Bytes of device workspace a forward call on a [B, L] batch needs.  Returns 0
+ * for invalid dims or sizes.  The size depends only on (dims, B, L).          */
+R2L_API size_t r2l_workspace_size(const r2l_dims *dims, int B, int L);
+
+/* The sidecar forward of §3.4 on hidden [B, L, d_model] (act dtype), updated in
+ * place: rows i < len_b become h⁺, rows i ≥ len_b are neither read nor written.
+ *
+ *   lengths   device int32 [B] of valid lengths, or NULL for all L.  Values
+ *             outside [0, L] are clamped on the device and flagged
+ *             (R2L_DEVFLAG_LENGTH_CLAMPED, see r2l_get_device_status).
+ *   s         the hook's scalar gate; g = tanh(s) is formed in double on the
+ *             host and rounded to float.  If g == 0 the call returns R2L_OK
+ *             without enqueuing anything (the identity at initialisation, §3.4 ❹).
+ *   workspace device scratch of at least r2l_workspace_size(dims, B, L) bytes,
+ *             16-byte aligned, caller-owned; its contents on entry do not
+ *             matter and on return are unspecified (the device status word
+ *             lives at its start).
+ * Checks on the host: non-null pointers, positive sizes, d_state == 16,
+ * d_conv == 4, 16-byte alignment, workspace size, supported tiling.  On any
+ * error nothing is enqueued.                                                   */
+R2L_API r2l_status r2l_sidecar_forward(void *hidden, const r2l_weights *weights, const r2l_dims *dims,
+                               float s, int B, int L, const int32_t *lengths,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same as r2l_sidecar_forward, and also copies the intermediates requested in
+ * *debug (non-NULL fields) into the caller's buffers.  For tests.  Unlike the
+ * forward call it runs the layer even when tanh(s) == 0.                       */
+R2L_API r2l_status r2l_sidecar_forward_debug(void *hidden, const r2l_weights *weights, const r2l_dims *dims,
+                                     float s, int B, int L, const int32_t *lengths,
+                                     void *workspace, size_t workspace_bytes, void *stream,
+                                     const r2l_debug_out *debug);
+
+/* n_hooks sidecar layers applied one after another to the same hidden tensor
+ * (§4.1: a hook after every 4th decoder layer; here the backbone between hooks
+ * is whatever the caller does between calls, i.e. nothing).  weights and s are
+ * host arrays of n_hooks entries.  Same contract as r2l_sidecar_forward.      */
+R2L_API r2l_status r2l_sidecar_stack(void *hidden, const r2l_weights *weights, const float *s, int n_hooks,
+                             const r2l_dims *dims, int B, int L, const int32_t *lengths,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Stages of one hook, in launch order, for r2l_sidecar_forward_profiled. */
+typedef enum {
+  R2L_STAGE_IN_PROJ = 0,      /* [x | z] = h·W_inᵀ                              */
+  R2L_STAGE_CONV = 1,         /* u = SiLU(anti-causal conv(x))                  */
+  R2L_STAGE_X_PROJ = 2,       /* [Δr | B | C] = u·W_xᵀ                          */
+  R2L_STAGE_DT_PROJ = 3,      /* Δr·W_dtᵀ                                       */
+  R2L_STAGE_SCAN = 4,         /* reverse selective scan and SiLU(z) gate        */
+  R2L_STAGE_OUT_PROJ = 5,     /* o = y·W_outᵀ                                   */
+  R2L_STAGE_LN_RESIDUAL = 6,  /* LayerNorm and tanh(s)-gated residual           */
+  R2L_NUM_STAGES = 7
+} r2l_stage;
+
+/* Same as r2l_sidecar_forward, and also records events[k] on `stream` just
+ * before stage k starts and events[R2L_NUM_STAGES] after the last stage.
+ * events: host array of n_events cudaEvent_t handles (passed as void*),
+ * created and owned by the caller; n_events must be R2L_NUM_STAGES + 1.  A
+ * stage that is fused into its neighbour shows zero time.  *launches (if not
+ * NULL) receives the number of kernels the call enqueued.  For measurement.  */
+R2L_API r2l_status r2l_sidecar_forward_profiled(void *hidden, const r2l_weights *weights,
+                                        const r2l_dims *dims, float s, int B, int L,
+                                        const int32_t *lengths, void *workspace,
+                                        size_t workspace_bytes, void *stream,
+                                        void *const *events, int n_events, int *launches);
+
+/* Synchronises `stream`, then reads the device status word that the last
+ * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*
+ * bits.  Returns R2L_ERR_DEVICE_CHECK if any bit is set, R2L_ERR_CUDA if the
+ * stream reported an error, R2L_OK otherwise.  Not for the hot path.          */
+R2L_API r2l_status r2l_get_device_status(const void *workspace, void *stream, uint32_t *flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* R2L_H */

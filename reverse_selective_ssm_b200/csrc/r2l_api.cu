@@ -1,0 +1,313 @@
+// libr2l: host side of the C ABI declared in include/r2l.h — argument checks,
+// workspace carve-up and the launch sequence of the R2L sidecar forward
+// ("Bifocal Diffusion Language Models", arXiv 2606.27732v1, §3.4 steps ❶–❹).
+//
+// Launch sequence for one hook (all on the caller's stream, no host sync):
+//   prep lengths → in_proj GEMM → conv+SiLU → x_proj GEMM → dt_proj GEMM
+//   → reverse selective scan (+SiLU(z) gate) → out_proj GEMM
+//   → LayerNorm + tanh(s)-gated residual (valid rows only)
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "r2l.h"
+#include "common.cuh"
+#include "simt_kernels.cuh"
+#include "scan_simple.cuh"
+
+using r2l::bf16;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Byte offsets of the workspace regions for a [B, L] batch.
+struct Plan {
+  size_t status, len, xz, u, dbc, dt, y, o, total;
+  long long M;
+  int E, d, R, N, ldd;
+  size_t act;
+};
+
+bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
+  if (!dm || B <= 0 || L <= 0) return false;
+  if (dm->d_model <= 0 || dm->d_inner <= 0 || dm->dt_rank <= 0 || dm->d_state <= 0) return false;
+  if (dm->dtype != R2L_BF16 && dm->dtype != R2L_FP32) return false;
+  p->M = (long long)B * L;
+  p->E = dm->d_inner;
+  p->d = dm->d_model;
+  p->R = dm->dt_rank;
+  p->N = dm->d_state;
+  p->ldd = p->R + 2 * p->N;
+  p->act = dm->dtype == R2L_BF16 ? 2 : 4;
+  const size_t M = (size_t)p->M;
+  size_t off = 0;
+  p->status = off; off = align_up(off + 16, kAlign);
+  p->len = off;    off = align_up(off + sizeof(int) * (size_t)B, kAlign);
+  p->xz = off;     off = align_up(off + M * 2 * p->E * p->act, kAlign);
+  p->u = off;      off = align_up(off + M * p->E * p->act, kAlign);
+  p->dbc = off;    off = align_up(off + M * p->ldd * sizeof(float), kAlign);
+  p->dt = off;     off = align_up(off + M * p->E * p->act, kAlign);
+  p->y = off;      off = align_up(off + M * p->E * p->act, kAlign);
+  p->o = off;      off = align_up(off + M * p->d * p->act, kAlign);
+  p->total = off;
+  return true;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+r2l_status check_weights(const r2l_weights* w) {
+  if (!w) return R2L_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->in_proj_w, w->conv_w, w->conv_b, w->x_proj_w, w->dt_proj_w,
+                        w->dt_proj_b, w->A_log, w->D, w->out_proj_w};
+  for (const void* q : ptrs) {
+    if (!q) return R2L_ERR_INVALID_ARG;
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  }
+  if ((w->ln_w == nullptr) != (w->ln_b == nullptr)) return R2L_ERR_INVALID_ARG;
+  if (w->ln_w && (!aligned16(w->ln_w) || !aligned16(w->ln_b))) return R2L_ERR_ALIGNMENT;
+  return R2L_OK;
+}
+
+r2l_status check_call(void* hidden, const r2l_dims* dm, int B, int L, void* ws, size_t ws_bytes,
+                      Plan* plan) {
+  if (!hidden || !dm) return R2L_ERR_INVALID_ARG;
+  if (!make_plan(dm, B, L, plan)) return R2L_ERR_INVALID_ARG;
+  if (dm->d_state != 16 || dm->d_conv != 4) return R2L_ERR_UNSUPPORTED;
+  // grid limits of the launches below
+  if (L > 65535 || B > 65535 || (plan->M + 63) / 64 > 65535) return R2L_ERR_UNSUPPORTED;
+  if (!aligned16(hidden)) return R2L_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < plan->total) return R2L_ERR_WORKSPACE;
+  if (!aligned16(ws)) return R2L_ERR_ALIGNMENT;
+  return R2L_OK;
+}
+
+#define R2L_LAUNCH_CHECK()                                   \
+  do {                                                       \
+    if (cudaPeekAtLastError() != cudaSuccess) {              \
+      (void)cudaGetLastError();                              \
+      return R2L_ERR_CUDA;                                   \
+    }                                                        \
+  } while (0)
+
+// Optional stage-boundary events and launch counting (profiled entry point).
+struct Prof {
+  cudaEvent_t* ev = nullptr;
+  int launches = 0;
+  r2l_status mark(int k, cudaStream_t st) {
+    if (ev && cudaEventRecord(ev[k], st) != cudaSuccess) return R2L_ERR_CUDA;
+    return R2L_OK;
+  }
+};
+
+template <typename TA, typename TW, typename TC>
+r2l_status gemm(const TA* A, int lda, const TW* W, int ldw, TC* C, int ldc, long long M, int N,
+                int K, const int* len, int L, cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
+  r2l::gemm_simt_kernel<TA, TW, TC><<<grid, 256, 0, st>>>(A, lda, W, ldw, C, ldc, (int)M, N, K, len, L);
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, cudaStream_t st,
+                Prof* prof = nullptr) {
+  if (prof) prof->launches++;
+  if (cudaMemsetAsync(ws + p.status, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
+  r2l::prep_lengths_kernel<<<(B + 127) / 128, 128, 0, st>>>(
+      lengths, (int*)(ws + p.len), B, L, (unsigned*)(ws + p.status));
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+#define R2L_TRY(expr)                  \
+  do {                                 \
+    r2l_status _s = (expr);            \
+    if (_s != R2L_OK) return _s;       \
+  } while (0)
+
+template <typename T>
+r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, int B, int L,
+                     char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof) {
+  Prof dummy;
+  if (!prof) prof = &dummy;
+  const long long M = p.M;
+  const int E = p.E, d = p.d, R = p.R;
+  const int* len = (const int*)(ws + p.len);
+  T* xz = (T*)(ws + p.xz);
+  T* u = (T*)(ws + p.u);
+  float* dbc = (float*)(ws + p.dbc);
+  T* dt = (T*)(ws + p.dt);
+  T* y = (T*)(ws + p.y);
+  T* o = (T*)(ws + p.o);
+  const size_t es = sizeof(T);
+
+  // a1: [x | z] = h · W_inᵀ
+  R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
+  prof->launches++;
+  R2L_TRY(gemm(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, st));
+  // a2: u = SiLU(anti-causal conv(x))
+  R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
+  prof->launches++;
+  {
+    dim3 grid((E + 127) / 128, L, B);
+    r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+    R2L_LAUNCH_CHECK();
+  }
+  // a3: [Δr | B | C] = u · W_xᵀ  (fp32 out)
+  R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
+  prof->launches++;
+  R2L_TRY(gemm(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, st));
+  // a4: dt_raw = Δr · W_dtᵀ  (bias + softplus applied in the scan)
+  R2L_TRY(prof->mark(R2L_STAGE_DT_PROJ, st));
+  prof->launches++;
+  R2L_TRY(gemm((const float*)dbc, p.ldd, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, st));
+  // a5: reverse selective scan, y = (C·H + D u) · SiLU(z)
+  R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
+  prof->launches++;
+  {
+    dim3 grid((E + 127) / 128, B);
+    r2l::scan_simple_kernel<T><<<grid, 128, 0, st>>>(u, xz + E, 2 * E, dt, dbc, p.ldd, R, w->A_log,
+                                                     w->D, w->dt_proj_b, y, E, len, L);
+    R2L_LAUNCH_CHECK();
+  }
+  // a6: o = y · W_outᵀ
+  R2L_TRY(prof->mark(R2L_STAGE_OUT_PROJ, st));
+  prof->launches++;
+  R2L_TRY(gemm(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, st));
+
+  if (dbg) {
+    const size_t rowsE = (size_t)M;
+    if (dbg->x && cudaMemcpy2DAsync(dbg->x, E * es, xz, 2 * E * es, E * es, rowsE, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (dbg->z && cudaMemcpy2DAsync(dbg->z, E * es, xz + E, 2 * E * es, E * es, rowsE, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (dbg->u && cudaMemcpyAsync(dbg->u, u, rowsE * E * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (dbg->dbc && cudaMemcpyAsync(dbg->dbc, dbc, rowsE * p.ldd * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (dbg->y && cudaMemcpyAsync(dbg->y, y, rowsE * E * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (dbg->o && cudaMemcpyAsync(dbg->o, o, rowsE * d * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+  }
+  // a7 + a8: LayerNorm (optional) and h += g · ĥ on valid rows
+  float* hhat = dbg ? dbg->hhat : nullptr;
+  R2L_TRY(prof->mark(R2L_STAGE_LN_RESIDUAL, st));
+  prof->launches++;
+  if (w->ln_w)
+    r2l::ln_gate_residual_kernel<T, true><<<(unsigned)M, 256, 0, st>>>(hidden, o, w->ln_w, w->ln_b, g, d, len, L, hhat);
+  else
+    r2l::ln_gate_residual_kernel<T, false><<<(unsigned)M, 256, 0, st>>>(hidden, o, nullptr, nullptr, g, d, len, L, hhat);
+  R2L_LAUNCH_CHECK();
+  R2L_TRY(prof->mark(R2L_NUM_STAGES, st));
+  return R2L_OK;
+}
+
+r2l_status forward_impl(void* hidden, const r2l_weights* weights, const r2l_dims* dims, float s,
+                        int B, int L, const int32_t* lengths, void* workspace,
+                        size_t workspace_bytes, void* stream, const r2l_debug_out* dbg,
+                        Prof* prof = nullptr) {
+  Plan p;
+  R2L_TRY(check_call(hidden, dims, B, L, workspace, workspace_bytes, &p));
+  R2L_TRY(check_weights(weights));
+  if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
+  const float g = (float)std::tanh((double)s);
+  if (g == 0.0f && !dbg) return R2L_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  R2L_TRY(prep(p, ws, lengths, B, L, st, prof));
+  if (dims->dtype == R2L_BF16)
+    return run_layer<bf16>((bf16*)hidden, weights, p, g, B, L, ws, st, dbg, prof);
+  return run_layer<float>((float*)hidden, weights, p, g, B, L, ws, st, dbg, prof);
+}
+
+}  // namespace
+
+extern "C" {
+
+int r2l_abi_version(void) { return R2L_ABI_VERSION; }
+
+const char* r2l_status_string(r2l_status s) {
+  switch (s) {
+    case R2L_OK: return "R2L_OK";
+    case R2L_ERR_INVALID_ARG: return "R2L_ERR_INVALID_ARG: null pointer, bad size or bad enum";
+    case R2L_ERR_UNSUPPORTED: return "R2L_ERR_UNSUPPORTED: shape outside what the kernels implement";
+    case R2L_ERR_ALIGNMENT: return "R2L_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case R2L_ERR_WORKSPACE: return "R2L_ERR_WORKSPACE: workspace missing or too small";
+    case R2L_ERR_CUDA: return "R2L_ERR_CUDA: a CUDA call or kernel launch failed";
+    case R2L_ERR_DEVICE_CHECK: return "R2L_ERR_DEVICE_CHECK: a device-side check raised a flag";
+  }
+  return "R2L_ERR_UNKNOWN";
+}
+
+size_t r2l_workspace_size(const r2l_dims* dims, int B, int L) {
+  Plan p;
+  if (!make_plan(dims, B, L, &p)) return 0;
+  return p.total;
+}
+
+r2l_status r2l_sidecar_forward(void* hidden, const r2l_weights* weights, const r2l_dims* dims,
+                               float s, int B, int L, const int32_t* lengths, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return forward_impl(hidden, weights, dims, s, B, L, lengths, workspace, workspace_bytes, stream,
+                      nullptr);
+}
+
+r2l_status r2l_sidecar_forward_debug(void* hidden, const r2l_weights* weights, const r2l_dims* dims,
+                                     float s, int B, int L, const int32_t* lengths,
+                                     void* workspace, size_t workspace_bytes, void* stream,
+                                     const r2l_debug_out* debug) {
+  if (!debug) return R2L_ERR_INVALID_ARG;
+  return forward_impl(hidden, weights, dims, s, B, L, lengths, workspace, workspace_bytes, stream,
+                      debug);
+}
+
+r2l_status r2l_sidecar_forward_profiled(void* hidden, const r2l_weights* weights,
+                                        const r2l_dims* dims, float s, int B, int L,
+                                        const int32_t* lengths, void* workspace,
+                                        size_t workspace_bytes, void* stream,
+                                        void* const* events, int n_events, int* launches) {
+  if (!events || n_events != R2L_NUM_STAGES + 1) return R2L_ERR_INVALID_ARG;
+  for (int k = 0; k < n_events; ++k)
+    if (!events[k]) return R2L_ERR_INVALID_ARG;
+  Prof prof;
+  prof.ev = (cudaEvent_t*)events;
+  const r2l_status st = forward_impl(hidden, weights, dims, s, B, L, lengths, workspace,
+                                     workspace_bytes, stream, nullptr, &prof);
+  if (launches) *launches = prof.launches;
+  return st;
+}
+
+r2l_status r2l_sidecar_stack(void* hidden, const r2l_weights* weights, const float* s, int n_hooks,
+                             const r2l_dims* dims, int B, int L, const int32_t* lengths,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!weights || !s || n_hooks <= 0) return R2L_ERR_INVALID_ARG;
+  Plan p;
+  R2L_TRY(check_call(hidden, dims, B, L, workspace, workspace_bytes, &p));
+  for (int k = 0; k < n_hooks; ++k) R2L_TRY(check_weights(&weights[k]));
+  if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  bool prepared = false;
+  for (int k = 0; k < n_hooks; ++k) {
+    const float g = (float)std::tanh((double)s[k]);
+    if (g == 0.0f) continue;
+    if (!prepared) {
+      R2L_TRY(prep(p, ws, lengths, B, L, st));
+      prepared = true;
+    }
+    if (dims->dtype == R2L_BF16)
+      R2L_TRY(run_layer<bf16>((bf16*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
+    else
+      R2L_TRY(run_layer<float>((float*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
+  }
+  return R2L_OK;
+}
+
+r2l_status r2l_get_device_status(const void* workspace, void* stream, uint32_t* flags_out) {
+  if (!workspace || !flags_out) return R2L_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return R2L_ERR_CUDA;
+  uint32_t f = 0;
+  if (cudaMemcpy(&f, workspace, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess) return R2L_ERR_CUDA;
+  *flags_out = f;
+  return f ? R2L_ERR_DEVICE_CHECK : R2L_OK;
+}
+
+}  // extern "C"

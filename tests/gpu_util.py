@@ -1,0 +1,112 @@
+"""Helpers shared by the GPU parity tests: run a synthetic case through the C
+ABI and through the CPU oracle, and the tolerance measures the tests use.
+
+Tolerances (the layer's contract):
+  fp32 path: max_i |a_i − b_i| / max(|b_i|, 1e-3·rms(b))  ≤ 1e-4
+  bf16 path: max |a − b| / max |b|                         ≤ 2e-2
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+from reverse_selective_ssm_b200 import binding as bd
+from reverse_selective_ssm_b200 import synthetic as S
+
+TOL_FP32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def err_fp32(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    rms = float(np.sqrt(np.mean(b * b))) if b.size else 0.0
+    den = np.maximum(np.abs(b), 1e-3 * rms)
+    den = np.where(den == 0, 1.0, den)
+    return float(np.max(np.abs(a - b) / den)) if a.size else 0.0
+
+
+def err_bf16(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    if not a.size:
+        return 0.0
+    m = float(np.max(np.abs(b)))
+    return float(np.max(np.abs(a - b))) / (m if m > 0 else 1.0)
+
+
+def err_for(dtype):
+    return err_fp32 if dtype == torch.float32 else err_bf16
+
+
+def tol_for(dtype):
+    return TOL_FP32 if dtype == torch.float32 else TOL_BF16
+
+
+def device_weights(case):
+    return [bd.weights_to_device(w) for w in case.weights]
+
+
+def run_gpu(case, debug=False, flags=0, s=None):
+    """Run ``case`` through libr2l.  Returns (h⁺ on CPU, debug dict on CPU)."""
+    dev = "cuda"
+    dims = bd.dims_of(case.dims, case.dtype, flags)
+    h = case.h.to(dev).contiguous()
+    lengths = None if case.lengths is None else case.lengths.to(dev)
+    ws = bd.alloc_workspace(dims, case.B, case.L)
+    wdev = device_weights(case)
+    outs = {}
+    if debug:
+        assert len(wdev) == 1
+        M, E, d = case.B * case.L, case.dims.d_inner, case.dims.d_model
+        ldd = case.dims.dt_rank + 2 * case.dims.d_state
+        for k in ("x", "z", "u", "y"):
+            outs[k] = torch.full((M, E), float("nan"), dtype=case.dtype, device=dev)
+        outs["o"] = torch.full((M, d), float("nan"), dtype=case.dtype, device=dev)
+        outs["dbc"] = torch.full((M, ldd), float("nan"), dtype=torch.float32, device=dev)
+        outs["hhat"] = torch.full((M, d), float("nan"), dtype=torch.float32, device=dev)
+        bd.sidecar_forward_debug(h, wdev[0], dims, case.s[0] if s is None else s, lengths, ws,
+                                 outputs=outs)
+    elif len(wdev) == 1:
+        bd.sidecar_forward(h, wdev[0], dims, case.s[0] if s is None else s, lengths, ws)
+    else:
+        bd.sidecar_stack(h, wdev, dims, case.s, lengths, ws)
+    torch.cuda.synchronize()
+    st, flags_out = bd.get_device_status(ws)
+    return h.cpu(), {k: v.cpu() for k, v in outs.items()}, flags_out
+
+
+def out_dtype_name(dtype):
+    return "f32" if dtype == torch.float32 else "bf16"
+
+
+def run_oracle(case, batch_indices, intermediates=False, suffix=None):
+    """Oracle h⁺ for the listed sequences (float64 array [B, L, d]).  With
+    ``suffix`` = S, each listed sequence is run on its last S valid positions
+    only (exact for those positions: the output at i depends on j ≥ i only)."""
+    h = S.to_f64(case.h)
+    ws = [S.weights_f64(w) for w in case.weights]
+    lengths = None if case.lengths is None else case.lengths.numpy()
+    od = out_dtype_name(case.dtype)
+    if suffix is None:
+        if len(ws) == 1:
+            return O.sidecar_forward(h, ws[0], case.s[0], lengths, od, batch_indices,
+                                     return_intermediates=intermediates)
+        return O.sidecar_stack(h, ws, case.s, lengths, od, batch_indices)
+    out = np.array(h, copy=True)
+    for b in batch_indices:
+        n = case.L if lengths is None else int(lengths[b])
+        lo = max(0, n - suffix)
+        sub = h[b:b + 1, lo:n]
+        if len(ws) == 1:
+            r = O.sidecar_forward(sub, ws[0], case.s[0], None, od)
+        else:
+            r = O.sidecar_stack(sub, ws, case.s, None, od)
+        out[b, lo:n] = r[0]
+    return out
+
+
+def valid_rows(case, b):
+    n = case.L if case.lengths is None else int(case.lengths[b])
+    return n

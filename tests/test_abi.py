@@ -1,0 +1,131 @@
+"""The C ABI on the CPU: the library loads, exports every function the header
+declares, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from reverse_selective_ssm_b200 import binding as bd
+from reverse_selective_ssm_b200 import build as bld
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bld.build()
+    return bd.load()
+
+
+def header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"R2L_API\s+[\w\s\*]*?\b(r2l_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_exports_every_declared_function(lib):
+    names = header_functions()
+    assert names, "no R2L_API declarations found"
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(bd.EXPORTS) <= set(names)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.r2l_abi_version() == 1
+    for code, name in bd.STATUS.items():
+        assert lib.r2l_status_string(code).decode().startswith(name)
+    assert lib.r2l_status_string(99).decode() == "R2L_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    d = bd.make_dims(2048, 4096)
+    a = bd.workspace_size(d, 8, 4096)
+    assert a > 8 * 4096 * 4096 * 2 * 5          # xz, u, dt, y at least
+    assert bd.workspace_size(d, 8, 4096) == a     # deterministic
+    assert bd.workspace_size(d, 16, 4096) > a
+    assert bd.workspace_size(d, 0, 4096) == 0
+    assert bd.workspace_size(d, 1, -1) == 0
+    assert bd.workspace_size(bd.make_dims(0, 4096), 1, 1) == 0
+    f = bd.make_dims(64, 128, dt_rank=4, dtype=torch.float32)
+    assert bd.workspace_size(f, 1, 64) > 64 * 128 * 4 * 5
+
+
+FAKE = 0x10000  # a 16-byte aligned non-null value; never dereferenced on the host
+
+
+def _weights(ln=True):
+    w = bd.Weights()
+    for f, _ in bd.Weights._fields_:
+        setattr(w, f, FAKE)
+    if not ln:
+        w.ln_w = None
+        w.ln_b = None
+    return w
+
+
+def _call(lib, hidden=FAKE, w=None, dims=None, s=0.5, B=1, L=8, lengths=None, ws=FAKE, ws_bytes=None):
+    dims = dims or bd.make_dims(64, 128, dt_rank=4, dtype=torch.float32)
+    w = w or _weights()
+    if ws_bytes is None:
+        ws_bytes = bd.workspace_size(dims, max(B, 1), max(L, 1)) or 1
+    return lib.r2l_sidecar_forward(hidden, ctypes.byref(w), ctypes.byref(dims), s, B, L, lengths, ws,
+                                   ws_bytes, None)
+
+
+def test_host_validation(lib):
+    assert _call(lib, hidden=None) == 1
+    assert _call(lib, B=0) == 1
+    assert _call(lib, L=0) == 1
+    d = bd.make_dims(64, 128, d_state=8, dt_rank=4, dtype=torch.float32)
+    assert _call(lib, dims=d) == 2
+    d = bd.make_dims(64, 128, d_conv=3, dt_rank=4, dtype=torch.float32)
+    assert _call(lib, dims=d) == 2
+    d = bd.make_dims(64, 128, dt_rank=4, dtype=torch.float32)
+    d.dtype = 7
+    assert _call(lib, dims=d) == 1
+    assert _call(lib, hidden=FAKE + 4) == 3
+    assert _call(lib, ws=FAKE + 8) == 3
+    assert _call(lib, ws=None) == 4
+    assert _call(lib, ws_bytes=16) == 4
+    w = _weights()
+    w.A_log = None
+    assert _call(lib, w=w) == 1
+    w = _weights()
+    w.ln_b = None            # only one of the two LN pointers
+    assert _call(lib, w=w) == 1
+    w = _weights()
+    w.x_proj_w = FAKE + 2
+    assert _call(lib, w=w) == 3
+    assert _call(lib, lengths=FAKE + 1) == 3
+
+
+def test_zero_gate_enqueues_nothing(lib):
+    """tanh(s) == 0 returns R2L_OK before any CUDA call (works with no GPU):
+    the identity at initialisation of §3.4 step ❹."""
+    assert _call(lib, s=0.0) == 0
+    assert _call(lib, s=-0.0) == 0
+    w = _weights()
+    arr = (bd.Weights * 3)(w, w, w)
+    s = (ctypes.c_float * 3)(0.0, 0.0, 0.0)
+    dims = bd.make_dims(64, 128, dt_rank=4, dtype=torch.float32)
+    n = bd.workspace_size(dims, 1, 8)
+    assert lib.r2l_sidecar_stack(FAKE, arr, s, 3, ctypes.byref(dims), 1, 8, None, FAKE, n, None) == 0
+
+
+def test_stack_and_debug_argument_checks(lib):
+    dims = bd.make_dims(64, 128, dt_rank=4, dtype=torch.float32)
+    n = bd.workspace_size(dims, 1, 8)
+    w = _weights()
+    s = (ctypes.c_float * 1)(0.5)
+    assert lib.r2l_sidecar_stack(FAKE, None, s, 1, ctypes.byref(dims), 1, 8, None, FAKE, n, None) == 1
+    assert lib.r2l_sidecar_stack(FAKE, ctypes.byref(w), s, 0, ctypes.byref(dims), 1, 8, None, FAKE, n, None) == 1
+    assert lib.r2l_sidecar_forward_debug(FAKE, ctypes.byref(w), ctypes.byref(dims), 0.5, 1, 8, None, FAKE,
+                                         n, None, None) == 1
+    st = lib.r2l_get_device_status(None, None, None)
+    assert st == 1

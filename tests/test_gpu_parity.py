@@ -1,0 +1,236 @@
+"""CUDA path (through the C ABI) against the float64 CPU oracle.
+
+Covers the five workloads (tiny fp32; single bf16 sequence; the batch-8 × 4096
+serving shape; the 7-hook stack; the ragged batch), plus cases that make the
+scan's state term dominate the output (D = 0, O(1) B and C), ragged tails,
+zero-length sequences, the no-LayerNorm variant, non-structured A, and the
+invariants of §3.4 of "Bifocal Diffusion Language Models" (arXiv 2606.27732v1):
+s = 0 is the identity bit for bit, and the output at position i does not
+depend on positions < i (bit for bit).
+"""
+import numpy as np
+import pytest
+import torch
+
+from reverse_selective_ssm_b200 import binding as bd
+from reverse_selective_ssm_b200 import synthetic as S
+
+from . import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    bd.load()
+
+
+def _check_seq(case, got, want, b, what=""):
+    n = G.valid_rows(case, b)
+    e = G.err_for(case.dtype)(S.to_f64(got[b, :n]), want[b, :n])
+    assert e <= G.tol_for(case.dtype), f"{case.name} {what} b={b}: err {e:.3e}"
+    return e
+
+
+def _check_inter(case, dbg, inter, b, keys=("u", "y", "o", "hhat")):
+    n = G.valid_rows(case, b)
+    L = case.L
+    errs = {}
+    for k in keys:
+        g = S.to_f64(dbg[k][b * L: b * L + n])
+        w = inter[b][k]
+        e = G.err_for(case.dtype)(g, w)
+        errs[k] = e
+        assert e <= G.tol_for(case.dtype), f"{case.name} intermediate {k} b={b}: err {e:.3e}"
+    return errs
+
+
+def _padding_untouched(case, got):
+    if case.lengths is None:
+        return
+    for b, n in enumerate(case.lengths.tolist()):
+        a = got[b, n:]
+        ref = case.h[b, n:]
+        assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                           ref.view(torch.int16) if ref.dtype == torch.bfloat16 else ref.view(torch.int32)), \
+            f"padding of sequence {b} was written"
+
+
+# ----------------------------------------------------------------- config 0
+
+def test_cfg0_fp32_against_oracle():
+    case = S.make_case(0)
+    got, dbg, _ = G.run_gpu(case, debug=True)
+    want, inter = G.run_oracle(case, [0], intermediates=True)
+    _check_seq(case, got, want, 0, "h+")
+    _check_inter(case, dbg, inter, 0, keys=("x", "z", "u", "y", "o", "hhat"))
+
+
+def test_cfg0_s_zero_is_bitwise_identity():
+    case = S.make_case(0)
+    got, _, _ = G.run_gpu(case, s=0.0)
+    assert torch.equal(got.view(torch.int32), case.h.view(torch.int32))
+
+
+def test_cfg0_scan_visible_fp32():
+    """D = 0 and O(1) B, C: the output is the scan's state term."""
+    case = S.make_case(0)
+    case.weights = [S.make_weights(case.dims, torch.float32, seed=200, x_proj_std=0.5, D_value=0.0,
+                                   ln="seeded")]
+    got, dbg, _ = G.run_gpu(case, debug=True)
+    want, inter = G.run_oracle(case, [0], intermediates=True)
+    _check_seq(case, got, want, 0, "h+")
+    _check_inter(case, dbg, inter, 0, keys=("u", "y", "o", "hhat"))
+
+
+def test_fp32_ragged_tails_and_empty():
+    """Sizes that are not multiples of any tile, a zero-length sequence and a
+    length-1 sequence (fp32, tight tolerance)."""
+    dims = S.Dims(d_model=72, d_inner=136, d_state=16, dt_rank=5, d_conv=4)
+    B, L = 4, 70
+    lengths = torch.tensor([70, 0, 1, 33], dtype=torch.int32)
+    h = S.poison_padding(S.make_hidden(B, L, dims.d_model, torch.float32, seed=9), lengths)
+    w = S.make_weights(dims, torch.float32, seed=209, x_proj_std=0.5, D_value=0.5, ln="seeded")
+    case = S.Case("fp32 ragged", dims, torch.float32, B, L, h, [w], [0.9], lengths=lengths)
+    got, _, _ = G.run_gpu(case)
+    want = G.run_oracle(case, range(B))
+    for b in range(B):
+        _check_seq(case, got, want, b)
+    _padding_untouched(case, got)
+
+
+# ----------------------------------------------------------------- config 1
+
+def test_cfg1_bf16_against_oracle():
+    case = S.make_case(1)
+    got, dbg, _ = G.run_gpu(case, debug=True)
+    want, inter = G.run_oracle(case, [0], intermediates=True)
+    _check_seq(case, got, want, 0, "h+")
+    _check_inter(case, dbg, inter, 0, keys=("x", "z", "u", "y", "o", "hhat"))
+
+
+def test_bf16_scan_visible_ragged():
+    """Config-1 widths, two sequences (one ragged), D = 0, O(1) B/C, seeded LN."""
+    case = S.make_case(1, B=2, L=1024)
+    case.lengths = torch.tensor([1024, 700], dtype=torch.int32)
+    case.h = S.poison_padding(case.h, case.lengths)
+    case.weights = [S.make_weights(case.dims, torch.bfloat16, seed=201, x_proj_std=0.8, D_value=0.0,
+                                   ln="seeded")]
+    got, dbg, _ = G.run_gpu(case, debug=True)
+    want, inter = G.run_oracle(case, [0, 1], intermediates=True)
+    for b in (0, 1):
+        _check_seq(case, got, want, b, "h+")
+        _check_inter(case, dbg, inter, b, keys=("u", "y", "o", "hhat"))
+    _padding_untouched(case, got)
+
+
+def test_bf16_general_A_and_no_ln():
+    """Non-structured A (random A_log) without LayerNorm."""
+    dims = S.BIG
+    g = torch.Generator().manual_seed(5)
+    A_log = torch.log(torch.rand((dims.d_inner, 16), generator=g) * 8 + 0.25)
+    case = S.make_case(1, B=1, L=512)
+    case.weights = [S.make_weights(dims, torch.bfloat16, seed=202, x_proj_std=0.8, D_value=0.0,
+                                   ln="none", A_log=A_log)]
+    got, dbg, _ = G.run_gpu(case, debug=True)
+    want, inter = G.run_oracle(case, [0], intermediates=True)
+    _check_seq(case, got, want, 0, "h+")
+    _check_inter(case, dbg, inter, 0, keys=("y", "o", "hhat"))
+
+
+def test_bf16_forced_general_path_matches():
+    """R2L_FLAG_GENERAL_A gives the same result within tolerance."""
+    case = S.make_case(1, B=1, L=512)
+    case.weights = [S.make_weights(case.dims, torch.bfloat16, seed=203, x_proj_std=0.8, D_value=0.0)]
+    a, _, _ = G.run_gpu(case)
+    b, _, _ = G.run_gpu(case, flags=bd.R2L_FLAG_GENERAL_A)
+    want = G.run_oracle(case, [0])
+    _check_seq(case, a, want, 0, "fast")
+    _check_seq(case, b, want, 0, "general")
+
+
+# ----------------------------------------------------------------- invariants
+
+def test_right_context_only_bitwise():
+    case = S.make_case(1, B=1, L=640)
+    case.weights = [S.make_weights(case.dims, torch.bfloat16, seed=204, x_proj_std=0.8)]
+    base, _, _ = G.run_gpu(case)
+    for i in (1, 200, 639):
+        c2 = S.make_case(1, B=1, L=640, weights=False)
+        c2.weights = case.weights
+        h2 = case.h.clone()
+        h2[:, :i] = S.make_hidden(1, i, case.dims.d_model, torch.bfloat16, seed=77)
+        c2.h = h2
+        got, _, _ = G.run_gpu(c2)
+        assert torch.equal(got[:, i:].view(torch.int16), base[:, i:].view(torch.int16)), f"i={i}"
+
+
+def test_deterministic_bitwise():
+    case = S.make_case(1, B=2, L=768)
+    a, _, _ = G.run_gpu(case)
+    b, _, _ = G.run_gpu(case)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_s_zero_bf16_bitwise_and_no_launch():
+    case = S.make_case(1, B=1, L=256)
+    got, _, _ = G.run_gpu(case, s=0.0)
+    assert torch.equal(got.view(torch.int16), case.h.view(torch.int16))
+
+
+def test_lengths_out_of_range_are_clamped_and_flagged():
+    case = S.make_case(1, B=3, L=256)
+    case.lengths = torch.tensor([-5, 100000, 100], dtype=torch.int32)
+    got, _, flags = G.run_gpu(case)
+    assert flags & bd.R2L_DEVFLAG_LENGTH_CLAMPED
+    clamped = S.make_case(1, B=3, L=256)
+    clamped.lengths = torch.tensor([0, 256, 100], dtype=torch.int32)
+    ref, _, flags2 = G.run_gpu(clamped)
+    assert flags2 == 0
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+
+
+# ----------------------------------------------------------------- full sizes
+
+def test_cfg2_serving_shape():
+    """B=8, L=4096: sequences 0 and 7 in full, the last 384 positions of the others."""
+    case = S.make_case(2)
+    got, _, _ = G.run_gpu(case)
+    full = G.run_oracle(case, [0, 7])
+    for b in (0, 7):
+        _check_seq(case, got, full, b, "full")
+    suf = G.run_oracle(case, [1, 2, 3, 4, 5, 6], suffix=384)
+    for b in (1, 2, 3, 4, 5, 6):
+        n = case.L
+        e = G.err_bf16(S.to_f64(got[b, n - 384:]), suf[b, n - 384:])
+        assert e <= G.TOL_BF16, f"suffix b={b}: {e:.3e}"
+
+
+def test_cfg3_stack_of_seven():
+    """B=4, L=8192, 7 hooks: sequence 3 in full, the last 256 positions of 0..2."""
+    case = S.make_case(3)
+    got, _, _ = G.run_gpu(case)
+    full = G.run_oracle(case, [3])
+    _check_seq(case, got, full, 3, "stack full")
+    suf = G.run_oracle(case, [0, 1, 2], suffix=256)
+    for b in (0, 1, 2):
+        e = G.err_bf16(S.to_f64(got[b, -256:]), suf[b, -256:])
+        assert e <= G.TOL_BF16, f"stack suffix b={b}: {e:.3e}"
+
+
+def test_cfg4_ragged_batch():
+    """B=256, L=512, lengths ~ U[64, 512], NaN padding: the shortest, the longest
+    and six random sequences against the oracle; all padding untouched."""
+    case = S.make_case(4)
+    got, _, flags = G.run_gpu(case)
+    assert flags == 0
+    lens = case.lengths.numpy()
+    rng = np.random.default_rng(4)
+    pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens))] + rng.choice(256, 6, replace=False).tolist()))
+    want = G.run_oracle(case, pick)
+    for b in pick:
+        _check_seq(case, got, want, b, "ragged")
+    _padding_untouched(case, got)
+    assert torch.isfinite(torch.cat([got[b, :int(n)].float().flatten() for b, n in enumerate(lens)])).all()
