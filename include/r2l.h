@@ -74,6 +74,7 @@ typedef enum {
 
 /* Device status bits, reported by r2l_get_device_status(). */
 #define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */
+#define R2L_DEVFLAG_TIMEOUT 0x2u          /* a kernel gave up waiting on a pipeline barrier (results invalid) */
 
 typedef struct {
   int d_model;       /* d: hidden width of the backbone                             */

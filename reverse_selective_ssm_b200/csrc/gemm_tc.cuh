@@ -1,0 +1,252 @@
+// Persistent warp-specialised bf16 GEMM on the 5th-generation tensor cores
+// (tcgen05 + TMEM), fed by TMA:
+//
+//     C[m, n] = Σ_k A[m, k] · B[n, k]        (A [M, K], B [N, K], both K-major)
+//
+// which is y = x Wᵀ for an nn.Linear weight W [out, in].  Used for the four
+// projections of the Mamba-1 block in the R2L sidecar (in_proj, x_proj,
+// dt_proj, out_proj; "Bifocal Diffusion Language Models", arXiv 2606.27732v1,
+// §3.4 step ❷).
+//
+// One CTA per SM (192 threads) loops over 128 × BN output tiles:
+//   warp 0     TMA producer: 64-wide K slices of A and B into a STAGES-deep
+//              shared-memory ring (128-byte swizzle), one mbarrier per slot.
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//              K=16) into one of two TMEM accumulators and commits the slot
+//              back to the producer when its MMAs retire.
+//   warps 2-5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//              32·(w%4) …), round, store rows of C; then release the
+//              accumulator so the next tile's MMAs overlap this epilogue.
+// Rows of padding (position ≥ the sequence's length) are not stored, and
+// 128-row tiles with no valid row are skipped by every role alike.
+// Every mbarrier wait is bounded; on a timeout the kernel raises a flag in the
+// workspace status word, drains what it issued and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace r2l {
+
+// True if rows [r0, r1) of a right-padded [B, L] batch contain a valid row.
+__device__ __forceinline__ bool rows_have_valid(const int* __restrict__ len, int L, long long r0,
+                                                long long r1) {
+  long long b = r0 / L;
+  long long start = b * L;
+  while (start < r1) {
+    const long long lo = r0 > start ? r0 : start;
+    if ((int)(lo - start) < len[b]) return true;
+    ++b;
+    start += L;
+  }
+  return false;
+}
+
+template <int BN>
+struct TcGemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;                       // 128 bytes of bf16: one swizzle row
+  static constexpr int STAGES = BN >= 256 ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (size_t)STAGE_BYTES + 256 /*barriers*/;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128 is a multiple of 16 up to 256");
+  static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte swizzle-atom alignment");
+};
+
+template <typename TOut>
+__device__ __forceinline__ void store_row32(TOut* dst, const float (&v)[32]);
+
+template <>
+__device__ __forceinline__ void store_row32<bf16>(bf16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(v[q * 8 + 2 * j], v[q * 8 + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <>
+__device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// C2 (optional): columns n < c2_cols are also written, rounded to bf16, into
+// C2[m, n] (row stride ldc2).  x_proj uses it to hand Δr to dt_proj in bf16.
+template <int BN, typename TOut>
+__global__ void __launch_bounds__(192, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               TOut* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols,
+               int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err) {
+  using Cfg = TcGemmCfg<BN>;
+  constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_k = (K + BK - 1) / BK;
+  const long long total = (long long)num_m * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(&tfull[a], 1);
+      sm100::mbar_init(&tempty[a], 128);
+    }
+    sm100::mbar_init(drain, 1);
+    sm100::fence_barrier_init();
+    sm100::prefetch_tmap(&tmA);
+    sm100::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) sm100::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto tile_live = [&](long long t) -> bool {
+    if (!len) return true;
+    const long long r0 = (t / num_n) * BM;
+    const long long r1 = r0 + BM < M ? r0 + BM : M;
+    return rows_have_valid(len, L, r0, r1);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!tile_live(t)) continue;
+        const int mb = (int)(t / num_n), nb = (int)(t % num_n);
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, err)) { ok = false; break; }
+          sm100::mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          sm100::tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
+          sm100::tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+          ++issued[stage];
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {  // drain the loads still in flight before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) sm100::mbar_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u, nullptr, 1000000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!tile_live(t)) continue;
+        if (!sm100::mbar_wait(&tempty[acc], aphase ^ 1u, err)) { ok = false; break; }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!sm100::mbar_wait(&full[stage], phase, err)) { ok = false; break; }
+          sm100::tc_fence_after();
+          const uint32_t a0 = sm100::smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b0 = sm100::smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            sm100::mma_bf16(d_tmem, sm100::smem_desc_k128(a0 + k * 32), sm100::smem_desc_k128(b0 + k * 32),
+                            idesc, (kb | k) != 0);
+          sm100::mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        sm100::mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1u;
+      }
+      // all MMAs issued by this thread have retired once `drain` completes
+      sm100::mma_commit(drain);
+      sm100::mbar_wait(drain, 0, err, 1000000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t aphase = 0;
+    for (long long t = blockIdx.x; t < total; t += gridDim.x) {
+      if (!tile_live(t)) continue;
+      if (!sm100::mbar_wait(&tfull[acc], aphase, err)) break;
+      sm100::tc_fence_after();
+      const int mb = (int)(t / num_n), nb = (int)(t % num_n);
+      const long long row = (long long)mb * BM + q * 32 + lane;
+      const bool row_ok = row < M && (!len || row_valid(len, L, row));
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), v);
+        const int col = nb * BN + c0;
+        if (row_ok && col < N) {
+          TOut* dst = C + row * (long long)ldc + col;
+          if (col + 32 <= N) {
+            store_row32<TOut>(dst, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < N - col) dst[j] = from_f32<TOut>(v[j]);
+          }
+          if (C2 && col < c2_cols) {
+            bf16* d2 = C2 + row * (long long)ldc2 + col;
+            if (col + 32 <= c2_cols) {
+              store_row32<bf16>(d2, v);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < c2_cols - col) d2[j] = __float2bfloat16_rn(v[j]);
+            }
+          }
+        }
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) aphase ^= 1u;
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 1) sm100::tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+}  // namespace r2l

@@ -14,6 +14,9 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "scan_simple.cuh"
+#include "tc_gemm.h"
+
+#include <type_traits>
 
 using r2l::bf16;
 
@@ -25,7 +28,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Byte offsets of the workspace regions for a [B, L] batch.
 struct Plan {
-  size_t status, len, xz, u, dbc, dt, y, o, total;
+  size_t status, len, xz, u, dbc, dr, dt, y, o, total;
   long long M;
   int E, d, R, N, ldd;
   size_t act;
@@ -49,6 +52,7 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->xz = off;     off = align_up(off + M * 2 * p->E * p->act, kAlign);
   p->u = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->dbc = off;    off = align_up(off + M * p->ldd * sizeof(float), kAlign);
+  p->dr = off;     off = align_up(off + M * p->R * 2, kAlign);   // Δr in bf16 (tensor-core path)
   p->dt = off;     off = align_up(off + M * p->E * p->act, kAlign);
   p->y = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->o = off;      off = align_up(off + M * p->d * p->act, kAlign);
@@ -76,6 +80,9 @@ r2l_status check_call(void* hidden, const r2l_dims* dm, int B, int L, void* ws, 
   if (!hidden || !dm) return R2L_ERR_INVALID_ARG;
   if (!make_plan(dm, B, L, plan)) return R2L_ERR_INVALID_ARG;
   if (dm->d_state != 16 || dm->d_conv != 4) return R2L_ERR_UNSUPPORTED;
+  // bf16 path: TMA needs 16-byte row strides for every GEMM operand
+  if (dm->dtype == R2L_BF16 && ((dm->d_model % 8) || (dm->d_inner % 8) || (dm->dt_rank % 8)))
+    return R2L_ERR_UNSUPPORTED;
   // grid limits of the launches below
   if (L > 65535 || B > 65535 || (plan->M + 63) / 64 > 65535) return R2L_ERR_UNSUPPORTED;
   if (!aligned16(hidden)) return R2L_ERR_ALIGNMENT;
@@ -127,6 +134,24 @@ r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, c
     if (_s != R2L_OK) return _s;       \
   } while (0)
 
+// One projection y = x Wᵀ: tensor cores (tcgen05) for bf16, SIMT fp32 otherwise.
+// c2 (bf16 path only): columns < c2_cols also stored in bf16 (Δr for dt_proj).
+template <typename T, typename TC>
+r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long long M, int N, int K,
+                const int* len, int L, unsigned* err, cudaStream_t st, bf16* c2 = nullptr, int ldc2 = 0,
+                int c2_cols = 0) {
+  if constexpr (std::is_same<T, bf16>::value) {
+    r2l::TcGemm g{};
+    g.A = A; g.lda = lda; g.B = W; g.ldb = ldw; g.C = C; g.ldc = ldc;
+    g.c_fp32 = std::is_same<TC, float>::value;
+    g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols;
+    g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
+    return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
+  } else {
+    return gemm(A, lda, W, ldw, C, ldc, M, N, K, len, L, st);
+  }
+}
+
 template <typename T>
 r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, int B, int L,
                      char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof) {
@@ -141,12 +166,15 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   T* dt = (T*)(ws + p.dt);
   T* y = (T*)(ws + p.y);
   T* o = (T*)(ws + p.o);
+  bf16* dr = (bf16*)(ws + p.dr);
+  unsigned* err = (unsigned*)(ws + p.status);
   const size_t es = sizeof(T);
+  constexpr bool kTC = std::is_same<T, bf16>::value;
 
   // a1: [x | z] = h · W_inᵀ
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
   prof->launches++;
-  R2L_TRY(gemm(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, st));
+  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
   // a2: u = SiLU(anti-causal conv(x))
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
   prof->launches++;
@@ -158,11 +186,14 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a3: [Δr | B | C] = u · W_xᵀ  (fp32 out)
   R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
   prof->launches++;
-  R2L_TRY(gemm(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, st));
+  R2L_TRY(proj(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, err, st, dr, R, R));
   // a4: dt_raw = Δr · W_dtᵀ  (bias + softplus applied in the scan)
   R2L_TRY(prof->mark(R2L_STAGE_DT_PROJ, st));
   prof->launches++;
-  R2L_TRY(gemm((const float*)dbc, p.ldd, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, st));
+  if constexpr (kTC)
+    R2L_TRY(proj((const T*)dr, R, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, err, st));
+  else
+    R2L_TRY(gemm((const float*)dbc, p.ldd, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, st));
   // a5: reverse selective scan, y = (C·H + D u) · SiLU(z)
   R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
   prof->launches++;
@@ -175,7 +206,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a6: o = y · W_outᵀ
   R2L_TRY(prof->mark(R2L_STAGE_OUT_PROJ, st));
   prof->launches++;
-  R2L_TRY(gemm(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, st));
+  R2L_TRY(proj(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, err, st));
 
   if (dbg) {
     const size_t rowsE = (size_t)M;

@@ -123,7 +123,7 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
   __syncthreads();
   float t = lane < 8 ? red[lane] : 0.0f;
 #pragma unroll
-  for (int o = 4; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);  // every lane gets the total
   return t;
 }
 

@@ -2,8 +2,13 @@
 ABI and through the CPU oracle, and the tolerance measures the tests use.
 
 Tolerances (the layer's contract):
-  fp32 path: max_i |a_i − b_i| / max(|b_i|, 1e-3·rms(b))  ≤ 1e-4
-  bf16 path: max |a − b| / max |b|                         ≤ 2e-2
+  fp32 path, output h⁺:               max_i |a_i − b_i| / max(|b_i|, 1e-3·rms(b))  ≤ 1e-4
+  fp32 path, ĥ and intermediates:     max |a − b| / max |b|                         ≤ 1e-4
+  bf16 path, everything:              max |a − b| / max |b|                         ≤ 2e-2
+The per-element form is used only where it is well conditioned (h⁺ is
+dominated by h ~ N(0, 1)); GEMM outputs and the LayerNorm output have
+elements near zero by cancellation, where a per-element ratio measures
+nothing but fp32 rounding of the cancelled terms.
 """
 from __future__ import annotations
 
@@ -37,7 +42,13 @@ def err_bf16(a, b) -> float:
 
 
 def err_for(dtype):
+    """Metric for the final output h⁺."""
     return err_fp32 if dtype == torch.float32 else err_bf16
+
+
+def err_norm(a, b) -> float:
+    """max |a − b| / max |b| (intermediates, ĥ)."""
+    return err_bf16(a, b)
 
 
 def tol_for(dtype):

@@ -41,7 +41,7 @@ def _check_inter(case, dbg, inter, b, keys=("u", "y", "o", "hhat")):
     for k in keys:
         g = S.to_f64(dbg[k][b * L: b * L + n])
         w = inter[b][k]
-        e = G.err_for(case.dtype)(g, w)
+        e = G.err_norm(g, w)
         errs[k] = e
         assert e <= G.tol_for(case.dtype), f"{case.name} intermediate {k} b={b}: err {e:.3e}"
     return errs
@@ -64,8 +64,8 @@ def test_cfg0_fp32_against_oracle():
     case = S.make_case(0)
     got, dbg, _ = G.run_gpu(case, debug=True)
     want, inter = G.run_oracle(case, [0], intermediates=True)
-    _check_seq(case, got, want, 0, "h+")
     _check_inter(case, dbg, inter, 0, keys=("x", "z", "u", "y", "o", "hhat"))
+    _check_seq(case, got, want, 0, "h+")
 
 
 def test_cfg0_s_zero_is_bitwise_identity():
@@ -81,8 +81,8 @@ def test_cfg0_scan_visible_fp32():
                                    ln="seeded")]
     got, dbg, _ = G.run_gpu(case, debug=True)
     want, inter = G.run_oracle(case, [0], intermediates=True)
-    _check_seq(case, got, want, 0, "h+")
     _check_inter(case, dbg, inter, 0, keys=("u", "y", "o", "hhat"))
+    _check_seq(case, got, want, 0, "h+")
 
 
 def test_fp32_ragged_tails_and_empty():
@@ -107,8 +107,8 @@ def test_cfg1_bf16_against_oracle():
     case = S.make_case(1)
     got, dbg, _ = G.run_gpu(case, debug=True)
     want, inter = G.run_oracle(case, [0], intermediates=True)
-    _check_seq(case, got, want, 0, "h+")
     _check_inter(case, dbg, inter, 0, keys=("x", "z", "u", "y", "o", "hhat"))
+    _check_seq(case, got, want, 0, "h+")
 
 
 def test_bf16_scan_visible_ragged():
@@ -121,8 +121,8 @@ def test_bf16_scan_visible_ragged():
     got, dbg, _ = G.run_gpu(case, debug=True)
     want, inter = G.run_oracle(case, [0, 1], intermediates=True)
     for b in (0, 1):
-        _check_seq(case, got, want, b, "h+")
         _check_inter(case, dbg, inter, b, keys=("u", "y", "o", "hhat"))
+        _check_seq(case, got, want, b, "h+")
     _padding_untouched(case, got)
 
 
@@ -136,8 +136,8 @@ def test_bf16_general_A_and_no_ln():
                                    ln="none", A_log=A_log)]
     got, dbg, _ = G.run_gpu(case, debug=True)
     want, inter = G.run_oracle(case, [0], intermediates=True)
-    _check_seq(case, got, want, 0, "h+")
     _check_inter(case, dbg, inter, 0, keys=("y", "o", "hhat"))
+    _check_seq(case, got, want, 0, "h+")
 
 
 def test_bf16_forced_general_path_matches():
