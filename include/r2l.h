@@ -185,6 +185,35 @@ R2L_API r2l_status r2l_sidecar_forward_profiled(void *hidden, const r2l_weights 
                                         size_t workspace_bytes, void *stream,
                                         void *const *events, int n_events, int *launches);
 
+/* Bytes of device workspace r2l_reverse_scan needs for a [B, L] batch split
+ * into chunks of chunk_tokens tokens (0 = automatic).  0 for invalid input. */
+R2L_API size_t r2l_reverse_scan_workspace_size(const r2l_dims *dims, int B, int L, int chunk_tokens);
+
+/* The selective scan of §3.4 step ❷ on its own (the Mamba-1 scan, run from
+ * each sequence's last valid token to its first) followed by the SiLU(z) gate:
+ *
+ *     Δ_i = softplus(dt_raw_i + dt_b);  H_i = exp(Δ_i ⊗ A) ⊙ H_{i+1} + (Δ_i ⊙ u_i) ⊗ B_i;
+ *     y_i = (H_i·C_i + D ⊙ u_i) ⊙ SiLU(z_i),   H entering position len_b − 1 is 0.
+ *
+ *   u        act  [B·L, E]     (row stride E)
+ *   z        act  [B·L, ldz]   first E columns are z
+ *   dt_raw   act  [B·L, E]     Δr·W_dtᵀ, before bias and softplus
+ *   bc       fp32 [B·L, ldbc]  B in columns 0..15, C in columns 16..31
+ *   A_log    fp32 [E, 16],  D, dt_b  fp32 [E]
+ *   y        act  [B·L, E]     output; rows i ≥ len_b are not written
+ *   lengths  as for r2l_sidecar_forward
+ *   chunk_tokens  bf16 path: tokens per chunk when sequences are split for
+ *            parallelism (rounded up to a multiple of 16; 0 = automatic).
+ *            Ignored by the fp32 path, which scans each sequence whole.
+ *   workspace  ≥ r2l_reverse_scan_workspace_size(dims, B, L, chunk_tokens) bytes,
+ *            16-byte aligned (chunk carries and the device status word).
+ * Device pointers, 16-byte aligned; ldz a multiple of 8 and ldbc of 4.        */
+R2L_API r2l_status r2l_reverse_scan(const void *u, const void *z, int ldz, const void *dt_raw,
+                                    const float *bc, int ldbc, const float *A_log, const float *D,
+                                    const float *dt_b, void *y, const r2l_dims *dims, int B, int L,
+                                    const int32_t *lengths, int chunk_tokens, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
 /* Synchronises `stream`, then reads the device status word that the last
  * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*
  * bits.  Returns R2L_ERR_DEVICE_CHECK if any bit is set, R2L_ERR_CUDA if the

@@ -25,7 +25,7 @@ STATUS = {0: "R2L_OK", 1: "R2L_ERR_INVALID_ARG", 2: "R2L_ERR_UNSUPPORTED", 3: "R
 
 EXPORTS = ("r2l_abi_version", "r2l_status_string", "r2l_workspace_size", "r2l_sidecar_forward",
            "r2l_sidecar_forward_debug", "r2l_sidecar_forward_profiled", "r2l_sidecar_stack",
-           "r2l_get_device_status")
+           "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan")
 
 STAGES = ("in_proj", "conv", "x_proj", "dt_proj", "scan", "out_proj", "ln_residual")
 
@@ -86,6 +86,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.r2l_sidecar_stack.restype = ci
     lib.r2l_sidecar_stack.argtypes = [vp, ctypes.POINTER(Weights), ctypes.POINTER(cf), ci,
                                       ctypes.POINTER(Dims), ci, ci, vp, vp, ctypes.c_size_t, vp]
+    lib.r2l_reverse_scan_workspace_size.restype = ctypes.c_size_t
+    lib.r2l_reverse_scan_workspace_size.argtypes = [ctypes.POINTER(Dims), ci, ci, ci]
+    lib.r2l_reverse_scan.restype = ci
+    lib.r2l_reverse_scan.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, ctypes.POINTER(Dims), ci, ci, vp,
+                                     ci, vp, ctypes.c_size_t, vp]
     lib.r2l_get_device_status.restype = ci
     lib.r2l_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -210,6 +215,28 @@ def sidecar_stack(hidden: torch.Tensor, weights_list: Sequence, dims: Dims, s_li
                                _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     if check and st != 0:
         raise R2LError(st, "r2l_sidecar_stack")
+    return st
+
+
+def reverse_scan_workspace_size(dims: Dims, B: int, L: int, chunk_tokens: int = 0) -> int:
+    return int(load().r2l_reverse_scan_workspace_size(ctypes.byref(dims), B, L, chunk_tokens))
+
+
+def reverse_scan(u: torch.Tensor, z: torch.Tensor, dt_raw: torch.Tensor, bc: torch.Tensor,
+                 A_log: torch.Tensor, D: torch.Tensor, dt_b: torch.Tensor, y: torch.Tensor, dims: Dims,
+                 B: int, L: int, lengths=None, chunk_tokens: int = 0,
+                 workspace: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """r2l_reverse_scan.  u, dt_raw, y: [B·L, E]; z: [B·L, ldz] (first E columns);
+    bc: [B·L, ldbc] fp32 with B in columns 0..15 and C in 16..31."""
+    lib = load()
+    if workspace is None:
+        n = reverse_scan_workspace_size(dims, B, L, chunk_tokens)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=u.device)
+    st = lib.r2l_reverse_scan(_ptr(u), _ptr(z), z.stride(0), _ptr(dt_raw), _ptr(bc), bc.stride(0), _ptr(A_log),
+                              _ptr(D), _ptr(dt_b), _ptr(y), ctypes.byref(dims), B, L, _ptr(lengths),
+                              chunk_tokens, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if check and st != 0:
+        raise R2LError(st, "r2l_reverse_scan")
     return st
 
 

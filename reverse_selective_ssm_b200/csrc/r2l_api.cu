@@ -15,6 +15,8 @@
 #include "simt_kernels.cuh"
 #include "scan_simple.cuh"
 #include "tc_gemm.h"
+#include "scan_fast.h"
+#include "conv_fast.cuh"
 
 #include <type_traits>
 
@@ -28,10 +30,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Byte offsets of the workspace regions for a [B, L] batch.
 struct Plan {
-  size_t status, len, xz, u, dbc, dr, dt, y, o, total;
+  size_t status, len, xz, u, dbc, dr, dt, y, o, carry, total;
+  int chunk_tokens;  // scan chunk length (bf16 path)
   long long M;
   int E, d, R, N, ldd;
   size_t act;
+  unsigned flags;
 };
 
 bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
@@ -45,6 +49,7 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->N = dm->d_state;
   p->ldd = p->R + 2 * p->N;
   p->act = dm->dtype == R2L_BF16 ? 2 : 4;
+  p->flags = dm->flags;
   const size_t M = (size_t)p->M;
   size_t off = 0;
   p->status = off; off = align_up(off + 16, kAlign);
@@ -56,6 +61,9 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->dt = off;     off = align_up(off + M * p->E * p->act, kAlign);
   p->y = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->o = off;      off = align_up(off + M * p->d * p->act, kAlign);
+  p->chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, p->E, 0);
+  p->carry = off;
+  if (dm->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, p->E, p->chunk_tokens), kAlign);
   p->total = off;
   return true;
 }
@@ -178,7 +186,12 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a2: u = SiLU(anti-causal conv(x))
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
   prof->launches++;
-  {
+  if constexpr (kTC) {
+    namespace cv = r2l::conv;
+    dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
+    cv::conv_silu_bf16_kernel<<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+    R2L_LAUNCH_CHECK();
+  } else {
     dim3 grid((E + 127) / 128, L, B);
     r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
     R2L_LAUNCH_CHECK();
@@ -197,7 +210,23 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a5: reverse selective scan, y = (C·H + D u) · SiLU(z)
   R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
   prof->launches++;
-  {
+  if constexpr (kTC) {
+    r2l::ScanArgs sa{};
+    sa.u = u; sa.ldu = E;
+    sa.z = xz + E; sa.ldz = 2 * E;
+    sa.dt = dt; sa.ldt = E;
+    sa.bc = dbc + R; sa.ldbc = p.ldd;
+    sa.A_log = w->A_log; sa.D = w->D; sa.dt_b = w->dt_proj_b;
+    sa.y = y; sa.ldy = E;
+    sa.B = B; sa.L = L; sa.E = E; sa.len = len;
+    sa.chunk_tokens = p.chunk_tokens;
+    sa.carry = (float*)(ws + p.carry);
+    sa.err = err;
+    sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
+    int nl = 0;
+    if (r2l::scan_bf16(sa, st, &nl) != cudaSuccess) return R2L_ERR_CUDA;
+    prof->launches += nl - 1;
+  } else {
     dim3 grid((E + 127) / 128, B);
     r2l::scan_simple_kernel<T><<<grid, 128, 0, st>>>(u, xz + E, 2 * E, dt, dbc, p.ldd, R, w->A_log,
                                                      w->D, w->dt_proj_b, y, E, len, L);
@@ -327,6 +356,65 @@ r2l_status r2l_sidecar_stack(void* hidden, const r2l_weights* weights, const flo
       R2L_TRY(run_layer<bf16>((bf16*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
     else
       R2L_TRY(run_layer<float>((float*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
+  }
+  return R2L_OK;
+}
+
+size_t r2l_reverse_scan_workspace_size(const r2l_dims* dims, int B, int L, int chunk_tokens) {
+  if (!dims || B <= 0 || L <= 0 || dims->d_inner <= 0) return 0;
+  if (dims->dtype != R2L_BF16 && dims->dtype != R2L_FP32) return 0;
+  size_t off = align_up(16, kAlign);
+  off = align_up(off + sizeof(int) * (size_t)B, kAlign);
+  if (dims->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, dims->d_inner, chunk_tokens), kAlign);
+  return off;
+}
+
+r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* dt_raw, const float* bc,
+                            int ldbc, const float* A_log, const float* D, const float* dt_b, void* y,
+                            const r2l_dims* dims, int B, int L, const int32_t* lengths, int chunk_tokens,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!u || !z || !dt_raw || !bc || !A_log || !D || !dt_b || !y || !dims) return R2L_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || dims->d_inner <= 0) return R2L_ERR_INVALID_ARG;
+  if (dims->dtype != R2L_BF16 && dims->dtype != R2L_FP32) return R2L_ERR_INVALID_ARG;
+  if (dims->d_state != 16) return R2L_ERR_UNSUPPORTED;
+  const int E = dims->d_inner;
+  if (ldz < E || ldbc < 32) return R2L_ERR_INVALID_ARG;
+  if (L > 65535 || B > 65535) return R2L_ERR_UNSUPPORTED;
+  for (const void* q : {u, z, dt_raw, (const void*)bc, (const void*)A_log, (const void*)D, (const void*)dt_b, (const void*)y})
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  if (dims->dtype == R2L_BF16 && ((ldz % 8) || (E % 8) || (ldbc % 4))) return R2L_ERR_ALIGNMENT;
+  if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
+  const size_t need = r2l_reverse_scan_workspace_size(dims, B, L, chunk_tokens);
+  if (!workspace || workspace_bytes < need) return R2L_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return R2L_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  unsigned* status = (unsigned*)ws;
+  int* len = (int*)(ws + align_up(16, kAlign));
+  float* carry = (float*)(ws + align_up(align_up(16, kAlign) + sizeof(int) * (size_t)B, kAlign));
+  if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
+  r2l::prep_lengths_kernel<<<(B + 127) / 128, 128, 0, st>>>(lengths, len, B, L, status);
+  R2L_LAUNCH_CHECK();
+  if (dims->dtype == R2L_BF16) {
+    r2l::ScanArgs sa{};
+    sa.u = (const bf16*)u; sa.ldu = E;
+    sa.z = (const bf16*)z; sa.ldz = ldz;
+    sa.dt = (const bf16*)dt_raw; sa.ldt = E;
+    sa.bc = bc; sa.ldbc = ldbc;
+    sa.A_log = A_log; sa.D = D; sa.dt_b = dt_b;
+    sa.y = (bf16*)y; sa.ldy = E;
+    sa.B = B; sa.L = L; sa.E = E; sa.len = len;
+    sa.chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, E, chunk_tokens);
+    sa.carry = carry;
+    sa.err = status;
+    sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
+    if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
+  } else {
+    dim3 grid((E + 127) / 128, B);
+    r2l::scan_simple_kernel<float><<<grid, 128, 0, st>>>((const float*)u, (const float*)z, ldz,
+                                                         (const float*)dt_raw, bc, ldbc, 0, A_log, D, dt_b,
+                                                         (float*)y, E, len, L);
+    R2L_LAUNCH_CHECK();
   }
   return R2L_OK;
 }

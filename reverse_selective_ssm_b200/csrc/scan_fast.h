@@ -1,0 +1,37 @@
+// Host interface of the bf16 reverse selective scan (scan_fast.cuh).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+
+namespace r2l {
+
+struct ScanArgs {
+  const __nv_bfloat16* u;   long long ldu;    // [B·L, E]
+  const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz)
+  const __nv_bfloat16* dt;  long long ldt;    // dt_raw [B·L, E] (before bias and softplus)
+  const float* bc;          long long ldbc;   // [B·L, 32]: B in columns 0..15, C in 16..31
+  const float* A_log;                          // [E, 16]
+  const float* D;                              // [E]
+  const float* dt_b;                           // [E]
+  __nv_bfloat16* y;         long long ldy;    // [B·L, E]
+  int B, L, E;
+  const int* len;                              // device [B], clamped to [0, L]
+  int chunk_tokens;                            // tokens per chunk (resolved, > 0)
+  float* carry;                                // scan_carry_bytes() of device scratch (may be null if 1 chunk)
+  unsigned* err;                               // device status word
+  int force_general;                           // never use the A = -(1..16) power path
+};
+
+// Tokens per chunk chosen from the shape alone (deterministic, no device query).
+int scan_auto_chunk_tokens(int B, int L, int E);
+// Chunk length actually used for a request (0 = automatic), a multiple of 16.
+int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens);
+// Bytes of carry scratch the scan needs for this shape and chunk length.
+size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens);
+// Enqueue the scan (1 or 3 launches).  Returns the number of kernels launched
+// through *launches when not null.
+cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches);
+
+}  // namespace r2l

@@ -1,0 +1,94 @@
+// Host launcher of the bf16 reverse selective scan: chunk choice, TMA
+// descriptors for the u / z / dt_raw / B|C tiles, and the launch sequence.
+#include <cuda.h>
+
+#include "scan_fast.cuh"
+#include "scan_fast.h"
+#include "tmap.h"
+
+namespace r2l {
+
+int scan_auto_chunk_tokens(int B, int L, int E) {
+  using namespace rscan;
+  // Compute warps with one chunk per sequence; below ~6 per SM of a 148-SM
+  // part the sequence is split so that about 24 per SM are in flight.
+  const long long warps1 = (long long)B * ((E + CH - 1) / CH) * CWARPS;
+  const long long target = 148LL * 24;
+  const int whole = (L + TS - 1) / TS * TS;
+  if (warps1 >= 148LL * 6) return whole;
+  long long nc = (target + warps1 - 1) / warps1;
+  long long T = (L + nc - 1) / nc;
+  T = (T + TS - 1) / TS * TS;
+  if (T < 4 * TS) T = 4 * TS;
+  return (int)(T < whole ? T : whole);
+}
+
+int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens) {
+  using namespace rscan;
+  if (chunk_tokens <= 0) return scan_auto_chunk_tokens(B, L, E);
+  const int T = (chunk_tokens + TS - 1) / TS * TS;
+  const int whole = (L + TS - 1) / TS * TS;
+  return T < whole ? T : whole;
+}
+
+size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
+  const int T = scan_resolve_chunk_tokens(B, L, E, chunk_tokens);
+  const long long nc = (L + T - 1) / T;
+  if (nc <= 1) return 0;
+  return (size_t)B * nc * E * 17 * sizeof(float);
+}
+
+cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
+  using namespace rscan;
+  if (launches) *launches = 0;
+  const long long M = (long long)a.B * a.L;
+  if (M <= 0 || a.E <= 0) return cudaSuccess;
+  const int T = a.chunk_tokens;
+  if (T <= 0 || T % TS) return cudaErrorInvalidValue;
+  const int nc = (a.L + T - 1) / T;
+  if (nc > 1 && !a.carry) return cudaErrorInvalidValue;
+
+  CUtensorMap tu, tz, tdt, tbc;
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CH, TS, false) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CH, TS, false) ||
+      !make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, CH, TS, false) ||
+      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, false))
+    return cudaErrorInvalidValue;
+
+  Params p;
+  p.A_log = a.A_log;
+  p.D = a.D;
+  p.dt_b = a.dt_b;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.E = a.E;
+  p.L = a.L;
+  p.T = T;
+  p.nc = nc;
+  p.len = a.len;
+  p.carry = a.carry;
+  p.carry_sum = a.carry ? a.carry + (size_t)a.B * nc * a.E * 16 : nullptr;
+  p.err = a.err;
+  p.force_general = a.force_general;
+
+  cudaError_t e;
+  e = cudaFuncSetAttribute(chunk_scan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
+  if (nc > 1) {
+    e = cudaFuncSetAttribute(chunk_scan_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    chunk_scan_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (launches) *launches += 2;
+  }
+  chunk_scan_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, p);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaSuccess;
+}
+
+}  // namespace r2l

@@ -1,43 +1,13 @@
 // Host launcher of the tcgen05 GEMM (gemm_tc.cuh): TMA descriptor encoding,
 // tile-width choice and the persistent launch (one CTA per SM).
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include "gemm_tc.cuh"
 #include "tc_gemm.h"
+#include "tmap.h"
 
 namespace r2l {
 namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  // Resolved once per process through the runtime, so the library needs no
-  // link-time dependency on libcuda.  The pointer never changes afterwards.
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
-  return fn;
-}
-
-// Row-major bf16 matrix [rows, inner] with row stride `ld` elements, read in
-// boxes of 64 (inner) × box_rows with 128-byte swizzle; out-of-range elements
-// read as zero.
-bool make_tmap(CUtensorMap* m, const void* base, int inner, long long rows, int ld, int box_rows) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-  cuuint32_t es[2] = {1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 int sm_count() {
   int dev = 0, n = 148;
@@ -49,8 +19,8 @@ template <int BN, typename TOut>
 cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   using Cfg = TcGemmCfg<BN>;
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, g.A, g.K, g.M, g.lda, Cfg::BM)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tb, g.B, g.K, g.N, g.ldb, BN)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, true)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, true)) return cudaErrorInvalidValue;
   auto kern = gemm_tc_kernel<BN, TOut>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
