@@ -214,6 +214,37 @@ R2L_API r2l_status r2l_reverse_scan(const void *u, const void *z, int ldz, const
                                     const int32_t *lengths, int chunk_tokens, void *workspace,
                                     size_t workspace_bytes, void *stream);
 
+/* Capacity, in bytes, of the scratch array behind r2l_reverse_scan_noalloc. */
+#define R2L_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* r2l_reverse_scan without a workspace argument, for callers that cannot
+ * allocate device memory while they run: for example a serving runtime that
+ * reserves all device memory when it starts and forbids allocation while it
+ * handles requests, or a plug-in whose host program owns the CUDA context and
+ * its allocator.  It computes exactly what r2l_reverse_scan computes.  (The
+ * paper has no counterpart; this entry point exists for such callers only.)
+ *
+ * Its scratch (status word, clamped lengths, chunk carries) is a fixed array
+ * of R2L_NOALLOC_SCRATCH_BYTES that the library's device code declares; every
+ * device that loads the library holds it until the process exits.  The entry
+ * point calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (each call rewrites what it reads).  Calls whose work overlaps on the
+ *     GPU (for instance on two streams) race on it; order them.
+ *   - A request that needs more scratch than the array holds
+ *     (r2l_reverse_scan_workspace_size() > R2L_NOALLOC_SCRATCH_BYTES) returns
+ *     R2L_ERR_WORKSPACE and enqueues nothing.  A smaller chunk count (larger
+ *     chunk_tokens) needs less scratch; one chunk per sequence needs almost none.
+ * r2l_get_device_status cannot read this scratch; use r2l_reverse_scan when
+ * device-side flags matter.  Other arguments and errors as r2l_reverse_scan. */
+R2L_API r2l_status r2l_reverse_scan_noalloc(const void *u, const void *z, int ldz, const void *dt_raw,
+                                            const float *bc, int ldbc, const float *A_log, const float *D,
+                                            const float *dt_b, void *y, const r2l_dims *dims, int B, int L,
+                                            const int32_t *lengths, int chunk_tokens, void *stream);
+
 /* Synchronises `stream`, then reads the device status word that the last
  * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*
  * bits.  Returns R2L_ERR_DEVICE_CHECK if any bit is set, R2L_ERR_CUDA if the

@@ -25,7 +25,10 @@ STATUS = {0: "R2L_OK", 1: "R2L_ERR_INVALID_ARG", 2: "R2L_ERR_UNSUPPORTED", 3: "R
 
 EXPORTS = ("r2l_abi_version", "r2l_status_string", "r2l_workspace_size", "r2l_sidecar_forward",
            "r2l_sidecar_forward_debug", "r2l_sidecar_forward_profiled", "r2l_sidecar_stack",
-           "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan")
+           "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan",
+           "r2l_reverse_scan_noalloc")
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 STAGES = ("in_proj", "conv", "x_proj", "dt_proj", "scan", "out_proj", "ln_residual")
 
@@ -91,6 +94,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.r2l_reverse_scan.restype = ci
     lib.r2l_reverse_scan.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, ctypes.POINTER(Dims), ci, ci, vp,
                                      ci, vp, ctypes.c_size_t, vp]
+    lib.r2l_reverse_scan_noalloc.restype = ci
+    lib.r2l_reverse_scan_noalloc.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, ctypes.POINTER(Dims), ci,
+                                             ci, vp, ci, vp]
     lib.r2l_get_device_status.restype = ci
     lib.r2l_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -237,6 +243,21 @@ def reverse_scan(u: torch.Tensor, z: torch.Tensor, dt_raw: torch.Tensor, bc: tor
                               chunk_tokens, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     if check and st != 0:
         raise R2LError(st, "r2l_reverse_scan")
+    return st
+
+
+def reverse_scan_noalloc(u: torch.Tensor, z: torch.Tensor, dt_raw: torch.Tensor, bc: torch.Tensor,
+                         A_log: torch.Tensor, D: torch.Tensor, dt_b: torch.Tensor, y: torch.Tensor, dims: Dims,
+                         B: int, L: int, lengths=None, chunk_tokens: int = 0, stream=None,
+                         check: bool = True) -> int:
+    """r2l_reverse_scan_noalloc: as :func:`reverse_scan`, with the library's
+    static device scratch instead of a caller workspace (nothing is allocated)."""
+    lib = load()
+    st = lib.r2l_reverse_scan_noalloc(_ptr(u), _ptr(z), z.stride(0), _ptr(dt_raw), _ptr(bc), bc.stride(0),
+                                      _ptr(A_log), _ptr(D), _ptr(dt_b), _ptr(y), ctypes.byref(dims), B, L,
+                                      _ptr(lengths), chunk_tokens, _stream_ptr(stream))
+    if check and st != 0:
+        raise R2LError(st, "r2l_reverse_scan_noalloc")
     return st
 
 
