@@ -70,7 +70,11 @@ typedef enum {
 } r2l_dtype;
 
 /* r2l_dims.flags */
-#define R2L_FLAG_GENERAL_A 0x1u   /* never take the A = -(1..16) power fast path of the scan */
+#define R2L_FLAG_GENERAL_A 0x1u     /* never take the A = -(1..16) power fast path of the scan  */
+#define R2L_FLAG_SCAN_SPLIT1 0x2u    /* scan layout: one thread per channel (bf16 path)           */
+#define R2L_FLAG_SCAN_SPLIT2 0x4u    /* scan layout: two threads per channel, 8 states each       */
+/* Neither SCAN_SPLIT flag set: the library picks the layout from the shape.
+ * Every layout computes the same function; they differ only in speed.       */
 
 /* Device status bits, reported by r2l_get_device_status(). */
 #define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */

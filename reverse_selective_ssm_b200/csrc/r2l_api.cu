@@ -223,6 +223,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.carry = (float*)(ws + p.carry);
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
+    sa.split = (p.flags & R2L_FLAG_SCAN_SPLIT2) ? 2 : (p.flags & R2L_FLAG_SCAN_SPLIT1) ? 1 : 0;
     int nl = 0;
     if (r2l::scan_bf16(sa, st, &nl) != cudaSuccess) return R2L_ERR_CUDA;
     prof->launches += nl - 1;
@@ -408,6 +409,7 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
     sa.carry = carry;
     sa.err = status;
     sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
+    sa.split = (dims->flags & R2L_FLAG_SCAN_SPLIT2) ? 2 : (dims->flags & R2L_FLAG_SCAN_SPLIT1) ? 1 : 0;
     if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
   } else {
     dim3 grid((E + 127) / 128, B);

@@ -7,12 +7,16 @@
 //   H_i = exp(Δ_i A) ⊙ H_{i+1} + Δ_i u_i B_i          (H entering the last token = 0)
 //   y_i = (⟨C_i, H_i⟩ + D u_i) · SiLU(z_i)
 //
-// Work split: a CTA owns 128 channels of one sequence over one chunk of
-// tokens; each of its 4 compute warps holds 32 channels, one channel per
-// thread, with the 16-entry state in registers (packed f32x2 arithmetic).  A
-// fifth warp streams [16 tokens × 128 channels] tiles of u, z, dt_raw and the
-// [16 tokens × 32] tile of B|C into a 4-deep shared-memory ring with TMA,
-// from the chunk's right end to its left end.
+// Work split: a CTA owns CH channels of one sequence over one chunk of tokens
+// with 4 compute warps; SPLIT = 1 gives one thread per channel (CH = 128) and
+// SPLIT = 2 two threads per channel that hold 8 of the 16 states each
+// (CH = 64), doubling the threads in flight.  State lives in registers and is
+// updated with packed f32x2 arithmetic.  A fifth warp streams
+// [16 tokens × CH channels] tiles of u, z, dt_raw and the [16 tokens × 32]
+// tile of B|C into a 4-deep shared-memory ring with TMA, from the chunk's right
+// end to its left end, and writes each finished y tile back with a TMA store
+// (tiles that cross the chunk's left edge are stored row by row by the compute
+// threads instead, so no row outside the chunk is ever written).
 //
 // When a sequence is split into several chunks (to give the GPU enough
 // independent work), three launches cooperate through a small carry buffer:
@@ -27,7 +31,8 @@
 // Decays: exp(Δ A_m) is exp2(Δ · A_m log2 e) on the MUFU unit.  When every
 // channel of a warp has A_m = −(m+1) (the S4D-real initialisation, checked on
 // the device to 1e-5 relative), the 16 decays are the powers r, r², …, r¹⁶ of
-// r = exp(−Δ): one exponential and 15 multiplications per (token, channel).
+// r = exp(−Δ) = 1 / (1 + e^v) for v = dt_raw + dt_b (since Δ = softplus(v)):
+// one reciprocal and a depth-4 product tree per (token, channel).
 #pragma once
 
 #include <cuda.h>
@@ -38,17 +43,24 @@
 namespace r2l {
 namespace rscan {
 
-constexpr int CH = 128;       // channels per CTA
 constexpr int TS = 16;        // tokens per pipeline stage
 constexpr int STAGES = 4;
 constexpr int CWARPS = 4;     // compute warps
-constexpr int THREADS = (CWARPS + 1) * 32;
+constexpr int CTHREADS = CWARPS * 32;
+constexpr int THREADS = CTHREADS + 32;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-constexpr uint32_t TILE_ACT_BYTES = TS * CH * 2;   // one bf16 tile
-constexpr uint32_t TILE_BC_BYTES = TS * 32 * 4;    // one B|C tile
-constexpr size_t SMEM_BYTES = 128 + STAGES * (3 * TILE_ACT_BYTES + TILE_BC_BYTES) + 2 * STAGES * 8;
+template <int SPLIT>
+struct Geo {
+  static constexpr int CH = CTHREADS / SPLIT;        // channels per CTA
+  static constexpr int NQ = 8 / SPLIT;               // state pairs per thread
+  static constexpr int SUB = 8 / SPLIT;              // tokens per phase-A / phase-B sub-tile
+  static constexpr uint32_t ACT_TILE = TS * CH * 2;  // one bf16 [TS × CH] tile
+  static constexpr uint32_t BC_TILE = TS * 32 * 4;   // one fp32 [TS × 32] tile
+  // per stage: u, dt, z, y tiles and the B|C tile
+  static constexpr size_t SMEM_BYTES = 128 + STAGES * (4 * (size_t)ACT_TILE + BC_TILE) + 2 * STAGES * 8;
+};
 
 struct Params {
   const float* A_log;   // [E, 16]
@@ -76,16 +88,24 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
-// softplus(v) = log(1 + x), x = e^v; v itself above 20.  For x < 1/16 the
-// Taylor series of log(1 + x) to x⁵ (truncation < x⁶/6 < 3e-8 relative) avoids
-// the cancellation in 1 + x; above, log2(1 + x)·ln 2 (|log| > 0.06).
-__device__ __forceinline__ float softplus_fast(float v) {
+// Δ = softplus(v) = log(1 + x), x = e^v (v itself above 20), and r = e^{-Δ} =
+// 1 / (1 + x).  For x < 1/16 the Taylor series of log(1 + x) to x⁵
+// (truncation < x⁶/6 < 3e-8 relative) avoids the cancellation in 1 + x;
+// above, log2(1 + x)·ln 2 (|log| > 0.06).
+__device__ __forceinline__ void softplus_and_decay(float v, float& delta, float& r) {
   const float x = ex2_approx(v * LOG2E);
+  const float w = 1.0f + x;
   const float series = x * (1.0f - x * (0.5f - x * (1.0f / 3.0f - x * (0.25f - x * 0.2f))));
-  const float direct = lg2_approx(1.0f + x) * LN2;
-  const float r = x < 0.0625f ? series : direct;
-  return v > 20.0f ? v : r;
+  const float direct = lg2_approx(w) * LN2;
+  const float sp = x < 0.0625f ? series : direct;
+  delta = v > 20.0f ? v : sp;
+  r = rcp_approx(w);
 }
 
 // SiLU(z) = z / (1 + e^{-z})
@@ -93,33 +113,35 @@ __device__ __forceinline__ float silu_fast(float z) {
   return __fdividef(z, 1.0f + ex2_approx(-z * LOG2E));
 }
 
-// Per-thread constants of one channel for scan_tile.
-struct TileCtx {
+// Per-thread constants.
+template <int SPLIT>
+struct Ctx {
   float dtb, Dc;
-  float A2[16];        // A_m · log2 e
-  bf16* y;             // y + channel
-  long long ldy;
-  bool cvalid;
+  float A2[16 / SPLIT];  // this thread's A_m · log2 e
+  int h;                 // which half of the states (SPLIT = 2)
 };
 
 // One sub-tile of SUB tokens [j0, j0 + SUB) of one channel, last token first.
-// Phase A computes everything that does not depend on the state for all of
-// its tokens (softplus, the decay base, Δu, D·u, SiLU(z)); phase B runs the
-// recurrence.  FULL: every token of the sub-tile is inside the chunk.
-constexpr int SUB = 8;
-
-template <bool FINAL, bool POW, bool FULL>
-__device__ __forceinline__ void scan_sub(const TileCtx& cx, float2 (&H)[8], float& sumd, const bf16* su,
-                                         const bf16* sdt, const bf16* sz, const float* sbc, long long row0,
-                                         int j0, int jmin) {
+// Phase A computes what does not depend on the state (softplus, the decay
+// base, Δu, D·u, SiLU(z)) for all of its tokens; phase B runs the recurrence.
+// FULL: every token of the sub-tile is inside the chunk.  Output: y rows to
+// shared memory (ys, stride CH) for tiles stored by TMA, else to global (yg).
+template <bool FINAL, int SPLIT, bool POW, bool FULL>
+__device__ __forceinline__ void scan_sub(const Ctx<SPLIT>& cx, float2 (&H)[8 / SPLIT], float& sumd,
+                                         const bf16* su, const bf16* sdt, const bf16* sz, const float* sbc,
+                                         bf16* ys, bf16* yg, long long ldy, bool store_ok, int j0, int jmin) {
+  constexpr int CH = Geo<SPLIT>::CH;
+  constexpr int NQ = Geo<SPLIT>::NQ;
+  constexpr int SUB = Geo<SPLIT>::SUB;
   float dec[SUB], du[SUB], gz[SUB], Du[SUB];
 #pragma unroll
   for (int t = 0; t < SUB; ++t) {
     const int j = j0 + t;
     if (!FULL && j < jmin) continue;
-    const float delta = softplus_fast(__bfloat162float(sdt[j * CH]) + cx.dtb);
+    float delta, r;
+    softplus_and_decay(__bfloat162float(sdt[j * CH]) + cx.dtb, delta, r);
     const float uu = __bfloat162float(su[j * CH]);
-    dec[t] = POW ? ex2_approx(-delta * LOG2E) : delta;
+    dec[t] = POW ? r : delta;
     du[t] = delta * uu;
     if (FINAL) {
       Du[t] = cx.Dc * uu;
@@ -134,92 +156,104 @@ __device__ __forceinline__ void scan_sub(const TileCtx& cx, float2 (&H)[8], floa
     if (!FULL && j < jmin) break;
     const float4* bc4 = reinterpret_cast<const float4*>(sbc + j * 32);
     const float2 du2 = make_float2(du[t], du[t]);
-    float2 a[8];
+    float2 a[NQ];
     if (POW) {
-      // r^1 … r^16 by a depth-4 product tree
+      // r^1 … r^8 by a product tree; SPLIT = 2, second half: times r^8
       const float r = dec[t];
       const float r2 = r * r;
-      a[0] = make_float2(r, r2);
-      a[1] = __fmul2_rn(a[0], make_float2(r2, r2));          // r3 r4
-      const float r4 = a[1].y;
-      a[2] = __fmul2_rn(a[0], make_float2(r4, r4));          // r5 r6
-      a[3] = __fmul2_rn(a[1], make_float2(r4, r4));          // r7 r8
-      const float r8 = a[3].y;
+      float2 pw[4];
+      pw[0] = make_float2(r, r2);
+      pw[1] = __fmul2_rn(pw[0], make_float2(r2, r2));          // r3 r4
+      const float r4 = pw[1].y;
+      pw[2] = __fmul2_rn(pw[0], make_float2(r4, r4));          // r5 r6
+      pw[3] = __fmul2_rn(pw[1], make_float2(r4, r4));          // r7 r8
+      const float r8 = pw[3].y;
+      if (SPLIT == 1) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) a[4 + q] = __fmul2_rn(a[q], make_float2(r8, r8));   // r9 … r16
+        for (int q = 0; q < 4; ++q) {
+          a[q] = pw[q];
+          a[4 + q] = __fmul2_rn(pw[q], make_float2(r8, r8));   // r9 … r16
+        }
+      } else {
+        const float m = cx.h ? r8 : 1.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[q] = __fmul2_rn(pw[q], make_float2(m, m));
+      }
     } else {
       const float delta = dec[t];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < NQ; ++q)
         a[q] = make_float2(ex2_approx(delta * cx.A2[2 * q]), ex2_approx(delta * cx.A2[2 * q + 1]));
     }
+    const int qb = SPLIT == 1 ? 0 : 2 * cx.h;    // first float4 of this thread's B (and C) half
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 Bq = bc4[q];
+    for (int q = 0; q < NQ / 2; ++q) {
+      const float4 Bq = bc4[qb + q];
       H[2 * q] = __ffma2_rn(a[2 * q], H[2 * q], __fmul2_rn(du2, make_float2(Bq.x, Bq.y)));
       H[2 * q + 1] = __ffma2_rn(a[2 * q + 1], H[2 * q + 1], __fmul2_rn(du2, make_float2(Bq.z, Bq.w)));
     }
     if (FINAL) {
       float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 Cq = bc4[4 + q];
+      for (int q = 0; q < NQ / 2; ++q) {
+        const float4 Cq = bc4[4 + qb + q];
         acc0 = __ffma2_rn(make_float2(Cq.x, Cq.y), H[2 * q], acc0);
         acc1 = __ffma2_rn(make_float2(Cq.z, Cq.w), H[2 * q + 1], acc1);
       }
-      const float yv = ((acc0.x + acc0.y) + (acc1.x + acc1.y) + Du[t]) * gz[t];
-      if (cx.cvalid) cx.y[(row0 + j) * cx.ldy] = __float2bfloat16_rn(yv);
+      float s = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      if (SPLIT == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);
+      const bf16 yv = __float2bfloat16_rn((s + Du[t]) * gz[t]);
+      if (store_ok) {
+        if (ys) ys[j * CH] = yv;
+        else yg[(long long)j * ldy] = yv;
+      }
     }
   }
 }
 
-// One [TS tokens] tile, last token first: its two sub-tiles, upper one first.
-template <bool FINAL, bool POW, bool FULL>
-__device__ __forceinline__ void scan_tile(const TileCtx& cx, float2 (&H)[8], float& sumd, const bf16* su,
-                                          const bf16* sdt, const bf16* sz, const float* sbc, long long row0,
-                                          int jmin) {
-#pragma unroll
-  for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
-    if (!FULL && j0 + SUB <= jmin) break;
-    scan_sub<FINAL, POW, FULL>(cx, H, sumd, su, sdt, sz, sbc, row0, j0, jmin);
-  }
-}
-
-template <bool FINAL>
-__global__ void __launch_bounds__(THREADS)
+template <bool FINAL, int SPLIT>
+__global__ void __launch_bounds__(THREADS, SPLIT == 2 ? 4 : 2)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap tm_y, const Params p) {
+  using Gm = Geo<SPLIT>;
+  constexpr int CH = Gm::CH;
+  constexpr int NQ = Gm::NQ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   bf16* s_u = reinterpret_cast<bf16*>(smem);
   bf16* s_dt = s_u + STAGES * TS * CH;
   bf16* s_z = s_dt + STAGES * TS * CH;
-  float* s_bc = reinterpret_cast<float*>(s_z + STAGES * TS * CH);
+  bf16* s_y = s_z + STAGES * TS * CH;
+  float* s_bc = reinterpret_cast<float*>(s_y + STAGES * TS * CH);
   uint64_t* full = reinterpret_cast<uint64_t*>(s_bc + STAGES * TS * 32);
   uint64_t* empty = full + STAGES;
 
   const int cb = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wc = warp * 32 + lane;        // channel within the block
-  const int c = cb * CH + wc;             // channel
-  const bool cvalid = warp < CWARPS && c < p.E;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const bool compute = tid < CTHREADS;
+  const int ch = compute ? tid / SPLIT : 0;    // channel within the block
+  const int h = SPLIT == 2 ? (tid & 1) : 0;     // state half (SPLIT = 2)
+  const int c = cb * CH + ch;
+  const bool cvalid = compute && c < p.E;
   const int n = p.len[b];
   const int s0 = k * p.T;
   const int e0 = min(s0 + p.T, n);
+  const int m0 = h * (16 / SPLIT);              // first state this thread holds
 
   if (s0 >= n) {  // chunk entirely in the padding: nothing to read or write
     if (!FINAL && cvalid) {
-      float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
+      float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
+      for (int q = 0; q < NQ / 2; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (h == 0) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
     }
     return;
   }
   const int ntiles = (e0 - s0 + TS - 1) / TS;
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       sm100::mbar_init(&full[s], 1);
       sm100::mbar_init(&empty[s], CWARPS);
@@ -228,28 +262,43 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   }
   __syncthreads();
 
-  if (warp == CWARPS) {
+  if (!compute) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       sm100::prefetch_tmap(&tm_u);
       sm100::prefetch_tmap(&tm_dt);
       sm100::prefetch_tmap(&tm_bc);
-      if (FINAL) sm100::prefetch_tmap(&tm_z);
-      constexpr uint32_t bytes = (FINAL ? 3 : 2) * TILE_ACT_BYTES + TILE_BC_BYTES;
+      if (FINAL) {
+        sm100::prefetch_tmap(&tm_z);
+        sm100::prefetch_tmap(&tm_y);
+      }
+      constexpr uint32_t bytes = (FINAL ? 3 : 2) * Gm::ACT_TILE + Gm::BC_TILE;
       int issued = 0;
       bool ok = true;
-      for (int it = 0; it < ntiles; ++it) {
+      const int iters = ntiles + (FINAL ? STAGES : 0);
+      for (int it = 0; it < iters; ++it) {
         const int st = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         if (!sm100::mbar_wait(&empty[st], ph ^ 1u, p.err)) { ok = false; break; }
-        const int row0 = b * p.L + e0 - (it + 1) * TS;   // may be negative for b = 0: reads zeros
-        sm100::mbar_arrive_expect_tx(&full[st], bytes);
-        sm100::tma_load_2d(s_u + st * TS * CH, &tm_u, cb * CH, row0, &full[st]);
-        sm100::tma_load_2d(s_dt + st * TS * CH, &tm_dt, cb * CH, row0, &full[st]);
-        if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, &tm_z, cb * CH, row0, &full[st]);
-        sm100::tma_load_2d(s_bc + st * TS * 32, &tm_bc, 0, row0, &full[st]);
-        ++issued;
+        if (FINAL && it >= STAGES) {
+          const int tb = e0 - (it - STAGES + 1) * TS;     // first position of the tile just finished
+          if (tb >= s0) {                                 // whole tile inside the chunk: y sits in s_y
+            sm100::tma_store_2d(&tm_y, s_y + st * TS * CH, cb * CH, b * p.L + tb);
+            sm100::bulk_commit();
+            sm100::bulk_wait_read_all();                  // s_y[st] is rewritten STAGES tiles later
+          }
+        }
+        if (it < ntiles) {
+          const int row0 = b * p.L + e0 - (it + 1) * TS;  // may be negative for b = 0: reads zeros
+          sm100::mbar_arrive_expect_tx(&full[st], bytes);
+          sm100::tma_load_2d(s_u + st * TS * CH, &tm_u, cb * CH, row0, &full[st]);
+          sm100::tma_load_2d(s_dt + st * TS * CH, &tm_dt, cb * CH, row0, &full[st]);
+          if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, &tm_z, cb * CH, row0, &full[st]);
+          sm100::tma_load_2d(s_bc + st * TS * 32, &tm_bc, 0, row0, &full[st]);
+          ++issued;
+        }
       }
+      if (FINAL) sm100::bulk_wait_all();
       if (!ok) {  // drain loads still in flight before the CTA can exit
         for (int it = issued - 1; it >= 0 && it >= issued - STAGES; --it)
           sm100::mbar_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u, nullptr, 1000000000ull);
@@ -259,43 +308,34 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   }
 
   // -------------------------------------------------------------- compute warps
-  float dtb = 0.0f, Dc = 0.0f;
-  float A2[16];
+  Ctx<SPLIT> cx;
+  cx.h = h;
+  cx.dtb = cvalid ? p.dt_b[c] : 0.0f;
+  cx.Dc = cvalid ? p.D[c] : 0.0f;
   bool pow_ok = true;
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const float a = cvalid ? -expf(p.A_log[c * 16 + m]) : -(float)(m + 1);
-    A2[m] = a * LOG2E;
-    pow_ok = pow_ok && fabsf(a + (float)(m + 1)) <= 1e-5f * (float)(m + 1);
-  }
-  if (cvalid) {
-    dtb = p.dt_b[c];
-    Dc = p.D[c];
+  for (int m = 0; m < 16 / SPLIT; ++m) {
+    const float a = cvalid ? -expf(p.A_log[c * 16 + m0 + m]) : -(float)(m0 + m + 1);
+    cx.A2[m] = a * LOG2E;
+    pow_ok = pow_ok && fabsf(a + (float)(m0 + m + 1)) <= 1e-5f * (float)(m0 + m + 1);
   }
   const bool use_pow = !p.force_general && __all_sync(0xffffffffu, pow_ok);
 
-  float2 H[8];
+  float2 H[NQ];
   if (FINAL && p.nc > 1 && cvalid) {
-    const float4* src = reinterpret_cast<const float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
+    const float4* src = reinterpret_cast<const float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < NQ / 2; ++q) {
       const float4 v = src[q];
       H[2 * q] = make_float2(v.x, v.y);
       H[2 * q + 1] = make_float2(v.z, v.w);
     }
   } else {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) H[q] = make_float2(0.0f, 0.0f);
+    for (int q = 0; q < NQ; ++q) H[q] = make_float2(0.0f, 0.0f);
   }
   float sumd = 0.0f;
-  TileCtx ctx;
-  ctx.dtb = dtb;
-  ctx.Dc = Dc;
-#pragma unroll
-  for (int m = 0; m < 16; ++m) ctx.A2[m] = A2[m];
-  ctx.y = p.y + c;
-  ctx.ldy = p.ldy;
-  ctx.cvalid = cvalid;
+  const bool writer = cvalid && h == 0;
 
   for (int it = 0; it < ntiles; ++it) {
     const int st = it % STAGES;
@@ -303,27 +343,35 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
     if (!sm100::mbar_wait(&full[st], ph, p.err)) break;
     const int tbase = e0 - (it + 1) * TS;        // sequence position of tile row 0
     const int jmin = s0 > tbase ? s0 - tbase : 0;
-    const long long row0 = (long long)b * p.L + tbase;
-    const bf16* su = s_u + st * TS * CH + wc;
-    const bf16* sdt = s_dt + st * TS * CH + wc;
-    const bf16* sz = s_z + st * TS * CH + wc;
+    const bf16* su = s_u + st * TS * CH + ch;
+    const bf16* sdt = s_dt + st * TS * CH + ch;
+    const bf16* sz = s_z + st * TS * CH + ch;
     const float* sbc = s_bc + st * TS * 32;
-    if (use_pow) {
-      if (jmin == 0) scan_tile<FINAL, true, true>(ctx, H, sumd, su, sdt, sz, sbc, row0, 0);
-      else scan_tile<FINAL, true, false>(ctx, H, sumd, su, sdt, sz, sbc, row0, jmin);
-    } else {
-      if (jmin == 0) scan_tile<FINAL, false, true>(ctx, H, sumd, su, sdt, sz, sbc, row0, 0);
-      else scan_tile<FINAL, false, false>(ctx, H, sumd, su, sdt, sz, sbc, row0, jmin);
+    // full tiles go out through shared memory and a TMA store; a tile that
+    // crosses the chunk's left edge is written row by row
+    bf16* ys = jmin == 0 ? s_y + st * TS * CH + ch : nullptr;
+    bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
+    constexpr int SUB = Gm::SUB;
+#pragma unroll
+    for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
+      if (jmin == 0) {
+        if (use_pow) scan_sub<FINAL, SPLIT, true, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, 0);
+        else scan_sub<FINAL, SPLIT, false, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, 0);
+      } else if (j0 + SUB > jmin) {
+        if (use_pow) scan_sub<FINAL, SPLIT, true, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, jmin);
+        else scan_sub<FINAL, SPLIT, false, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, jmin);
+      }
     }
+    if (FINAL && ys) sm100::fence_proxy_async_smem();   // make the y tile visible to the TMA store
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[st]);
   }
 
   if (!FINAL && cvalid) {
-    float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
+    float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
-    p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
+    for (int q = 0; q < NQ / 2; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
+    if (h == 0) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
   }
 }
 

@@ -12,7 +12,7 @@ int scan_auto_chunk_tokens(int B, int L, int E) {
   using namespace rscan;
   // Compute warps with one chunk per sequence; below ~6 per SM of a 148-SM
   // part the sequence is split so that about 24 per SM are in flight.
-  const long long warps1 = (long long)B * ((E + CH - 1) / CH) * CWARPS;
+  const long long warps1 = (long long)B * ((E + CTHREADS - 1) / CTHREADS) * CWARPS;
   const long long target = 148LL * 24;
   const int whole = (L + TS - 1) / TS * TS;
   if (warps1 >= 148LL * 6) return whole;
@@ -38,6 +38,49 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
   return (size_t)B * nc * E * 17 * sizeof(float);
 }
 
+int scan_resolve_split(int B, int L, int E, int request) {
+  if (request == 1 || request == 2) return request;
+  (void)B; (void)L; (void)E;
+  return 1;
+}
+
+namespace {
+
+template <int SPLIT>
+cudaError_t launch_split(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
+  using namespace rscan;
+  using Gm = Geo<SPLIT>;
+  const long long M = (long long)a.B * a.L;
+  CUtensorMap tu, tz, tdt, tbc, ty;
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, Gm::CH, TS, false) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, Gm::CH, TS, false) ||
+      !make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, Gm::CH, TS, false) ||
+      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, false) ||
+      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, Gm::CH, TS, false))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  e = cudaFuncSetAttribute(chunk_scan_kernel<true, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Gm::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.E + Gm::CH - 1) / Gm::CH, nc, a.B);
+  if (nc > 1) {
+    e = cudaFuncSetAttribute(chunk_scan_kernel<false, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Gm::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    chunk_scan_kernel<false, SPLIT><<<grid, THREADS, Gm::SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (launches) *launches += 2;
+  }
+  chunk_scan_kernel<true, SPLIT><<<grid, THREADS, Gm::SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   using namespace rscan;
   if (launches) *launches = 0;
@@ -47,13 +90,6 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   if (T <= 0 || T % TS) return cudaErrorInvalidValue;
   const int nc = (a.L + T - 1) / T;
   if (nc > 1 && !a.carry) return cudaErrorInvalidValue;
-
-  CUtensorMap tu, tz, tdt, tbc;
-  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CH, TS, false) ||
-      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CH, TS, false) ||
-      !make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, CH, TS, false) ||
-      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, false))
-    return cudaErrorInvalidValue;
 
   Params p;
   p.A_log = a.A_log;
@@ -70,25 +106,8 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.carry_sum = a.carry ? a.carry + (size_t)a.B * nc * a.E * 16 : nullptr;
   p.err = a.err;
   p.force_general = a.force_general;
-
-  cudaError_t e;
-  e = cudaFuncSetAttribute(chunk_scan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
-  if (nc > 1) {
-    e = cudaFuncSetAttribute(chunk_scan_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    chunk_scan_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, p);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-    if (launches) *launches += 2;
-  }
-  chunk_scan_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, p);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  if (launches) *launches += 1;
-  return cudaSuccess;
+  if (scan_resolve_split(a.B, a.L, a.E, a.split) == 2) return launch_split<2>(a, p, nc, st, launches);
+  return launch_split<1>(a, p, nc, st, launches);
 }
 
 }  // namespace r2l
