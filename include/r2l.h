@@ -71,11 +71,6 @@ typedef enum {
 
 /* r2l_dims.flags */
 #define R2L_FLAG_GENERAL_A 0x1u     /* never take the A = -(1..16) power fast path of the scan  */
-#define R2L_FLAG_SCAN_SPLIT1 0x2u    /* scan layout: one thread per channel (bf16 path)           */
-#define R2L_FLAG_SCAN_SPLIT2 0x4u    /* scan layout: two threads per channel, 8 states each       */
-/* Neither SCAN_SPLIT flag set: the library picks the layout from the shape.
- * Every layout computes the same function; they differ only in speed.       */
-
 /* Device status bits, reported by r2l_get_device_status(). */
 #define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */
 #define R2L_DEVFLAG_TIMEOUT 0x2u          /* a kernel gave up waiting on a pipeline barrier (results invalid) */
@@ -111,7 +106,9 @@ typedef struct {
  * unspecified values, except in hhat where they are not written.             */
 typedef struct {
   void  *x;        /* act  [B·L, E]      in_proj, first half                  */
-  void  *z;        /* act  [B·L, E]      in_proj, second half                 */
+  void  *z;        /* act  [B·L, E]      in_proj, second half; the bf16 path
+                                           stores SiLU(z) here (its in_proj
+                                           epilogue applies the gate activation) */
   void  *u;        /* act  [B·L, E]      conv + SiLU                          */
   float *dbc;      /* fp32 [B·L, R+2N]   x_proj output Δr | B | C             */
   void  *y;        /* act  [B·L, E]      scan output after the SiLU(z) gate   */

@@ -85,10 +85,12 @@ __device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[
 
 // C2 (optional): columns n < c2_cols are also written, rounded to bf16, into
 // C2[m, n] (row stride ldc2).  x_proj uses it to hand Δr to dt_proj in bf16.
+// silu_from_col >= 0: columns n >= silu_from_col are stored as SiLU(C[m, n])
+// (in_proj applies the Mamba-1 gate activation to its z half here).
 template <int BN, typename TOut>
 __global__ void __launch_bounds__(192, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               TOut* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols,
+               TOut* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols, int silu_from_col,
                int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err) {
   using Cfg = TcGemmCfg<BN>;
   constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES;
@@ -215,6 +217,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         float v[32];
         sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), v);
         const int col = nb * BN + c0;
+        if (silu_from_col >= 0 && col + 32 > silu_from_col) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col + j >= silu_from_col) v[j] = __fdividef(v[j], 1.0f + __expf(-v[j]));
+        }
         if (row_ok && col < N) {
           TOut* dst = C + row * (long long)ldc + col;
           if (col + 32 <= N) {

@@ -70,6 +70,7 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+
 r2l_status check_weights(const r2l_weights* w) {
   if (!w) return R2L_ERR_INVALID_ARG;
   const void* ptrs[] = {w->in_proj_w, w->conv_w, w->conv_b, w->x_proj_w, w->dt_proj_w,
@@ -147,16 +148,43 @@ r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, c
 template <typename T, typename TC>
 r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long long M, int N, int K,
                 const int* len, int L, unsigned* err, cudaStream_t st, bf16* c2 = nullptr, int ldc2 = 0,
-                int c2_cols = 0) {
+                int c2_cols = 0, int silu_from_col = -1) {
   if constexpr (std::is_same<T, bf16>::value) {
     r2l::TcGemm g{};
     g.A = A; g.lda = lda; g.B = W; g.ldb = ldw; g.C = C; g.ldc = ldc;
     g.c_fp32 = std::is_same<TC, float>::value;
-    g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols;
+    g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols; g.silu_from_col = silu_from_col;
     g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
     return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
   } else {
     return gemm(A, lda, W, ldw, C, ldc, M, N, K, len, L, st);
+  }
+}
+
+// LayerNorm + gated residual for bf16 rows of d <= 2048 (nv = ceil(d / 256)).
+template <int NV>
+r2l_status ln_bf16_nv(bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o, const float* lw,
+                      const float* lb, float g, int d, const int* len, int L, long long M, float* hhat) {
+  if (has_ln)
+    r2l::ln_residual_bf16_kernel<NV, true><<<blocks, 128, 0, st>>>(h, o, lw, lb, g, d, len, L, M, hhat);
+  else
+    r2l::ln_residual_bf16_kernel<NV, false><<<blocks, 128, 0, st>>>(h, o, lw, lb, g, d, len, L, M, hhat);
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+r2l_status launch_ln_bf16(int nv, bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o,
+                          const float* lw, const float* lb, float g, int d, const int* len, int L, long long M,
+                          float* hhat) {
+  switch (nv) {
+    case 1: return ln_bf16_nv<1>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 2: return ln_bf16_nv<2>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 3: return ln_bf16_nv<3>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 4: return ln_bf16_nv<4>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 5: return ln_bf16_nv<5>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 6: return ln_bf16_nv<6>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 7: return ln_bf16_nv<7>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    default: return ln_bf16_nv<8>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
   }
 }
 
@@ -182,7 +210,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a1: [x | z] = h · W_inᵀ
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
   prof->launches++;
-  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
+  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st, nullptr, 0, 0,
+               /*silu_from_col=*/kTC ? E : -1));
   // a2: u = SiLU(anti-causal conv(x))
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
   prof->launches++;
@@ -223,7 +252,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.carry = (float*)(ws + p.carry);
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
-    sa.split = (p.flags & R2L_FLAG_SCAN_SPLIT2) ? 2 : (p.flags & R2L_FLAG_SCAN_SPLIT1) ? 1 : 0;
+    sa.gated = 1;   // the in_proj epilogue stored SiLU(z)
     int nl = 0;
     if (r2l::scan_bf16(sa, st, &nl) != cudaSuccess) return R2L_ERR_CUDA;
     prof->launches += nl - 1;
@@ -251,11 +280,18 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   float* hhat = dbg ? dbg->hhat : nullptr;
   R2L_TRY(prof->mark(R2L_STAGE_LN_RESIDUAL, st));
   prof->launches++;
-  if (w->ln_w)
+  if (kTC && d <= 2048) {
+    const unsigned blocks = (unsigned)((M + 3) / 4);
+    const int nv = (d + 255) / 256;
+    R2L_TRY(launch_ln_bf16(nv, w->ln_w != nullptr, blocks, st, (bf16*)hidden, (const bf16*)o, w->ln_w, w->ln_b,
+                           g, d, len, L, M, hhat));
+  } else if (w->ln_w) {
     r2l::ln_gate_residual_kernel<T, true><<<(unsigned)M, 256, 0, st>>>(hidden, o, w->ln_w, w->ln_b, g, d, len, L, hhat);
-  else
+    R2L_LAUNCH_CHECK();
+  } else {
     r2l::ln_gate_residual_kernel<T, false><<<(unsigned)M, 256, 0, st>>>(hidden, o, nullptr, nullptr, g, d, len, L, hhat);
-  R2L_LAUNCH_CHECK();
+    R2L_LAUNCH_CHECK();
+  }
   R2L_TRY(prof->mark(R2L_NUM_STAGES, st));
   return R2L_OK;
 }
@@ -409,7 +445,7 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
     sa.carry = carry;
     sa.err = status;
     sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
-    sa.split = (dims->flags & R2L_FLAG_SCAN_SPLIT2) ? 2 : (dims->flags & R2L_FLAG_SCAN_SPLIT1) ? 1 : 0;
+    sa.gated = 0;
     if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
   } else {
     dim3 grid((E + 127) / 128, B);

@@ -7,12 +7,11 @@
 //   H_i = exp(Δ_i A) ⊙ H_{i+1} + Δ_i u_i B_i          (H entering the last token = 0)
 //   y_i = (⟨C_i, H_i⟩ + D u_i) · SiLU(z_i)
 //
-// Work split: a CTA owns CH channels of one sequence over one chunk of tokens
-// with 4 compute warps; SPLIT = 1 gives one thread per channel (CH = 128) and
-// SPLIT = 2 two threads per channel that hold 8 of the 16 states each
-// (CH = 64), doubling the threads in flight.  State lives in registers and is
-// updated with packed f32x2 arithmetic.  A fifth warp streams
-// [16 tokens × CH channels] tiles of u, z, dt_raw and the [16 tokens × 32]
+// Work split: a CTA owns 128 channels of one sequence over one chunk of
+// tokens; each of its 4 compute warps holds 32 channels, one channel per
+// thread, with the 16-entry state in registers updated by packed f32x2
+// arithmetic.  A fifth warp streams [16 tokens × 128 channels] tiles of u,
+// z (or SiLU(z), see GATED), dt_raw and the [16 tokens × 32]
 // tile of B|C into a 4-deep shared-memory ring with TMA, from the chunk's right
 // end to its left end, and writes each finished y tile back with a TMA store
 // (tiles that cross the chunk's left edge are stored row by row by the compute
@@ -51,16 +50,12 @@ constexpr int THREADS = CTHREADS + 32;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-template <int SPLIT>
-struct Geo {
-  static constexpr int CH = CTHREADS / SPLIT;        // channels per CTA
-  static constexpr int NQ = 8 / SPLIT;               // state pairs per thread
-  static constexpr int SUB = 8 / SPLIT;              // tokens per phase-A / phase-B sub-tile
-  static constexpr uint32_t ACT_TILE = TS * CH * 2;  // one bf16 [TS × CH] tile
-  static constexpr uint32_t BC_TILE = TS * 32 * 4;   // one fp32 [TS × 32] tile
-  // per stage: u, dt, z, y tiles and the B|C tile
-  static constexpr size_t SMEM_BYTES = 128 + STAGES * (4 * (size_t)ACT_TILE + BC_TILE) + 2 * STAGES * 8;
-};
+constexpr int CH = CTHREADS;                      // channels per CTA
+constexpr int SUB = 8;                            // tokens per phase-A / phase-B sub-tile
+constexpr uint32_t ACT_TILE = TS * CH * 2;        // one bf16 [TS × CH] tile
+constexpr uint32_t BC_TILE = TS * 32 * 4;         // one fp32 [TS × 32] tile
+// per stage: u, dt, z, y tiles and the B|C tile
+constexpr size_t SMEM_BYTES = 128 + STAGES * (4 * (size_t)ACT_TILE + BC_TILE) + 2 * STAGES * 8;
 
 struct Params {
   const float* A_log;   // [E, 16]
@@ -113,26 +108,22 @@ __device__ __forceinline__ float silu_fast(float z) {
   return __fdividef(z, 1.0f + ex2_approx(-z * LOG2E));
 }
 
-// Per-thread constants.
-template <int SPLIT>
+// Per-thread constants of one channel.
 struct Ctx {
   float dtb, Dc;
-  float A2[16 / SPLIT];  // this thread's A_m · log2 e
-  int h;                 // which half of the states (SPLIT = 2)
+  float A2[16];          // A_m · log2 e
 };
 
 // One sub-tile of SUB tokens [j0, j0 + SUB) of one channel, last token first.
 // Phase A computes what does not depend on the state (softplus, the decay
-// base, Δu, D·u, SiLU(z)) for all of its tokens; phase B runs the recurrence.
-// FULL: every token of the sub-tile is inside the chunk.  Output: y rows to
-// shared memory (ys, stride CH) for tiles stored by TMA, else to global (yg).
-template <bool FINAL, int SPLIT, bool POW, bool FULL>
-__device__ __forceinline__ void scan_sub(const Ctx<SPLIT>& cx, float2 (&H)[8 / SPLIT], float& sumd,
-                                         const bf16* su, const bf16* sdt, const bf16* sz, const float* sbc,
-                                         bf16* ys, bf16* yg, long long ldy, bool store_ok, int j0, int jmin) {
-  constexpr int CH = Geo<SPLIT>::CH;
-  constexpr int NQ = Geo<SPLIT>::NQ;
-  constexpr int SUB = Geo<SPLIT>::SUB;
+// base, Δu, D·u, the gate) for all of its tokens; phase B runs the
+// recurrence.  FULL: every token of the sub-tile is inside the chunk.  GATED:
+// the z tile already holds SiLU(z).  Output: y rows to shared memory (ys,
+// stride CH) for tiles stored by TMA, else to global (yg).
+template <bool FINAL, bool GATED, bool POW, bool FULL>
+__device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& sumd, const bf16* su,
+                                         const bf16* sdt, const bf16* sz, const float* sbc, bf16* ys, bf16* yg,
+                                         long long ldy, bool store_ok, int j0, int jmin) {
   float dec[SUB], du[SUB], gz[SUB], Du[SUB];
 #pragma unroll
   for (int t = 0; t < SUB; ++t) {
@@ -145,7 +136,8 @@ __device__ __forceinline__ void scan_sub(const Ctx<SPLIT>& cx, float2 (&H)[8 / S
     du[t] = delta * uu;
     if (FINAL) {
       Du[t] = cx.Dc * uu;
-      gz[t] = silu_fast(__bfloat162float(sz[j * CH]));
+      const float zz = __bfloat162float(sz[j * CH]);
+      gz[t] = GATED ? zz : silu_fast(zz);
     } else {
       sumd += delta;
     }
@@ -156,52 +148,40 @@ __device__ __forceinline__ void scan_sub(const Ctx<SPLIT>& cx, float2 (&H)[8 / S
     if (!FULL && j < jmin) break;
     const float4* bc4 = reinterpret_cast<const float4*>(sbc + j * 32);
     const float2 du2 = make_float2(du[t], du[t]);
-    float2 a[NQ];
+    float2 a[8];
     if (POW) {
-      // r^1 … r^8 by a product tree; SPLIT = 2, second half: times r^8
+      // r^1 … r^16 by a depth-4 product tree
       const float r = dec[t];
       const float r2 = r * r;
-      float2 pw[4];
-      pw[0] = make_float2(r, r2);
-      pw[1] = __fmul2_rn(pw[0], make_float2(r2, r2));          // r3 r4
-      const float r4 = pw[1].y;
-      pw[2] = __fmul2_rn(pw[0], make_float2(r4, r4));          // r5 r6
-      pw[3] = __fmul2_rn(pw[1], make_float2(r4, r4));          // r7 r8
-      const float r8 = pw[3].y;
-      if (SPLIT == 1) {
+      a[0] = make_float2(r, r2);
+      a[1] = __fmul2_rn(a[0], make_float2(r2, r2));          // r3 r4
+      const float r4 = a[1].y;
+      a[2] = __fmul2_rn(a[0], make_float2(r4, r4));          // r5 r6
+      a[3] = __fmul2_rn(a[1], make_float2(r4, r4));          // r7 r8
+      const float r8 = a[3].y;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          a[q] = pw[q];
-          a[4 + q] = __fmul2_rn(pw[q], make_float2(r8, r8));   // r9 … r16
-        }
-      } else {
-        const float m = cx.h ? r8 : 1.0f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) a[q] = __fmul2_rn(pw[q], make_float2(m, m));
-      }
+      for (int q = 0; q < 4; ++q) a[4 + q] = __fmul2_rn(a[q], make_float2(r8, r8));   // r9 … r16
     } else {
       const float delta = dec[t];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q)
+      for (int q = 0; q < 8; ++q)
         a[q] = make_float2(ex2_approx(delta * cx.A2[2 * q]), ex2_approx(delta * cx.A2[2 * q + 1]));
     }
-    const int qb = SPLIT == 1 ? 0 : 2 * cx.h;    // first float4 of this thread's B (and C) half
 #pragma unroll
-    for (int q = 0; q < NQ / 2; ++q) {
-      const float4 Bq = bc4[qb + q];
+    for (int q = 0; q < 4; ++q) {
+      const float4 Bq = bc4[q];
       H[2 * q] = __ffma2_rn(a[2 * q], H[2 * q], __fmul2_rn(du2, make_float2(Bq.x, Bq.y)));
       H[2 * q + 1] = __ffma2_rn(a[2 * q + 1], H[2 * q + 1], __fmul2_rn(du2, make_float2(Bq.z, Bq.w)));
     }
     if (FINAL) {
       float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int q = 0; q < NQ / 2; ++q) {
-        const float4 Cq = bc4[4 + qb + q];
+      for (int q = 0; q < 4; ++q) {
+        const float4 Cq = bc4[4 + q];
         acc0 = __ffma2_rn(make_float2(Cq.x, Cq.y), H[2 * q], acc0);
         acc1 = __ffma2_rn(make_float2(Cq.z, Cq.w), H[2 * q + 1], acc1);
       }
-      float s = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-      if (SPLIT == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);
+      const float s = (acc0.x + acc0.y) + (acc1.x + acc1.y);
       const bf16 yv = __float2bfloat16_rn((s + Du[t]) * gz[t]);
       if (store_ok) {
         if (ys) ys[j * CH] = yv;
@@ -211,14 +191,60 @@ __device__ __forceinline__ void scan_sub(const Ctx<SPLIT>& cx, float2 (&H)[8 / S
   }
 }
 
-template <bool FINAL, int SPLIT>
-__global__ void __launch_bounds__(THREADS, SPLIT == 2 ? 4 : 2)
+// The TMA producer (one thread): streams the chunk's tiles right to left into
+// the STAGES-deep ring and, for the final scan, writes each finished y tile
+// that lies wholly inside the chunk back with a bulk tensor store.
+template <bool FINAL>
+__device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUtensorMap* tm_z,
+                                             const CUtensorMap* tm_dt, const CUtensorMap* tm_bc,
+                                             const CUtensorMap* tm_y, bf16* s_u, bf16* s_dt, bf16* s_z,
+                                             bf16* s_y, float* s_bc, uint64_t* full, uint64_t* empty, int b,
+                                             int cb, int s0, int e0, int ntiles, const Params& p) {
+  sm100::prefetch_tmap(tm_u);
+  sm100::prefetch_tmap(tm_dt);
+  sm100::prefetch_tmap(tm_bc);
+  if (FINAL) {
+    sm100::prefetch_tmap(tm_z);
+    sm100::prefetch_tmap(tm_y);
+  }
+  constexpr uint32_t bytes = (FINAL ? 3 : 2) * ACT_TILE + BC_TILE;
+  int issued = 0;
+  bool ok = true;
+  const int iters = ntiles + (FINAL ? STAGES : 0);
+  for (int it = 0; it < iters; ++it) {
+    const int st = it % STAGES;
+    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+    if (!sm100::mbar_wait(&empty[st], ph ^ 1u, p.err)) { ok = false; break; }
+    if (FINAL && it >= STAGES) {
+      const int tb = e0 - (it - STAGES + 1) * TS;     // first position of the tile just finished
+      if (tb >= s0) {                                 // whole tile inside the chunk: y sits in s_y
+        sm100::tma_store_2d(tm_y, s_y + st * TS * CH, cb * CH, b * p.L + tb);
+        sm100::bulk_commit();
+        sm100::bulk_wait_read_all();                  // s_y[st] is rewritten STAGES tiles later
+      }
+    }
+    if (it < ntiles) {
+      const int row0 = b * p.L + e0 - (it + 1) * TS;  // may be negative for b = 0: reads zeros
+      sm100::mbar_arrive_expect_tx(&full[st], bytes);
+      sm100::tma_load_2d(s_u + st * TS * CH, tm_u, cb * CH, row0, &full[st]);
+      sm100::tma_load_2d(s_dt + st * TS * CH, tm_dt, cb * CH, row0, &full[st]);
+      if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, tm_z, cb * CH, row0, &full[st]);
+      sm100::tma_load_2d(s_bc + st * TS * 32, tm_bc, 0, row0, &full[st]);
+      ++issued;
+    }
+  }
+  if (FINAL) sm100::bulk_wait_all();
+  if (!ok) {  // drain loads still in flight before the CTA can exit
+    for (int it = issued - 1; it >= 0 && it >= issued - STAGES; --it)
+      sm100::mbar_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u, nullptr, 1000000000ull);
+  }
+}
+
+template <bool FINAL, bool GATED>
+__global__ void __launch_bounds__(THREADS, 2)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
                   const __grid_constant__ CUtensorMap tm_y, const Params p) {
-  using Gm = Geo<SPLIT>;
-  constexpr int CH = Gm::CH;
-  constexpr int NQ = Gm::NQ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   bf16* s_u = reinterpret_cast<bf16*>(smem);
@@ -233,21 +259,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const bool compute = tid < CTHREADS;
-  const int ch = compute ? tid / SPLIT : 0;    // channel within the block
-  const int h = SPLIT == 2 ? (tid & 1) : 0;     // state half (SPLIT = 2)
+  const int ch = compute ? tid : 0;             // channel within the block
   const int c = cb * CH + ch;
   const bool cvalid = compute && c < p.E;
   const int n = p.len[b];
   const int s0 = k * p.T;
   const int e0 = min(s0 + p.T, n);
-  const int m0 = h * (16 / SPLIT);              // first state this thread holds
 
   if (s0 >= n) {  // chunk entirely in the padding: nothing to read or write
     if (!FINAL && cvalid) {
-      float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
+      float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
 #pragma unroll
-      for (int q = 0; q < NQ / 2; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (h == 0) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
+      for (int q = 0; q < 4; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
     }
     return;
   }
@@ -263,79 +287,39 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   __syncthreads();
 
   if (!compute) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      sm100::prefetch_tmap(&tm_u);
-      sm100::prefetch_tmap(&tm_dt);
-      sm100::prefetch_tmap(&tm_bc);
-      if (FINAL) {
-        sm100::prefetch_tmap(&tm_z);
-        sm100::prefetch_tmap(&tm_y);
-      }
-      constexpr uint32_t bytes = (FINAL ? 3 : 2) * Gm::ACT_TILE + Gm::BC_TILE;
-      int issued = 0;
-      bool ok = true;
-      const int iters = ntiles + (FINAL ? STAGES : 0);
-      for (int it = 0; it < iters; ++it) {
-        const int st = it % STAGES;
-        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!sm100::mbar_wait(&empty[st], ph ^ 1u, p.err)) { ok = false; break; }
-        if (FINAL && it >= STAGES) {
-          const int tb = e0 - (it - STAGES + 1) * TS;     // first position of the tile just finished
-          if (tb >= s0) {                                 // whole tile inside the chunk: y sits in s_y
-            sm100::tma_store_2d(&tm_y, s_y + st * TS * CH, cb * CH, b * p.L + tb);
-            sm100::bulk_commit();
-            sm100::bulk_wait_read_all();                  // s_y[st] is rewritten STAGES tiles later
-          }
-        }
-        if (it < ntiles) {
-          const int row0 = b * p.L + e0 - (it + 1) * TS;  // may be negative for b = 0: reads zeros
-          sm100::mbar_arrive_expect_tx(&full[st], bytes);
-          sm100::tma_load_2d(s_u + st * TS * CH, &tm_u, cb * CH, row0, &full[st]);
-          sm100::tma_load_2d(s_dt + st * TS * CH, &tm_dt, cb * CH, row0, &full[st]);
-          if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, &tm_z, cb * CH, row0, &full[st]);
-          sm100::tma_load_2d(s_bc + st * TS * 32, &tm_bc, 0, row0, &full[st]);
-          ++issued;
-        }
-      }
-      if (FINAL) sm100::bulk_wait_all();
-      if (!ok) {  // drain loads still in flight before the CTA can exit
-        for (int it = issued - 1; it >= 0 && it >= issued - STAGES; --it)
-          sm100::mbar_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u, nullptr, 1000000000ull);
-      }
-    }
+    if (lane == 0)
+      run_producer<FINAL>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, s_u, s_dt, s_z, s_y, s_bc, full, empty, b, cb, s0,
+                          e0, ntiles, p);
     return;
   }
 
   // -------------------------------------------------------------- compute warps
-  Ctx<SPLIT> cx;
-  cx.h = h;
+  Ctx cx;
   cx.dtb = cvalid ? p.dt_b[c] : 0.0f;
   cx.Dc = cvalid ? p.D[c] : 0.0f;
   bool pow_ok = true;
 #pragma unroll
-  for (int m = 0; m < 16 / SPLIT; ++m) {
-    const float a = cvalid ? -expf(p.A_log[c * 16 + m0 + m]) : -(float)(m0 + m + 1);
+  for (int m = 0; m < 16; ++m) {
+    const float a = cvalid ? -expf(p.A_log[c * 16 + m]) : -(float)(m + 1);
     cx.A2[m] = a * LOG2E;
-    pow_ok = pow_ok && fabsf(a + (float)(m0 + m + 1)) <= 1e-5f * (float)(m0 + m + 1);
+    pow_ok = pow_ok && fabsf(a + (float)(m + 1)) <= 1e-5f * (float)(m + 1);
   }
   const bool use_pow = !p.force_general && __all_sync(0xffffffffu, pow_ok);
 
-  float2 H[NQ];
+  float2 H[8];
   if (FINAL && p.nc > 1 && cvalid) {
-    const float4* src = reinterpret_cast<const float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
+    const float4* src = reinterpret_cast<const float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
 #pragma unroll
-    for (int q = 0; q < NQ / 2; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const float4 v = src[q];
       H[2 * q] = make_float2(v.x, v.y);
       H[2 * q + 1] = make_float2(v.z, v.w);
     }
   } else {
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) H[q] = make_float2(0.0f, 0.0f);
+    for (int q = 0; q < 8; ++q) H[q] = make_float2(0.0f, 0.0f);
   }
   float sumd = 0.0f;
-  const bool writer = cvalid && h == 0;
 
   for (int it = 0; it < ntiles; ++it) {
     const int st = it % STAGES;
@@ -351,15 +335,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
     // crosses the chunk's left edge is written row by row
     bf16* ys = jmin == 0 ? s_y + st * TS * CH + ch : nullptr;
     bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
-    constexpr int SUB = Gm::SUB;
 #pragma unroll
     for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
       if (jmin == 0) {
-        if (use_pow) scan_sub<FINAL, SPLIT, true, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, 0);
-        else scan_sub<FINAL, SPLIT, false, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, 0);
+        if (use_pow) scan_sub<FINAL, GATED, true, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+        else scan_sub<FINAL, GATED, false, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
       } else if (j0 + SUB > jmin) {
-        if (use_pow) scan_sub<FINAL, SPLIT, true, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, jmin);
-        else scan_sub<FINAL, SPLIT, false, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, writer, j0, jmin);
+        if (use_pow) scan_sub<FINAL, GATED, true, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+        else scan_sub<FINAL, GATED, false, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
       }
     }
     if (FINAL && ys) sm100::fence_proxy_async_smem();   // make the y tile visible to the TMA store
@@ -368,10 +351,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   }
 
   if (!FINAL && cvalid) {
-    float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 + m0);
+    float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
 #pragma unroll
-    for (int q = 0; q < NQ / 2; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
-    if (h == 0) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
+    p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
   }
 }
 

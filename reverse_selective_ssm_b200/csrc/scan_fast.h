@@ -9,7 +9,7 @@ namespace r2l {
 
 struct ScanArgs {
   const __nv_bfloat16* u;   long long ldu;    // [B·L, E]
-  const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz)
+  const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz): z, or SiLU(z) when gated
   const __nv_bfloat16* dt;  long long ldt;    // dt_raw [B·L, E] (before bias and softplus)
   const float* bc;          long long ldbc;   // [B·L, 32]: B in columns 0..15, C in 16..31
   const float* A_log;                          // [E, 16]
@@ -22,7 +22,7 @@ struct ScanArgs {
   float* carry;                                // scan_carry_bytes() of device scratch (may be null if 1 chunk)
   unsigned* err;                               // device status word
   int force_general;                           // never use the A = -(1..16) power path
-  int split;                                   // threads per channel: 1, 2, or 0 = automatic
+  int gated;                                   // z already holds SiLU(z)
 };
 
 // Tokens per chunk chosen from the shape alone (deterministic, no device query).
@@ -31,8 +31,6 @@ int scan_auto_chunk_tokens(int B, int L, int E);
 int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens);
 // Bytes of carry scratch the scan needs for this shape and chunk length.
 size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens);
-// Threads per channel the scan uses for this shape (request 1 or 2, or 0 = automatic).
-int scan_resolve_split(int B, int L, int E, int request);
 // Enqueue the scan (1 or 3 launches).  Returns the number of kernels launched
 // through *launches when not null.
 cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches);

@@ -38,42 +38,35 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
   return (size_t)B * nc * E * 17 * sizeof(float);
 }
 
-int scan_resolve_split(int B, int L, int E, int request) {
-  if (request == 1 || request == 2) return request;
-  (void)B; (void)L; (void)E;
-  return 1;
-}
-
 namespace {
 
-template <int SPLIT>
-cudaError_t launch_split(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
+template <bool GATED>
+cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
   using namespace rscan;
-  using Gm = Geo<SPLIT>;
   const long long M = (long long)a.B * a.L;
   CUtensorMap tu, tz, tdt, tbc, ty;
-  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, Gm::CH, TS, false) ||
-      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, Gm::CH, TS, false) ||
-      !make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, Gm::CH, TS, false) ||
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CH, TS, false) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CH, TS, false) ||
+      !make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, CH, TS, false) ||
       !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, false) ||
-      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, Gm::CH, TS, false))
+      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, CH, TS, false))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  e = cudaFuncSetAttribute(chunk_scan_kernel<true, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)Gm::SMEM_BYTES);
+  e = cudaFuncSetAttribute(chunk_scan_kernel<true, GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.E + Gm::CH - 1) / Gm::CH, nc, a.B);
+  const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
   if (nc > 1) {
-    e = cudaFuncSetAttribute(chunk_scan_kernel<false, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Gm::SMEM_BYTES);
+    e = cudaFuncSetAttribute(chunk_scan_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chunk_scan_kernel<false, SPLIT><<<grid, THREADS, Gm::SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
+    chunk_scan_kernel<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     if (launches) *launches += 2;
   }
-  chunk_scan_kernel<true, SPLIT><<<grid, THREADS, Gm::SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
+  chunk_scan_kernel<true, GATED><<<grid, THREADS, SMEM_BYTES, st>>>(tu, tz, tdt, tbc, ty, p);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;
@@ -106,8 +99,7 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.carry_sum = a.carry ? a.carry + (size_t)a.B * nc * a.E * 16 : nullptr;
   p.err = a.err;
   p.force_general = a.force_general;
-  if (scan_resolve_split(a.B, a.L, a.E, a.split) == 2) return launch_split<2>(a, p, nc, st, launches);
-  return launch_split<1>(a, p, nc, st, launches);
+  return a.gated ? launch<true>(a, p, nc, st, launches) : launch<false>(a, p, nc, st, launches);
 }
 
 }  // namespace r2l

@@ -165,4 +165,98 @@ ln_gate_residual_kernel(T* __restrict__ h, const T* __restrict__ o, const float*
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 path of the LayerNorm + gated residual: one warp per valid row, 16-byte
+// accesses, the row of o held in registers (NV chunks of 8 per lane, so
+// d ≤ 256·NV) for a two-pass mean / variance without re-reading memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int NV, bool HAS_LN>
+__global__ void __launch_bounds__(128)
+ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const float* __restrict__ ln_w,
+                        const float* __restrict__ ln_b, float g, int d, const int* __restrict__ len, int L,
+                        long long M, float* __restrict__ hhat_out) {
+  const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const long long b = row / L;
+  if ((int)(row - b * L) >= len[b]) return;
+  const bf16* orow = o + row * d;
+  bf16* hrow = h + row * d;
+  float v[NV][8];
+  float s = 0.0f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int col = (k * 32 + lane) * 8;
+    if (col < d) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(orow + col);
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(p2[q]);
+        v[k][2 * q] = f.x;
+        v[k][2 * q + 1] = f.y;
+        s += f.x + f.y;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[k][q] = 0.0f;
+    }
+  }
+  float mean = 0.0f, rstd = 1.0f;
+  if (HAS_LN) {
+    mean = warp_sum(s) / (float)d;
+    float q2 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int col = (k * 32 + lane) * 8;
+      if (col < d) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float t = v[k][q] - mean;
+          q2 = fmaf(t, t, q2);
+        }
+      }
+    }
+    rstd = rsqrtf(warp_sum(q2) / (float)d + 1e-5f);
+  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int col = (k * 32 + lane) * 8;
+    if (col >= d) continue;
+    float hv[8];
+    if (HAS_LN) {
+      const float4 w0 = *reinterpret_cast<const float4*>(ln_w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(ln_w + col + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(ln_b + col);
+      const float4 b1 = *reinterpret_cast<const float4*>(ln_b + col + 4);
+      const float gw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float gb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hv[q] = fmaf((v[k][q] - mean) * rstd, gw[q], gb[q]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hv[q] = v[k][q];
+    }
+    if (hhat_out) {
+      float4* dst = reinterpret_cast<float4*>(hhat_out + row * d + col);
+      dst[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      dst[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+    }
+    uint4 hraw = *reinterpret_cast<const uint4*>(hrow + col);
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&hraw);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h2[q]);
+      h2[q] = __floats2bfloat162_rn(fmaf(g, hv[2 * q], f.x), fmaf(g, hv[2 * q + 1], f.y));
+    }
+    *reinterpret_cast<uint4*>(hrow + col) = hraw;
+  }
+}
+
 }  // namespace r2l

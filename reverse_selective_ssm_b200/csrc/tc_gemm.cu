@@ -27,7 +27,7 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   const long long tiles = (long long)((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, static_cast<TOut*>(g.C), g.ldc, g.C2, g.ldc2, g.c2_cols,
+  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, static_cast<TOut*>(g.C), g.ldc, g.C2, g.ldc2, g.c2_cols, g.silu_from_col,
                                             g.M, g.N, g.K, g.len, g.L, g.err);
   return cudaPeekAtLastError();
 }

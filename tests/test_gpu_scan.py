@@ -78,39 +78,33 @@ def check(got, want, B, L, lengths, tol):
             assert torch.isnan(got[b * L + n: (b + 1) * L].float()).all(), f"padding of sequence {b} written"
 
 
-LAYOUTS = {"auto": 0, "split1": bd.R2L_FLAG_SCAN_SPLIT1, "split2": bd.R2L_FLAG_SCAN_SPLIT2}
-
-
-@pytest.mark.parametrize("layout", sorted(LAYOUTS))
 @pytest.mark.parametrize("chunk_tokens", [0, 16, 48, 96, 100000])
 @pytest.mark.parametrize("structured", [True, False])
-def test_scan_bf16_chunks(chunk_tokens, structured, layout):
+def test_scan_bf16_chunks(chunk_tokens, structured):
     B, L, E = 3, 301, 384
     lengths = [301, 1, 170]
     inp = make_scan_inputs(B, L, E, seed=11 + structured, structured_A=structured)
-    got = run_scan(inp, B, L, E, lengths, chunk_tokens, flags=LAYOUTS[layout])
+    got = run_scan(inp, B, L, E, lengths, chunk_tokens)
     want = oracle_scan(inp, B, L, E, lengths)
     check(got, want, B, L, lengths, 5e-3)
 
 
-@pytest.mark.parametrize("layout", ["split1", "split2"])
-def test_scan_bf16_partial_channel_block_and_empty(layout):
+def test_scan_bf16_partial_channel_block_and_empty():
     B, L, E = 4, 130, 200            # 200 = full 128- or 64-channel blocks + a partial one
     lengths = [0, 130, 64, 17]
     inp = make_scan_inputs(B, L, E, seed=21)
     want = oracle_scan(inp, B, L, E, lengths)
     for T in (0, 32):
-        got = run_scan(inp, B, L, E, lengths, T, flags=LAYOUTS[layout])
+        got = run_scan(inp, B, L, E, lengths, T)
         check(got, want, B, L, lengths, 5e-3)
 
 
-@pytest.mark.parametrize("layout", ["split1", "split2"])
-def test_scan_bf16_forced_general_path(layout):
+def test_scan_bf16_forced_general_path():
     B, L, E = 2, 257, 256
     inp = make_scan_inputs(B, L, E, seed=31, structured_A=True)
     want = oracle_scan(inp, B, L, E, None)
-    a = run_scan(inp, B, L, E, None, 64, flags=LAYOUTS[layout])
-    b = run_scan(inp, B, L, E, None, 64, flags=bd.R2L_FLAG_GENERAL_A | LAYOUTS[layout])
+    a = run_scan(inp, B, L, E, None, 64)
+    b = run_scan(inp, B, L, E, None, 64, flags=bd.R2L_FLAG_GENERAL_A)
     check(a, want, B, L, None, 5e-3)
     check(b, want, B, L, None, 5e-3)
 
@@ -130,8 +124,7 @@ def test_scan_long_sequence_many_chunks():
     B, L, E = 1, 4096, 4096
     inp = make_scan_inputs(B, L, E, seed=51)
     want = oracle_scan(inp, B, L, E, None)
-    for flags in (0, bd.R2L_FLAG_SCAN_SPLIT2):
-        auto = run_scan(inp, B, L, E, None, 0, flags=flags)
-        whole = run_scan(inp, B, L, E, None, 1 << 20, flags=flags)
-        check(auto, want, B, L, None, 5e-3)
-        check(whole, want, B, L, None, 5e-3)
+    auto = run_scan(inp, B, L, E, None, 0)
+    whole = run_scan(inp, B, L, E, None, 1 << 20)
+    check(auto, want, B, L, None, 5e-3)
+    check(whole, want, B, L, None, 5e-3)
