@@ -232,10 +232,14 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a4: dt_raw = Δr · W_dtᵀ  (bias + softplus applied in the scan)
   R2L_TRY(prof->mark(R2L_STAGE_DT_PROJ, st));
   prof->launches++;
-  if constexpr (kTC)
-    R2L_TRY(proj((const T*)dr, R, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, err, st));
-  else
+  // bf16 with dt_rank 128: dt_proj runs on the tensor cores inside the scan
+  const bool dt_fused = kTC && R == r2l::kScanFusedDtRank;
+  if constexpr (kTC) {
+    if (!dt_fused) R2L_TRY(proj((const T*)dr, R, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, err, st));
+    else prof->launches--;
+  } else {
     R2L_TRY(gemm((const float*)dbc, p.ldd, (const T*)w->dt_proj_w, R, dt, E, M, E, R, len, L, st));
+  }
   // a5: reverse selective scan, y = (C·H + D u) · SiLU(z)
   R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
   prof->launches++;
@@ -253,6 +257,9 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
     sa.gated = 1;   // the in_proj epilogue stored SiLU(z)
+    sa.dt_mma = dt_fused ? 1 : 0;
+    sa.dr = dr; sa.lddr = R;
+    sa.wdt = (const bf16*)w->dt_proj_w;
     int nl = 0;
     if (r2l::scan_bf16(sa, st, &nl) != cudaSuccess) return R2L_ERR_CUDA;
     prof->launches += nl - 1;

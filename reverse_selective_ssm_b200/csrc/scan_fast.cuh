@@ -3,19 +3,26 @@
 // flipped sequence, run here from each sequence's last valid token to its
 // first):
 //
-//   Δ_i = softplus(dt_raw_i + dt_b)
+//   Δ_i = softplus(dt_raw_i + dt_b),   dt_raw_i = W_dt · Δr_i
 //   H_i = exp(Δ_i A) ⊙ H_{i+1} + Δ_i u_i B_i          (H entering the last token = 0)
 //   y_i = (⟨C_i, H_i⟩ + D u_i) · SiLU(z_i)
 //
 // Work split: a CTA owns 128 channels of one sequence over one chunk of
 // tokens; each of its 4 compute warps holds 32 channels, one channel per
 // thread, with the 16-entry state in registers updated by packed f32x2
-// arithmetic.  A fifth warp streams [16 tokens × 128 channels] tiles of u,
-// z (or SiLU(z), see GATED), dt_raw and the [16 tokens × 32]
-// tile of B|C into a 4-deep shared-memory ring with TMA, from the chunk's right
-// end to its left end, and writes each finished y tile back with a TMA store
-// (tiles that cross the chunk's left edge are stored row by row by the compute
-// threads instead, so no row outside the chunk is ever written).
+// arithmetic.  A producer warp streams [16 tokens × 128 channels] tiles of u
+// and z (or SiLU(z), see GATED), the [16 tokens × 32] tile of B|C, and either
+// the dt_raw tile or, with DTMMA, the [16 tokens × R] tile of Δr, into a
+// 4-deep shared-memory ring with TMA, from the chunk's right end to its left
+// end; it writes each finished y tile back with a TMA store (tiles that cross
+// the chunk's left edge are stored row by row by the compute threads, so no
+// row outside the chunk is ever written).
+//
+// DTMMA (dt_proj fused, R = 128): a sixth warp keeps the CTA's W_dt slice
+// [128 channels × R] in shared memory and, per tile, issues tcgen05.mma
+// (M = 128 channels, N = 16 tokens, K = R) into a TMEM column block; the
+// accumulator's lane is the channel, so each compute thread reads its 16
+// dt_raw values with one tcgen05.ld.  dt_raw never touches HBM.
 //
 // When a sequence is split into several chunks (to give the GPU enough
 // independent work), three launches cooperate through a small carry buffer:
@@ -43,19 +50,38 @@ namespace r2l {
 namespace rscan {
 
 constexpr int TS = 16;        // tokens per pipeline stage
+constexpr int SUB = 8;        // tokens per phase-A / phase-B sub-tile
 constexpr int STAGES = 4;
 constexpr int CWARPS = 4;     // compute warps
 constexpr int CTHREADS = CWARPS * 32;
-constexpr int THREADS = CTHREADS + 32;
+constexpr int CH = CTHREADS;  // channels per CTA
+constexpr int DT_R = 128;     // dt_rank of the fused dt_proj (kScanFusedDtRank)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-constexpr int CH = CTHREADS;                      // channels per CTA
-constexpr int SUB = 8;                            // tokens per phase-A / phase-B sub-tile
 constexpr uint32_t ACT_TILE = TS * CH * 2;        // one bf16 [TS × CH] tile
 constexpr uint32_t BC_TILE = TS * 32 * 4;         // one fp32 [TS × 32] tile
-// per stage: u, dt, z, y tiles and the B|C tile
-constexpr size_t SMEM_BYTES = 128 + STAGES * (4 * (size_t)ACT_TILE + BC_TILE) + 2 * STAGES * 8;
+constexpr uint32_t DR_TILE = TS * DT_R * 2;       // one bf16 [TS × R] Δr tile (2 swizzle atoms)
+constexpr uint32_t W_SLICE = CH * DT_R * 2;       // bf16 W_dt [CH × R] (2 atoms of 16 KB)
+constexpr uint32_t TMEM_COLS = 64;                // STAGES × TS fp32 columns
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).  Without
+// DTMMA: u, dt, z, y tiles, B|C tiles, barriers.  With DTMMA: W slice, Δr
+// tiles, u, z, y tiles, B|C tiles, barriers.
+template <bool DTMMA>
+struct Smem {
+  static constexpr uint32_t W = 0;
+  static constexpr uint32_t DR = DTMMA ? W_SLICE : 0;
+  static constexpr uint32_t U = DR + (DTMMA ? STAGES * DR_TILE : 0);
+  static constexpr uint32_t DT = U + STAGES * ACT_TILE;           // unused with DTMMA
+  static constexpr uint32_t Z = DT + (DTMMA ? 0 : STAGES * ACT_TILE);
+  static constexpr uint32_t Y = Z + STAGES * ACT_TILE;
+  static constexpr uint32_t BC = Y + STAGES * ACT_TILE;
+  static constexpr uint32_t BAR = BC + STAGES * BC_TILE;          // full, empty, dtready [STAGES], wfull, drain
+  static constexpr uint32_t SLOT = BAR + (3 * STAGES + 2) * 8;    // TMEM base address
+  static constexpr size_t BYTES = 1024 + SLOT + 16;
+  static constexpr int THREADS = CTHREADS + 32 + (DTMMA ? 32 : 0);
+};
 
 struct Params {
   const float* A_log;   // [E, 16]
@@ -118,19 +144,22 @@ struct Ctx {
 // Phase A computes what does not depend on the state (softplus, the decay
 // base, Δu, D·u, the gate) for all of its tokens; phase B runs the
 // recurrence.  FULL: every token of the sub-tile is inside the chunk.  GATED:
-// the z tile already holds SiLU(z).  Output: y rows to shared memory (ys,
-// stride CH) for tiles stored by TMA, else to global (yg).
-template <bool FINAL, bool GATED, bool POW, bool FULL>
+// the z tile already holds SiLU(z).  dtv: the tile's 16 dt_raw values (DTMMA)
+// or unused (read sdt).  Output: y rows to shared memory (ys, stride CH) for
+// tiles stored by TMA, else to global (yg).
+template <bool FINAL, bool GATED, bool POW, bool FULL, bool DTMMA>
 __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& sumd, const bf16* su,
-                                         const bf16* sdt, const bf16* sz, const float* sbc, bf16* ys, bf16* yg,
-                                         long long ldy, bool store_ok, int j0, int jmin) {
+                                         const bf16* sdt, const float (&dtv)[16], const bf16* sz,
+                                         const float* sbc, bf16* ys, bf16* yg, long long ldy, bool store_ok,
+                                         int j0, int jmin) {
   float dec[SUB], du[SUB], gz[SUB], Du[SUB];
 #pragma unroll
   for (int t = 0; t < SUB; ++t) {
     const int j = j0 + t;
     if (!FULL && j < jmin) continue;
     float delta, r;
-    softplus_and_decay(__bfloat162float(sdt[j * CH]) + cx.dtb, delta, r);
+    const float raw = DTMMA ? dtv[j] : __bfloat162float(sdt[j * CH]);
+    softplus_and_decay(raw + cx.dtb, delta, r);
     const float uu = __bfloat162float(su[j * CH]);
     dec[t] = POW ? r : delta;
     du[t] = delta * uu;
@@ -193,13 +222,21 @@ __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& s
 
 // The TMA producer (one thread): streams the chunk's tiles right to left into
 // the STAGES-deep ring and, for the final scan, writes each finished y tile
-// that lies wholly inside the chunk back with a bulk tensor store.
-template <bool FINAL>
+// that lies wholly inside the chunk back with a bulk tensor store.  With
+// DTMMA it first loads the CTA's W_dt slice, and streams Δr tiles instead of
+// dt_raw tiles.
+template <bool FINAL, bool DTMMA>
 __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUtensorMap* tm_z,
                                              const CUtensorMap* tm_dt, const CUtensorMap* tm_bc,
-                                             const CUtensorMap* tm_y, bf16* s_u, bf16* s_dt, bf16* s_z,
-                                             bf16* s_y, float* s_bc, uint64_t* full, uint64_t* empty, int b,
-                                             int cb, int s0, int e0, int ntiles, const Params& p) {
+                                             const CUtensorMap* tm_y, const CUtensorMap* tm_w, uint8_t* smem,
+                                             uint64_t* full, uint64_t* empty, uint64_t* wfull, int b, int cb,
+                                             int s0, int e0, int ntiles, const Params& p) {
+  using S = Smem<DTMMA>;
+  bf16* s_u = reinterpret_cast<bf16*>(smem + S::U);
+  bf16* s_dt = reinterpret_cast<bf16*>(smem + S::DT);
+  bf16* s_z = reinterpret_cast<bf16*>(smem + S::Z);
+  bf16* s_y = reinterpret_cast<bf16*>(smem + S::Y);
+  float* s_bc = reinterpret_cast<float*>(smem + S::BC);
   sm100::prefetch_tmap(tm_u);
   sm100::prefetch_tmap(tm_dt);
   sm100::prefetch_tmap(tm_bc);
@@ -207,7 +244,13 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
     sm100::prefetch_tmap(tm_z);
     sm100::prefetch_tmap(tm_y);
   }
-  constexpr uint32_t bytes = (FINAL ? 3 : 2) * ACT_TILE + BC_TILE;
+  if (DTMMA) {
+    sm100::prefetch_tmap(tm_w);
+    sm100::mbar_arrive_expect_tx(wfull, W_SLICE);
+    for (int a = 0; a < DT_R / 64; ++a)
+      sm100::tma_load_2d(smem + S::W + a * (CH * 128), tm_w, a * 64, cb * CH, wfull);
+  }
+  constexpr uint32_t bytes = (FINAL ? 2 : 1) * ACT_TILE + BC_TILE + (DTMMA ? DR_TILE : ACT_TILE);
   int issued = 0;
   bool ok = true;
   const int iters = ntiles + (FINAL ? STAGES : 0);
@@ -227,7 +270,12 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
       const int row0 = b * p.L + e0 - (it + 1) * TS;  // may be negative for b = 0: reads zeros
       sm100::mbar_arrive_expect_tx(&full[st], bytes);
       sm100::tma_load_2d(s_u + st * TS * CH, tm_u, cb * CH, row0, &full[st]);
-      sm100::tma_load_2d(s_dt + st * TS * CH, tm_dt, cb * CH, row0, &full[st]);
+      if (DTMMA) {
+        uint8_t* dr = smem + S::DR + st * DR_TILE;
+        for (int a = 0; a < DT_R / 64; ++a) sm100::tma_load_2d(dr + a * (TS * 128), tm_dt, a * 64, row0, &full[st]);
+      } else {
+        sm100::tma_load_2d(s_dt + st * TS * CH, tm_dt, cb * CH, row0, &full[st]);
+      }
       if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, tm_z, cb * CH, row0, &full[st]);
       sm100::tma_load_2d(s_bc + st * TS * 32, tm_bc, 0, row0, &full[st]);
       ++issued;
@@ -237,27 +285,61 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
   if (!ok) {  // drain loads still in flight before the CTA can exit
     for (int it = issued - 1; it >= 0 && it >= issued - STAGES; --it)
       sm100::mbar_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u, nullptr, 1000000000ull);
+    if (DTMMA) sm100::mbar_wait(wfull, 0, nullptr, 1000000000ull);
   }
 }
 
-template <bool FINAL, bool GATED>
-__global__ void __launch_bounds__(THREADS, 2)
+// The dt_proj MMA issuer (one thread, DTMMA): per tile, dt_rawᵀ[128 ch × 16
+// tokens] = W_dt slice · Δr tileᵀ into TMEM columns [16·st, 16·st + 16).
+__device__ __forceinline__ void run_dt_mma(uint8_t* smem, uint32_t tmem_base, uint64_t* full, uint64_t* dtready,
+                                           uint64_t* wfull, uint64_t* drain, int ntiles, unsigned* err) {
+  using S = Smem<true>;
+  constexpr uint32_t idesc = sm100::idesc_bf16_f32(128, TS);
+  bool ok = sm100::mbar_wait(wfull, 0, err);
+  const uint32_t w0 = sm100::smem_u32(smem + S::W);
+  for (int it = 0; it < ntiles && ok; ++it) {
+    const int st = it % STAGES;
+    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+    if (!sm100::mbar_wait(&full[st], ph, err)) break;
+    sm100::tc_fence_after();
+    const uint32_t d0 = sm100::smem_u32(smem + S::DR + st * DR_TILE);
+#pragma unroll
+    for (int k = 0; k < DT_R / 16; ++k) {
+      const uint32_t a_addr = w0 + (k / 4) * (CH * 128) + (k % 4) * 32;
+      const uint32_t b_addr = d0 + (k / 4) * (TS * 128) + (k % 4) * 32;
+      sm100::mma_bf16(tmem_base + (uint32_t)(st * TS), sm100::smem_desc_k128(a_addr), sm100::smem_desc_k128(b_addr),
+                      idesc, k != 0);
+    }
+    sm100::mma_commit(&dtready[st]);
+  }
+  sm100::mma_commit(drain);
+  sm100::mbar_wait(drain, 0, err, 1000000000ull);
+}
+
+template <bool FINAL, bool GATED, bool DTMMA>
+__global__ void __launch_bounds__(Smem<DTMMA>::THREADS, 2)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
-                  const __grid_constant__ CUtensorMap tm_y, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
+                  const Params p) {
+  using S = Smem<DTMMA>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  bf16* s_u = reinterpret_cast<bf16*>(smem);
-  bf16* s_dt = s_u + STAGES * TS * CH;
-  bf16* s_z = s_dt + STAGES * TS * CH;
-  bf16* s_y = s_z + STAGES * TS * CH;
-  float* s_bc = reinterpret_cast<float*>(s_y + STAGES * TS * CH);
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_bc + STAGES * TS * 32);
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const bf16* s_u = reinterpret_cast<const bf16*>(smem + S::U);
+  const bf16* s_dt = reinterpret_cast<const bf16*>(smem + S::DT);
+  const bf16* s_z = reinterpret_cast<const bf16*>(smem + S::Z);
+  bf16* s_y = reinterpret_cast<bf16*>(smem + S::Y);
+  const float* s_bc = reinterpret_cast<const float*>(smem + S::BC);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR);
   uint64_t* empty = full + STAGES;
+  uint64_t* dtready = empty + STAGES;
+  uint64_t* wfull = dtready + STAGES;
+  uint64_t* drain = wfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::SLOT);
 
   const int cb = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
+  const int warp = tid >> 5, lane = tid & 31;
   const bool compute = tid < CTHREADS;
   const int ch = compute ? tid : 0;             // channel within the block
   const int c = cb * CH + ch;
@@ -281,15 +363,30 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
     for (int s = 0; s < STAGES; ++s) {
       sm100::mbar_init(&full[s], 1);
       sm100::mbar_init(&empty[s], CWARPS);
+      sm100::mbar_init(&dtready[s], 1);
     }
+    sm100::mbar_init(wfull, 1);
+    sm100::mbar_init(drain, 1);
     sm100::fence_barrier_init();
   }
+  if (DTMMA && warp == CWARPS + 1) sm100::tmem_alloc(tmem_slot, TMEM_COLS);
+  sm100::tc_fence_before();
   __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = DTMMA ? *tmem_slot : 0u;
 
-  if (!compute) {
+  if (warp == CWARPS) {
     if (lane == 0)
-      run_producer<FINAL>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, s_u, s_dt, s_z, s_y, s_bc, full, empty, b, cb, s0,
-                          e0, ntiles, p);
+      run_producer<FINAL, DTMMA>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b, cb, s0,
+                                 e0, ntiles, p);
+    return;   // the producer warp takes no part in the teardown below
+  }
+  if (DTMMA && warp == CWARPS + 1) {
+    if (lane == 0) run_dt_mma(smem, tmem_base, full, dtready, wfull, drain, ntiles, p.err);
+    __syncwarp();
+    sm100::named_bar_sync(1, CTHREADS + 32);   // every compute warp has finished reading TMEM
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem_base, TMEM_COLS);
     return;
   }
 
@@ -320,11 +417,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
     for (int q = 0; q < 8; ++q) H[q] = make_float2(0.0f, 0.0f);
   }
   float sumd = 0.0f;
+  float dtv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) dtv[j] = 0.0f;
 
   for (int it = 0; it < ntiles; ++it) {
     const int st = it % STAGES;
     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
     if (!sm100::mbar_wait(&full[st], ph, p.err)) break;
+    if (DTMMA) {
+      if (!sm100::mbar_wait(&dtready[st], ph, p.err)) break;
+      sm100::tc_fence_after();
+      sm100::tmem_ld16(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(st * TS), dtv);
+    }
     const int tbase = e0 - (it + 1) * TS;        // sequence position of tile row 0
     const int jmin = s0 > tbase ? s0 - tbase : 0;
     const bf16* su = s_u + st * TS * CH + ch;
@@ -338,14 +443,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
 #pragma unroll
     for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
       if (jmin == 0) {
-        if (use_pow) scan_sub<FINAL, GATED, true, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
-        else scan_sub<FINAL, GATED, false, true>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+        if (use_pow)
+          scan_sub<FINAL, GATED, true, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+        else
+          scan_sub<FINAL, GATED, false, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
       } else if (j0 + SUB > jmin) {
-        if (use_pow) scan_sub<FINAL, GATED, true, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
-        else scan_sub<FINAL, GATED, false, false>(cx, H, sumd, su, sdt, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+        if (use_pow)
+          scan_sub<FINAL, GATED, true, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+        else
+          scan_sub<FINAL, GATED, false, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
       }
     }
     if (FINAL && ys) sm100::fence_proxy_async_smem();   // make the y tile visible to the TMA store
+    if (DTMMA) sm100::tc_fence_before();
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[st]);
   }
@@ -355,6 +465,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
     p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
+  }
+  if (DTMMA) {
+    sm100::tc_fence_before();
+    sm100::named_bar_sync(1, CTHREADS + 32);   // release TMEM to the dealloc
   }
 }
 

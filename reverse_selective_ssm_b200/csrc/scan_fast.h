@@ -7,10 +7,15 @@
 
 namespace r2l {
 
+// dt_rank for which the scan computes dt_proj itself on the tensor cores.
+constexpr int kScanFusedDtRank = 128;
+
 struct ScanArgs {
   const __nv_bfloat16* u;   long long ldu;    // [B·L, E]
   const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz): z, or SiLU(z) when gated
-  const __nv_bfloat16* dt;  long long ldt;    // dt_raw [B·L, E] (before bias and softplus)
+  const __nv_bfloat16* dt;  long long ldt;    // dt_raw [B·L, E] (before bias and softplus); unused with dt_mma
+  const __nv_bfloat16* dr;  long long lddr;   // dt_mma: Δr [B·L, 128] (x_proj output)
+  const __nv_bfloat16* wdt;                    // dt_mma: W_dt [E, 128]
   const float* bc;          long long ldbc;   // [B·L, 32]: B in columns 0..15, C in 16..31
   const float* A_log;                          // [E, 16]
   const float* D;                              // [E]
@@ -23,6 +28,7 @@ struct ScanArgs {
   unsigned* err;                               // device status word
   int force_general;                           // never use the A = -(1..16) power path
   int gated;                                   // z already holds SiLU(z)
+  int dt_mma;                                  // compute dt_raw = Δr·W_dtᵀ inside the scan (dt_rank 128)
 };
 
 // Tokens per chunk chosen from the shape alone (deterministic, no device query).
