@@ -44,6 +44,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, default=2, help="workload 1..4 (2 = the headline)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (profiling)")
+    ap.add_argument("--seq", type=int, default=None, help="override the workload's sequence length (profiling)")
     ap.add_argument("--general-a", action="store_true", help="force the general-A scan path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -147,8 +149,13 @@ def algorithmic(case, stage):
         return "tensor", 2.0 * T * E * d, "flop"
     if stage == "conv":
         return "hbm", float(T) * E * (a + a), "byte"
-    if stage == "scan":       # u, z, dt_raw read, y written (act) + B, C read (fp32)
-        return "hbm", float(T) * (E * 4 * a + 2 * N * 4), "byte"
+    if stage == "scan":
+        # u, z read and y written (act) + B, C read (fp32), plus either the dt_raw
+        # row (act) or, when dt_proj runs inside the scan (bf16, dt_rank 128),
+        # the dt_rank-wide Δr row (bf16)
+        fused = a == 2 and R == 128
+        dt_bytes = R * 2 if fused else E * a
+        return "hbm", float(T) * (E * 3 * a + dt_bytes + 2 * N * 4), "byte"
     if stage == "ln_residual":  # o read, h read, h written
         return "hbm", float(T) * d * 3 * a, "byte"
     raise KeyError(stage)
@@ -183,7 +190,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     bd.load()
-    case = S.make_case(args.config)
+    case = S.make_case(args.config, B=args.batch, L=args.seq)
+    if args.batch or args.seq:
+        case.name += f" (resized to B={case.B} L={case.L})"
     flags = bd.R2L_FLAG_GENERAL_A if args.general_a else 0
     dims = bd.dims_of(case.dims, case.dtype, flags)
     h = case.h.to(dev)
@@ -287,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     peaks, peak_kind = load_peaks()
-    workload_tag = f"config{args.config}"
+    workload_tag = f"config{args.config}-B{case.B}-L{case.L}"
     dom = max(per_launch, key=per_launch.get)
     line = {
         "metric": METRIC,

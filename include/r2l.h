@@ -106,9 +106,7 @@ typedef struct {
  * unspecified values, except in hhat where they are not written.             */
 typedef struct {
   void  *x;        /* act  [B·L, E]      in_proj, first half                  */
-  void  *z;        /* act  [B·L, E]      in_proj, second half; the bf16 path
-                                           stores SiLU(z) here (its in_proj
-                                           epilogue applies the gate activation) */
+  void  *z;        /* act  [B·L, E]      in_proj, second half                 */
   void  *u;        /* act  [B·L, E]      conv + SiLU                          */
   float *dbc;      /* fp32 [B·L, R+2N]   x_proj output Δr | B | C             */
   void  *y;        /* act  [B·L, E]      scan output after the SiLU(z) gate   */

@@ -44,19 +44,56 @@ __device__ __forceinline__ bool rows_have_valid(const int* __restrict__ len, int
   return false;
 }
 
-template <int BN>
+template <int BN, typename TOut>
 struct TcGemmCfg {
   static constexpr int BM = 128;
   static constexpr int BK = 64;                       // 128 bytes of bf16: one swizzle row
-  static constexpr int STAGES = BN >= 256 ? 4 : 6;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  // epilogue staging: per epilogue warp two [32 rows × 32 cols] buffers
+  static constexpr uint32_t STG_BYTES = 32 * 32 * sizeof(TOut);
+  static constexpr int STG_SWIZZLE = 32 * sizeof(TOut);   // 64 (bf16 rows) or 128 (fp32 rows)
+  static constexpr size_t BUDGET = 227 * 1024 - 1024 - 256 - 8 * STG_BYTES;
+  static constexpr int STAGES_FIT = (int)(BUDGET / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT < 6 ? STAGES_FIT : 6;
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (size_t)STAGE_BYTES + 256 /*barriers*/;
+  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (size_t)STAGE_BYTES + 8 * STG_BYTES + 256;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128 is a multiple of 16 up to 256");
   static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte swizzle-atom alignment");
+  static_assert(STAGES >= 3, "shared memory too small for the pipeline");
 };
+
+// Write one thread's row of 32 values into a [32 × 32] staging buffer laid
+// out for a TMA store with STG_SWIZZLE: the 16-byte chunk k of row r sits at
+// chunk k ^ ((r >> 1) & 3) for 64-byte rows, k ^ (r & 7) for 128-byte rows,
+// so the 32 rows written by a warp hit distinct banks.
+template <typename TOut>
+__device__ __forceinline__ void stage_row32(uint8_t* buf, int r, const float (&v)[32]);
+
+template <>
+__device__ __forceinline__ void stage_row32<bf16>(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(v[k * 8 + 2 * j], v[k * 8 + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    const int pk = k ^ ((r >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + r * 64 + pk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <>
+__device__ __forceinline__ void stage_row32<float>(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int pk = k ^ (r & 7);
+    *reinterpret_cast<float4*>(buf + r * 128 + pk * 16) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  }
+}
 
 template <typename TOut>
 __device__ __forceinline__ void store_row32(TOut* dst, const float (&v)[32]);
@@ -85,20 +122,19 @@ __device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[
 
 // C2 (optional): columns n < c2_cols are also written, rounded to bf16, into
 // C2[m, n] (row stride ldc2).  x_proj uses it to hand Δr to dt_proj in bf16.
-// silu_from_col >= 0: columns n >= silu_from_col are stored as SiLU(C[m, n])
-// (in_proj applies the Mamba-1 gate activation to its z half here).
 template <int BN, typename TOut>
 __global__ void __launch_bounds__(192, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               TOut* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols, int silu_from_col,
+               const __grid_constant__ CUtensorMap tmC, bf16* __restrict__ C2, int ldc2, int c2_cols,
                int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err) {
-  using Cfg = TcGemmCfg<BN>;
+  using Cfg = TcGemmCfg<BN, TOut>;
   constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_BYTES);
+  uint8_t* sStg = sB + STAGES * Cfg::B_BYTES;          // 8 staging buffers (1024-byte aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 8 * Cfg::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -125,6 +161,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     sm100::fence_barrier_init();
     sm100::prefetch_tmap(&tmA);
     sm100::prefetch_tmap(&tmB);
+    sm100::prefetch_tmap(&tmC);
   }
   if (warp == 1) sm100::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
   sm100::tc_fence_before();
@@ -202,9 +239,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each 32 × 32 block goes TMEM -> registers -> swizzled staging buffer ->
+    // TMA store (rows past M or columns past N are clipped by the store).
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* stg = sStg + (warp - 2) * 2 * Cfg::STG_BYTES;
     int acc = 0;
     uint32_t aphase = 0;
+    int chunk = 0;
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       if (!tile_live(t)) continue;
       if (!sm100::mbar_wait(&tfull[acc], aphase, err)) break;
@@ -213,33 +254,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const long long row = (long long)mb * BM + q * 32 + lane;
       const bool row_ok = row < M && (!len || row_valid(len, L, row));
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32, ++chunk) {
         float v[32];
         sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), v);
         const int col = nb * BN + c0;
-        if (silu_from_col >= 0 && col + 32 > silu_from_col) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col + j >= silu_from_col) v[j] = __fdividef(v[j], 1.0f + __expf(-v[j]));
+        uint8_t* buf = stg + (chunk & 1) * Cfg::STG_BYTES;
+        if (lane == 0) sm100::bulk_wait_read_le1();   // the store that used `buf` has read it
+        __syncwarp();
+        stage_row32<TOut>(buf, lane, v);
+        sm100::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && col < N) {
+          sm100::tma_store_2d(&tmC, buf, col, mb * BM + q * 32);
+          sm100::bulk_commit();
         }
-        if (row_ok && col < N) {
-          TOut* dst = C + row * (long long)ldc + col;
-          if (col + 32 <= N) {
-            store_row32<TOut>(dst, v);
+        if (C2 && row_ok && col < c2_cols) {
+          bf16* d2 = C2 + row * (long long)ldc2 + col;
+          if (col + 32 <= c2_cols) {
+            store_row32<bf16>(d2, v);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < N - col) dst[j] = from_f32<TOut>(v[j]);
-          }
-          if (C2 && col < c2_cols) {
-            bf16* d2 = C2 + row * (long long)ldc2 + col;
-            if (col + 32 <= c2_cols) {
-              store_row32<bf16>(d2, v);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < c2_cols - col) d2[j] = __float2bfloat16_rn(v[j]);
-            }
+              if (j < c2_cols - col) d2[j] = __float2bfloat16_rn(v[j]);
           }
         }
       }
@@ -248,6 +284,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       acc ^= 1;
       if (acc == 0) aphase ^= 1u;
     }
+    if (lane == 0) sm100::bulk_wait_all();
   }
 
   sm100::tc_fence_before();

@@ -148,12 +148,12 @@ r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, c
 template <typename T, typename TC>
 r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long long M, int N, int K,
                 const int* len, int L, unsigned* err, cudaStream_t st, bf16* c2 = nullptr, int ldc2 = 0,
-                int c2_cols = 0, int silu_from_col = -1) {
+                int c2_cols = 0) {
   if constexpr (std::is_same<T, bf16>::value) {
     r2l::TcGemm g{};
     g.A = A; g.lda = lda; g.B = W; g.ldb = ldw; g.C = C; g.ldc = ldc;
     g.c_fp32 = std::is_same<TC, float>::value;
-    g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols; g.silu_from_col = silu_from_col;
+    g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols;
     g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
     return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
   } else {
@@ -210,8 +210,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a1: [x | z] = h · W_inᵀ
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
   prof->launches++;
-  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st, nullptr, 0, 0,
-               /*silu_from_col=*/kTC ? E : -1));
+  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
   // a2: u = SiLU(anti-causal conv(x))
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
   prof->launches++;
@@ -256,7 +255,6 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.carry = (float*)(ws + p.carry);
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
-    sa.gated = 1;   // the in_proj epilogue stored SiLU(z)
     sa.dt_mma = dt_fused ? 1 : 0;
     sa.dr = dr; sa.lddr = R;
     sa.wdt = (const bf16*)w->dt_proj_w;
@@ -452,7 +450,6 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
     sa.carry = carry;
     sa.err = status;
     sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
-    sa.gated = 0;
     if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
   } else {
     dim3 grid((E + 127) / 128, B);

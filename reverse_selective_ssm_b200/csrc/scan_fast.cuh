@@ -11,7 +11,7 @@
 // tokens; each of its 4 compute warps holds 32 channels, one channel per
 // thread, with the 16-entry state in registers updated by packed f32x2
 // arithmetic.  A producer warp streams [16 tokens × 128 channels] tiles of u
-// and z (or SiLU(z), see GATED), the [16 tokens × 32] tile of B|C, and either
+// and z, the [16 tokens × 32] tile of B|C, and either
 // the dt_raw tile or, with DTMMA, the [16 tokens × R] tile of Δr, into a
 // 4-deep shared-memory ring with TMA, from the chunk's right end to its left
 // end; it writes each finished y tile back with a TMA store (tiles that cross
@@ -143,11 +143,11 @@ struct Ctx {
 // One sub-tile of SUB tokens [j0, j0 + SUB) of one channel, last token first.
 // Phase A computes what does not depend on the state (softplus, the decay
 // base, Δu, D·u, the gate) for all of its tokens; phase B runs the
-// recurrence.  FULL: every token of the sub-tile is inside the chunk.  GATED:
-// the z tile already holds SiLU(z).  dtv: the tile's 16 dt_raw values (DTMMA)
+// recurrence.  FULL: every token of the sub-tile is inside the chunk.
+// dtv: the tile's 16 dt_raw values (DTMMA)
 // or unused (read sdt).  Output: y rows to shared memory (ys, stride CH) for
 // tiles stored by TMA, else to global (yg).
-template <bool FINAL, bool GATED, bool POW, bool FULL, bool DTMMA>
+template <bool FINAL, bool POW, bool FULL, bool DTMMA>
 __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& sumd, const bf16* su,
                                          const bf16* sdt, const float (&dtv)[16], const bf16* sz,
                                          const float* sbc, bf16* ys, bf16* yg, long long ldy, bool store_ok,
@@ -165,8 +165,7 @@ __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& s
     du[t] = delta * uu;
     if (FINAL) {
       Du[t] = cx.Dc * uu;
-      const float zz = __bfloat162float(sz[j * CH]);
-      gz[t] = GATED ? zz : silu_fast(zz);
+      gz[t] = silu_fast(__bfloat162float(sz[j * CH]));
     } else {
       sumd += delta;
     }
@@ -316,7 +315,7 @@ __device__ __forceinline__ void run_dt_mma(uint8_t* smem, uint32_t tmem_base, ui
   sm100::mbar_wait(drain, 0, err, 1000000000ull);
 }
 
-template <bool FINAL, bool GATED, bool DTMMA>
+template <bool FINAL, bool DTMMA>
 __global__ void __launch_bounds__(Smem<DTMMA>::THREADS, 2)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
@@ -444,14 +443,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
     for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
       if (jmin == 0) {
         if (use_pow)
-          scan_sub<FINAL, GATED, true, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+          scan_sub<FINAL, true, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
         else
-          scan_sub<FINAL, GATED, false, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+          scan_sub<FINAL, false, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
       } else if (j0 + SUB > jmin) {
         if (use_pow)
-          scan_sub<FINAL, GATED, true, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+          scan_sub<FINAL, true, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
         else
-          scan_sub<FINAL, GATED, false, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+          scan_sub<FINAL, false, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
       }
     }
     if (FINAL && ys) sm100::fence_proxy_async_smem();   // make the y tile visible to the TMA store

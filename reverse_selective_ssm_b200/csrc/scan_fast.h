@@ -12,7 +12,7 @@ constexpr int kScanFusedDtRank = 128;
 
 struct ScanArgs {
   const __nv_bfloat16* u;   long long ldu;    // [B·L, E]
-  const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz): z, or SiLU(z) when gated
+  const __nv_bfloat16* z;   long long ldz;    // [B·L, E] (row stride ldz)
   const __nv_bfloat16* dt;  long long ldt;    // dt_raw [B·L, E] (before bias and softplus); unused with dt_mma
   const __nv_bfloat16* dr;  long long lddr;   // dt_mma: Δr [B·L, 128] (x_proj output)
   const __nv_bfloat16* wdt;                    // dt_mma: W_dt [E, 128]
@@ -27,7 +27,6 @@ struct ScanArgs {
   float* carry;                                // scan_carry_bytes() of device scratch (may be null if 1 chunk)
   unsigned* err;                               // device status word
   int force_general;                           // never use the A = -(1..16) power path
-  int gated;                                   // z already holds SiLU(z)
   int dt_mma;                                  // compute dt_raw = Δr·W_dtᵀ inside the scan (dt_rank 128)
 };
 

@@ -40,43 +40,43 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
 
 namespace {
 
-template <bool FINAL, bool GATED, bool DTMMA>
+template <bool FINAL, bool DTMMA>
 cudaError_t prep_kernel() {
-  return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, GATED, DTMMA>,
+  return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, DTMMA>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rscan::Smem<DTMMA>::BYTES);
 }
 
-template <bool GATED, bool DTMMA>
+template <bool DTMMA>
 cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
   using namespace rscan;
   using Sm = Smem<DTMMA>;
   const long long M = (long long)a.B * a.L;
   CUtensorMap tu, tz, tdt, tbc, ty, tw;
-  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CH, TS, false) ||
-      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CH, TS, false) ||
-      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, false) ||
-      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, CH, TS, false))
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CH, TS, 0) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CH, TS, 0) ||
+      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, 0) ||
+      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, CH, TS, 0))
     return cudaErrorInvalidValue;
   if (DTMMA) {
-    if (!make_tmap_2d(&tdt, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, true) ||
-        !make_tmap_2d(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CH, true))
+    if (!make_tmap_2d(&tdt, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, 128) ||
+        !make_tmap_2d(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CH, 128))
       return cudaErrorInvalidValue;
   } else {
-    if (!make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, CH, TS, false)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tdt, a.dt, 2, a.E, M, a.ldt * 2, CH, TS, 0)) return cudaErrorInvalidValue;
     tw = tdt;
   }
   cudaError_t e;
-  if ((e = prep_kernel<true, GATED, DTMMA>()) != cudaSuccess) return e;
+  if ((e = prep_kernel<true, DTMMA>()) != cudaSuccess) return e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
   if (nc > 1) {
-    if ((e = prep_kernel<false, false, DTMMA>()) != cudaSuccess) return e;
-    chunk_scan_kernel<false, false, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+    if ((e = prep_kernel<false, DTMMA>()) != cudaSuccess) return e;
+    chunk_scan_kernel<false, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     if (launches) *launches += 2;
   }
-  chunk_scan_kernel<true, GATED, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+  chunk_scan_kernel<true, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;
@@ -111,9 +111,9 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.force_general = a.force_general;
   if (a.dt_mma) {
     if (!a.dr || !a.wdt || (a.lddr % 8)) return cudaErrorInvalidValue;
-    return a.gated ? launch<true, true>(a, p, nc, st, launches) : launch<false, true>(a, p, nc, st, launches);
+    return launch<true>(a, p, nc, st, launches);
   }
-  return a.gated ? launch<true, false>(a, p, nc, st, launches) : launch<false, false>(a, p, nc, st, launches);
+  return launch<false>(a, p, nc, st, launches);
 }
 
 }  // namespace r2l

@@ -17,17 +17,19 @@ int sm_count() {
 
 template <int BN, typename TOut>
 cudaError_t launch(const TcGemm& g, cudaStream_t st) {
-  using Cfg = TcGemmCfg<BN>;
-  CUtensorMap ta, tb;
-  if (!make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, true)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, true)) return cudaErrorInvalidValue;
+  using Cfg = TcGemmCfg<BN, TOut>;
+  CUtensorMap ta, tb, tc;
+  if (!make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tc, g.C, (int)sizeof(TOut), g.N, g.M, (long long)g.ldc * sizeof(TOut), 32, 32, Cfg::STG_SWIZZLE))
+    return cudaErrorInvalidValue;
   auto kern = gemm_tc_kernel<BN, TOut>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, static_cast<TOut*>(g.C), g.ldc, g.C2, g.ldc2, g.c2_cols, g.silu_from_col,
+  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, g.C2, g.ldc2, g.c2_cols,
                                             g.M, g.N, g.K, g.len, g.L, g.err);
   return cudaPeekAtLastError();
 }
@@ -48,6 +50,7 @@ cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
 cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;
   if ((g.lda % 8) || (g.ldb % 8) || (g.K % 8)) return cudaErrorInvalidValue;  // TMA: 16-byte strides
+  if ((g.ldc * (g.c_fp32 ? 4 : 2)) % 16) return cudaErrorInvalidValue;
   return g.c_fp32 ? dispatch<float>(g, st) : dispatch<bf16>(g, st);
 }
 

@@ -17,7 +17,6 @@ struct TcGemm {
   __nv_bfloat16* C2;       // optional bf16 copy of columns < c2_cols (row stride ldc2)
   int ldc2;
   int c2_cols;
-  int silu_from_col;       // columns n >= silu_from_col are stored as SiLU(C[m, n]); -1: none
   int M, N, K;
   const int* len;          // device lengths [B] (rows i >= len[b] of each sequence are skipped)
   int L;

@@ -25,7 +25,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, long long inner, long long rows,
-                  long long ld_bytes, int box_inner, int box_rows, bool swizzle128) {
+                  long long ld_bytes, int box_inner, int box_rows, int swizzle_bytes) {
   auto enc = encode_fn();
   if (!enc || inner <= 0 || rows <= 0) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
@@ -34,7 +34,9 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, long long in
   cuuint32_t es[2] = {1u, 1u};
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+             : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
