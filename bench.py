@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (profiling)")
     ap.add_argument("--seq", type=int, default=None, help="override the workload's sequence length (profiling)")
     ap.add_argument("--general-a", action="store_true", help="force the general-A scan path")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and time its replays (no per-stage times)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -179,6 +181,25 @@ def roofline_obj(case, stage, ms, peaks, peak_kind, workload_tag):
             "traffic": read_traffic(stage, workload_tag)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank must call this, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Tokens per second over all ranks: every rank runs its own batch (weak
+    scaling), and the job takes as long as its slowest rank."""
+    return tokens_per_rank * world * steps / (ms_max * 1e-3)
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -204,12 +225,14 @@ def run_ours(args, rank, world, local_rank):
     nst = len(bd.STAGES)
 
     def step(events=None):
+        # always the stream current at call time (the capture stream under a graph)
+        st = torch.cuda.current_stream()
         launches = 0
         for k in range(hooks):
             if events is not None:
-                launches += bd.sidecar_forward_profiled(h, wdev[k], dims, case.s[k], events[k], lengths, ws, stream)
+                launches += bd.sidecar_forward_profiled(h, wdev[k], dims, case.s[k], events[k], lengths, ws, st)
             else:
-                bd.sidecar_forward(h, wdev[k], dims, case.s[k], lengths, ws, stream)
+                bd.sidecar_forward(h, wdev[k], dims, case.s[k], lengths, ws, st)
         return launches
 
     def barrier():
@@ -224,6 +247,8 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {st} flags {fl}")
 
     K = args.steps
+    if args.graph:
+        return run_graph(args, case, step, barrier, rank, world, local_rank, dev)
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(hooks)]
            for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -256,10 +281,7 @@ def run_ours(args, rank, world, local_rank):
                 stage_ms[s] += e[i].elapsed_time(e[i + 1])
     per_launch = {s: v / (K * hooks) for s, v in stage_ms.items()}
 
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
 
     # ---- end to end through host buffers
     e2e = None
@@ -282,13 +304,9 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms_e2e = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
         nbytes = h_host.numel() * h_host.element_size()
-        e2e = {"value": round(case.valid_tokens * world * K / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+        e2e = {"value": round(whole_job_rate(case.valid_tokens, world, K, ms_e2e), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                "api": "r2l_sidecar_forward via binding, pinned host hidden in/out"}
 
@@ -300,7 +318,7 @@ def run_ours(args, rank, world, local_rank):
     dom = max(per_launch, key=per_launch.get)
     line = {
         "metric": METRIC,
-        "value": round(case.valid_tokens * world * K / (ms_total * 1e-3), 1),
+        "value": round(whole_job_rate(case.valid_tokens, world, K, ms_total), 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -329,6 +347,53 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     return line
+
+
+def run_graph(args, case, step, barrier, rank, world, local_rank, dev):
+    """Time K replays of one step captured as a CUDA graph (launch overhead out
+    of the loop); the denoise-step workload is launch-bound without it."""
+    import torch
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                      # one eager call on the capture stream first
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    t0.record()
+    for _ in range(K):
+        graph.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    del graph
+    if rank != 0:
+        return None
+    hooks = len(case.weights)
+    return {
+        "metric": METRIC if args.config == 2 else f"R2L sidecar tokens/sec, {case.name}",
+        "value": round(whole_job_rate(case.valid_tokens, world, K, ms), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": case.name, "B": case.B, "L": case.L, "hooks": hooks,
+                                         "cuda_graph": True, "per_hook_us": round(ms / K / hooks * 1e3, 2)},
+        "clocks": clk, "source_sha": source_sha(),
+    }
 
 
 def _blas_threads():

@@ -137,6 +137,7 @@ CONFIG_NAMES = {
     2: "serving bf16 B=8 L=4096 d=2048 E=4096 N=16 R=128",
     3: "stack7 bf16 B=4 L=8192 d=2048 E=4096 N=16 R=128 x7 hooks",
     4: "ragged bf16 B=256 L=512 len~U[64,512] d=2048 E=4096 N=16 R=128",
+    5: "denoise-step bf16 B=8 G=128 d=2048 E=4096 N=16 R=128 x7 hooks",
 }
 
 
@@ -176,6 +177,17 @@ def make_case(cfg: int, *, B: Optional[int] = None, L: Optional[int] = None,
         h = poison_padding(make_hidden(Bv, Lv, dims.d_model, dt, seed=4), lengths)
         ws = [make_weights(dims, dt, seed=104)] if weights else []
         return Case(CONFIG_NAMES[4], dims, dt, Bv, Lv, h, ws, [0.7], lengths=lengths)
+    if cfg == 5:
+        # one denoising step of cached parallel decoding (§3.5, "Inference with
+        # prefix KV cache"): the 7 hooks run over the generation block alone,
+        # G = 128 positions of each of B = 8 requests (§4.1 throughput setup)
+        dims, dt = BIG, torch.bfloat16
+        Bv, Lv = (B or 8), (L or 128)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=5)
+        g = torch.Generator().manual_seed(5)
+        s = (torch.rand((7,), generator=g, dtype=torch.float64) * 2.0 - 1.0).tolist()
+        ws = [make_weights(dims, dt, seed=500 + k) for k in range(7)] if weights else []
+        return Case(CONFIG_NAMES[5], dims, dt, Bv, Lv, h, ws, s)
     raise ValueError(f"unknown config {cfg}")
 
 

@@ -1,0 +1,54 @@
+"""The multi-rank path of bench.py on the CPU: two gloo ranks agree on the
+slowest rank's time and on the whole-job throughput (weak scaling: every rank
+runs its own batch; sequences are independent, so no data moves between
+ranks)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        my_ms = 10.0 + 5.0 * rank             # rank 1 is the slow one
+        got = bench.max_over_ranks(my_ms, world)
+        rate = bench.whole_job_rate(1000, world, 4, got)
+        dist.barrier()
+        out[rank] = (got, rate)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 15.0
+    # 1000 tokens per rank per step, 4 steps, 2 ranks, 15 ms -> 533,333 tokens/s
+    assert res[0][1] == res[1][1] == pytest.approx(2 * 1000 * 4 / 0.015)
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.whole_job_rate(32768, 1, 10, 25.0) == pytest.approx(32768 * 10 / 0.025)
