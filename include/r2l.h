@@ -70,7 +70,10 @@ typedef enum {
 } r2l_dtype;
 
 /* r2l_dims.flags */
-#define R2L_FLAG_GENERAL_A 0x1u     /* never take the A = -(1..16) power fast path of the scan  */
+#define R2L_FLAG_GENERAL_A 0x1u     /* never take the A = -(1..16) power fast path of the scan    */
+#define R2L_FLAG_FORWARD_SCAN 0x2u  /* run the block left to right instead: causal conv and a
+                                       forward scan (the "L2R Mamba" control of Table 4); every
+                                       other step is unchanged                                    */
 /* Device status bits, reported by r2l_get_device_status(). */
 #define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */
 #define R2L_DEVFLAG_TIMEOUT 0x2u          /* a kernel gave up waiting on a pipeline barrier (results invalid) */

@@ -61,6 +61,7 @@ __all__ = [
     "sidecar_sequence",
     "sidecar_forward",
     "sidecar_stack",
+    "flip_valid",
 ]
 
 SOFTPLUS_THRESHOLD = 20.0
@@ -239,8 +240,20 @@ def sidecar_sequence(h, w, s, length=None, return_intermediates=False):
     return out
 
 
+def flip_valid(h, lengths=None):
+    """Reverse each sequence's valid prefix [0, len_b) of a right-padded batch
+    along the sequence axis (§3.4 step ❶'s flip, per sequence); padding stays."""
+    h = np.array(h, copy=True)
+    L = h.shape[1]
+    for b in range(h.shape[0]):
+        n = L if lengths is None else int(lengths[b])
+        n = min(max(n, 0), L)
+        h[b, :n] = h[b, :n][::-1]
+    return h
+
+
 def sidecar_forward(h, w, s, lengths=None, out_dtype="f64", batch_indices=None,
-                    return_intermediates=False):
+                    return_intermediates=False, direction="r2l"):
     """The hook on a right-padded batch h [B, L, d_model] (float64 values).
 
     Sequences are independent; ``batch_indices`` restricts the work to a subset
@@ -249,6 +262,16 @@ def sidecar_forward(h, w, s, lengths=None, out_dtype="f64", batch_indices=None,
     rounds h⁺ once to bfloat16; "f32" rounds once to float32; "f64" keeps it.
     """
     h = np.asarray(h, dtype=np.float64)
+    if direction == "l2r":
+        # The same block scanning left to right (the "L2R Mamba" control of
+        # Table 4): since the reverse block is flip ∘ Mamba ∘ flip (§3.4
+        # steps ❶–❸), the forward block on h is flip(R2L(flip(h))).
+        if return_intermediates:
+            raise ValueError("intermediates are reported for direction='r2l' only")
+        hf = flip_valid(h, lengths)
+        return flip_valid(sidecar_forward(hf, w, s, lengths, out_dtype, batch_indices), lengths)
+    if direction != "r2l":
+        raise ValueError(direction)
     Bsz, L, _ = h.shape
     out = np.array(h, copy=True)
     inters = {}

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libr2l.so")
 
 R2L_BF16, R2L_FP32 = 0, 1
 R2L_FLAG_GENERAL_A = 0x1
+R2L_FLAG_FORWARD_SCAN = 0x2
 R2L_DEVFLAG_LENGTH_CLAMPED = 0x1
 
 STATUS = {0: "R2L_OK", 1: "R2L_ERR_INVALID_ARG", 2: "R2L_ERR_UNSUPPORTED", 3: "R2L_ERR_ALIGNMENT",

@@ -40,6 +40,8 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 __device__ __forceinline__ float silu_hw(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 // x: row stride ldx (elements, multiple of 8); u: [B·L, E].  E % 8 == 0.
+// FWD: the causal conv of the left-to-right block (taps on x[i-k], x[j<0] = 0).
+template <bool FWD>
 __global__ void __launch_bounds__(THREADS)
 conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u, int E,
                       const float* __restrict__ conv_w, const float* __restrict__ conv_b,
@@ -64,11 +66,14 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
     bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
   }
   const long long row0 = (long long)b * L + t0;
+  // window rows: token t0 + r (reverse block) or t0 - 3 + r (forward block)
+  const int first = FWD ? t0 - 3 : t0;
   float xw[CT + 3][8];
 #pragma unroll
   for (int r = 0; r < CT + 3; ++r) {
-    if (t0 + r < n) {
-      const uint4 v = *reinterpret_cast<const uint4*>(x + (row0 + r) * ldx + c0);
+    const int tok = first + r;
+    if (tok >= 0 && tok < n) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + ((long long)b * L + tok) * ldx + c0);
       unpack8(v, xw[r]);
     } else {
 #pragma unroll
@@ -83,7 +88,7 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
     for (int ch = 0; ch < 8; ++ch) {
       float acc = bias[ch];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc = fmaf(w[ch][3 - k], xw[t + k][ch], acc);
+      for (int k = 0; k < 4; ++k) acc = fmaf(w[ch][3 - k], xw[FWD ? t + 3 - k : t + k][ch], acc);
       o[ch] = silu_hw(acc);
     }
     *reinterpret_cast<uint4*>(u + (row0 + t) * E + c0) = pack8(o);

@@ -206,6 +206,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   unsigned* err = (unsigned*)(ws + p.status);
   const size_t es = sizeof(T);
   constexpr bool kTC = std::is_same<T, bf16>::value;
+  const bool fwd = (p.flags & R2L_FLAG_FORWARD_SCAN) != 0;   // left-to-right block
 
   // a1: [x | z] = h · W_inᵀ
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
@@ -217,11 +218,14 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   if constexpr (kTC) {
     namespace cv = r2l::conv;
     dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
-    cv::conv_silu_bf16_kernel<<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+    if (fwd)
+      cv::conv_silu_bf16_kernel<true><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+    else
+      cv::conv_silu_bf16_kernel<false><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
     R2L_LAUNCH_CHECK();
   } else {
     dim3 grid((E + 127) / 128, L, B);
-    r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+    r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L, fwd);
     R2L_LAUNCH_CHECK();
   }
   // a3: [Δr | B | C] = u · W_xᵀ  (fp32 out)
@@ -256,6 +260,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
     sa.dt_mma = dt_fused ? 1 : 0;
+    sa.forward = fwd ? 1 : 0;
     sa.dr = dr; sa.lddr = R;
     sa.wdt = (const bf16*)w->dt_proj_w;
     int nl = 0;
@@ -264,7 +269,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   } else {
     dim3 grid((E + 127) / 128, B);
     r2l::scan_simple_kernel<T><<<grid, 128, 0, st>>>(u, xz + E, 2 * E, dt, dbc, p.ldd, R, w->A_log,
-                                                     w->D, w->dt_proj_b, y, E, len, L);
+                                                     w->D, w->dt_proj_b, y, E, len, L, fwd);
     R2L_LAUNCH_CHECK();
   }
   // a6: o = y · W_outᵀ
@@ -450,12 +455,14 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
     sa.carry = carry;
     sa.err = status;
     sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
+    sa.forward = (dims->flags & R2L_FLAG_FORWARD_SCAN) ? 1 : 0;
     if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
   } else {
     dim3 grid((E + 127) / 128, B);
     r2l::scan_simple_kernel<float><<<grid, 128, 0, st>>>((const float*)u, (const float*)z, ldz,
                                                          (const float*)dt_raw, bc, ldbc, 0, A_log, D, dt_b,
-                                                         (float*)y, E, len, L);
+                                                         (float*)y, E, len, L,
+                                                         (dims->flags & R2L_FLAG_FORWARD_SCAN) != 0);
     R2L_LAUNCH_CHECK();
   }
   return R2L_OK;

@@ -34,6 +34,10 @@
 //   3. chunk_scan_kernel<true>: each chunk rescans from H_in(k) and writes y.
 // With one chunk per sequence only step 3 runs, from a zero state.
 //
+// FWD runs the same block left to right (the "L2R Mamba" control of Table 4):
+// tiles stream from the chunk's left end, tokens are visited in increasing
+// order, and chunk carries flow from each chunk to the one on its right.
+//
 // Decays: exp(Δ A_m) is exp2(Δ · A_m log2 e) on the MUFU unit.  When every
 // channel of a warp has A_m = −(m+1) (the S4D-real initialisation, checked on
 // the device to 1e-5 relative), the 16 decays are the powers r, r², …, r¹⁶ of
@@ -97,6 +101,7 @@ struct Params {
   float* carry_sum;     // [B][nc][E]: Σ Δ over chunk k
   unsigned* err;
   int force_general;
+  int fwd;              // left-to-right block (chunk carry direction)
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -143,20 +148,21 @@ struct Ctx {
 // One sub-tile of SUB tokens [j0, j0 + SUB) of one channel, last token first.
 // Phase A computes what does not depend on the state (softplus, the decay
 // base, Δu, D·u, the gate) for all of its tokens; phase B runs the
-// recurrence.  FULL: every token of the sub-tile is inside the chunk.
-// dtv: the tile's 16 dt_raw values (DTMMA)
+// recurrence (tokens in decreasing order, increasing with FWD).  FULL: every
+// token of the sub-tile is inside the chunk; otherwise only tokens
+// j in [jlo, jhi) are.  dtv: the tile's 16 dt_raw values (DTMMA)
 // or unused (read sdt).  Output: y rows to shared memory (ys, stride CH) for
 // tiles stored by TMA, else to global (yg).
-template <bool FINAL, bool POW, bool FULL, bool DTMMA>
+template <bool FINAL, bool POW, bool FULL, bool DTMMA, bool FWD>
 __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& sumd, const bf16* su,
                                          const bf16* sdt, const float (&dtv)[16], const bf16* sz,
                                          const float* sbc, bf16* ys, bf16* yg, long long ldy, bool store_ok,
-                                         int j0, int jmin) {
+                                         int j0, int jlo, int jhi) {
   float dec[SUB], du[SUB], gz[SUB], Du[SUB];
 #pragma unroll
   for (int t = 0; t < SUB; ++t) {
     const int j = j0 + t;
-    if (!FULL && j < jmin) continue;
+    if (!FULL && (j < jlo || j >= jhi)) continue;
     float delta, r;
     const float raw = DTMMA ? dtv[j] : __bfloat162float(sdt[j * CH]);
     softplus_and_decay(raw + cx.dtb, delta, r);
@@ -171,9 +177,10 @@ __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& s
     }
   }
 #pragma unroll
-  for (int t = SUB - 1; t >= 0; --t) {
+  for (int tt = 0; tt < SUB; ++tt) {
+    const int t = FWD ? tt : SUB - 1 - tt;
     const int j = j0 + t;
-    if (!FULL && j < jmin) break;
+    if (!FULL && (j < jlo || j >= jhi)) continue;
     const float4* bc4 = reinterpret_cast<const float4*>(sbc + j * 32);
     const float2 du2 = make_float2(du[t], du[t]);
     float2 a[8];
@@ -224,7 +231,7 @@ __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& s
 // that lies wholly inside the chunk back with a bulk tensor store.  With
 // DTMMA it first loads the CTA's W_dt slice, and streams Δr tiles instead of
 // dt_raw tiles.
-template <bool FINAL, bool DTMMA>
+template <bool FINAL, bool DTMMA, bool FWD>
 __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUtensorMap* tm_z,
                                              const CUtensorMap* tm_dt, const CUtensorMap* tm_bc,
                                              const CUtensorMap* tm_y, const CUtensorMap* tm_w, uint8_t* smem,
@@ -258,15 +265,17 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
     if (!sm100::mbar_wait(&empty[st], ph ^ 1u, p.err)) { ok = false; break; }
     if (FINAL && it >= STAGES) {
-      const int tb = e0 - (it - STAGES + 1) * TS;     // first position of the tile just finished
-      if (tb >= s0) {                                 // whole tile inside the chunk: y sits in s_y
+      const int pt = it - STAGES;                     // the tile just finished in this slot
+      const int tb = FWD ? s0 + pt * TS : e0 - (pt + 1) * TS;
+      if (FWD ? tb + TS <= e0 : tb >= s0) {           // whole tile inside the chunk: y sits in s_y
         sm100::tma_store_2d(tm_y, s_y + st * TS * CH, cb * CH, b * p.L + tb);
         sm100::bulk_commit();
         sm100::bulk_wait_read_all();                  // s_y[st] is rewritten STAGES tiles later
       }
     }
     if (it < ntiles) {
-      const int row0 = b * p.L + e0 - (it + 1) * TS;  // may be negative for b = 0: reads zeros
+      // may start before row 0 (reverse, b = 0) or run past the last row (FWD): reads zeros
+      const int row0 = b * p.L + (FWD ? s0 + it * TS : e0 - (it + 1) * TS);
       sm100::mbar_arrive_expect_tx(&full[st], bytes);
       sm100::tma_load_2d(s_u + st * TS * CH, tm_u, cb * CH, row0, &full[st]);
       if (DTMMA) {
@@ -315,7 +324,7 @@ __device__ __forceinline__ void run_dt_mma(uint8_t* smem, uint32_t tmem_base, ui
   sm100::mbar_wait(drain, 0, err, 1000000000ull);
 }
 
-template <bool FINAL, bool DTMMA>
+template <bool FINAL, bool DTMMA, bool FWD>
 __global__ void __launch_bounds__(Smem<DTMMA>::THREADS, 2)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
@@ -376,7 +385,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
 
   if (warp == CWARPS) {
     if (lane == 0)
-      run_producer<FINAL, DTMMA>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b, cb, s0,
+      run_producer<FINAL, DTMMA, FWD>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b, cb, s0,
                                  e0, ntiles, p);
     return;   // the producer warp takes no part in the teardown below
   }
@@ -429,28 +438,31 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
       sm100::tc_fence_after();
       sm100::tmem_ld16(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(st * TS), dtv);
     }
-    const int tbase = e0 - (it + 1) * TS;        // sequence position of tile row 0
-    const int jmin = s0 > tbase ? s0 - tbase : 0;
+    const int tbase = FWD ? s0 + it * TS : e0 - (it + 1) * TS;   // sequence position of tile row 0
+    const int jlo = (!FWD && s0 > tbase) ? s0 - tbase : 0;       // tokens [jlo, jhi) are in the chunk
+    const int jhi = (FWD && e0 - tbase < TS) ? e0 - tbase : TS;
+    const bool full = jlo == 0 && jhi == TS;
     const bf16* su = s_u + st * TS * CH + ch;
     const bf16* sdt = s_dt + st * TS * CH + ch;
     const bf16* sz = s_z + st * TS * CH + ch;
     const float* sbc = s_bc + st * TS * 32;
     // full tiles go out through shared memory and a TMA store; a tile that
-    // crosses the chunk's left edge is written row by row
-    bf16* ys = jmin == 0 ? s_y + st * TS * CH + ch : nullptr;
+    // crosses the chunk's edge is written row by row
+    bf16* ys = full ? s_y + st * TS * CH + ch : nullptr;
     bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
 #pragma unroll
-    for (int j0 = TS - SUB; j0 >= 0; j0 -= SUB) {
-      if (jmin == 0) {
+    for (int sb = 0; sb < TS / SUB; ++sb) {
+      const int j0 = FWD ? sb * SUB : TS - SUB - sb * SUB;
+      if (full) {
         if (use_pow)
-          scan_sub<FINAL, true, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
+          scan_sub<FINAL, true, true, DTMMA, FWD>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0, TS);
         else
-          scan_sub<FINAL, false, true, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0);
-      } else if (j0 + SUB > jmin) {
+          scan_sub<FINAL, false, true, DTMMA, FWD>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, 0, TS);
+      } else if (j0 + SUB > jlo && j0 < jhi) {
         if (use_pow)
-          scan_sub<FINAL, true, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+          scan_sub<FINAL, true, false, DTMMA, FWD>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jlo, jhi);
         else
-          scan_sub<FINAL, false, false, DTMMA>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jmin);
+          scan_sub<FINAL, false, false, DTMMA, FWD>(cx, H, sumd, su, sdt, dtv, sz, sbc, ys, yg, p.ldy, cvalid, j0, jlo, jhi);
       }
     }
     if (FINAL && ys) sm100::fence_proxy_async_smem();   // make the y tile visible to the TMA store
@@ -472,7 +484,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
 }
 
 // Per (sequence, channel): turn chunk end states S_k into the states entering
-// each chunk from the right, in place (see the header comment, step 2).
+// each chunk from the right (from the left with fwd), in place (see the
+// header comment, step 2).
 __global__ void chunk_carry_kernel(const Params p) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
@@ -486,7 +499,8 @@ __global__ void chunk_carry_kernel(const Params p) {
     A[m] = -expf(p.A_log[c * 16 + m]);
     carry[m] = 0.0f;
   }
-  for (int k = nk - 1; k >= 0; --k) {
+  for (int kk = 0; kk < nk; ++kk) {
+    const int k = p.fwd ? kk : nk - 1 - kk;   // from the chunk the state enters first
     float4* S = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
     const float sd = p.carry_sum[((long long)b * p.nc + k) * p.E + c];
     float s[16];

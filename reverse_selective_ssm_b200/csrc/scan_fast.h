@@ -28,6 +28,7 @@ struct ScanArgs {
   unsigned* err;                               // device status word
   int force_general;                           // never use the A = -(1..16) power path
   int dt_mma;                                  // compute dt_raw = Δr·W_dtᵀ inside the scan (dt_rank 128)
+  int forward;                                 // left-to-right block
 };
 
 // Tokens per chunk chosen from the shape alone (deterministic, no device query).

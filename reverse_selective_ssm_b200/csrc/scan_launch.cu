@@ -40,13 +40,13 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
 
 namespace {
 
-template <bool FINAL, bool DTMMA>
+template <bool FINAL, bool DTMMA, bool FWD>
 cudaError_t prep_kernel() {
-  return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, DTMMA>,
+  return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, DTMMA, FWD>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rscan::Smem<DTMMA>::BYTES);
 }
 
-template <bool DTMMA>
+template <bool DTMMA, bool FWD>
 cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
   using namespace rscan;
   using Sm = Smem<DTMMA>;
@@ -66,17 +66,17 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
     tw = tdt;
   }
   cudaError_t e;
-  if ((e = prep_kernel<true, DTMMA>()) != cudaSuccess) return e;
+  if ((e = prep_kernel<true, DTMMA, FWD>()) != cudaSuccess) return e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
   if (nc > 1) {
-    if ((e = prep_kernel<false, DTMMA>()) != cudaSuccess) return e;
-    chunk_scan_kernel<false, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+    if ((e = prep_kernel<false, DTMMA, FWD>()) != cudaSuccess) return e;
+    chunk_scan_kernel<false, DTMMA, FWD><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     if (launches) *launches += 2;
   }
-  chunk_scan_kernel<true, DTMMA><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+  chunk_scan_kernel<true, DTMMA, FWD><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;
@@ -109,11 +109,12 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.carry_sum = a.carry ? a.carry + (size_t)a.B * nc * a.E * 16 : nullptr;
   p.err = a.err;
   p.force_general = a.force_general;
+  p.fwd = a.forward;
   if (a.dt_mma) {
     if (!a.dr || !a.wdt || (a.lddr % 8)) return cudaErrorInvalidValue;
-    return launch<true>(a, p, nc, st, launches);
+    return a.forward ? launch<true, true>(a, p, nc, st, launches) : launch<true, false>(a, p, nc, st, launches);
   }
-  return launch<false>(a, p, nc, st, launches);
+  return a.forward ? launch<false, true>(a, p, nc, st, launches) : launch<false, false>(a, p, nc, st, launches);
 }
 
 }  // namespace r2l

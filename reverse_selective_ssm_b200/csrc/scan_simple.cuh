@@ -1,5 +1,6 @@
 // Sequential reverse selective scan: one thread per (sequence b, channel c),
-// walking i = len_b-1 … 0 with the d_state = 16 state in registers.  Used for
+// walking i = len_b-1 … 0 (or 0 … len_b-1 for the left-to-right block, fwd)
+// with the d_state = 16 state in registers.  Used for
 // the fp32 path (config-0 sizes) where parallelism is not the point.
 //
 // "Bifocal Diffusion Language Models" (arXiv 2606.27732v1), §3.4 step ❷ (the
@@ -19,7 +20,8 @@ __global__ void scan_simple_kernel(const T* __restrict__ u, const T* __restrict_
                                    const T* __restrict__ dt_raw, const float* __restrict__ dbc,
                                    int ldd, int R, const float* __restrict__ A_log,
                                    const float* __restrict__ Dv, const float* __restrict__ dt_b,
-                                   T* __restrict__ y, int E, const int* __restrict__ len, int L) {
+                                   T* __restrict__ y, int E, const int* __restrict__ len, int L,
+                                   bool fwd) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
   if (c >= E) return;
@@ -31,7 +33,8 @@ __global__ void scan_simple_kernel(const T* __restrict__ u, const T* __restrict_
     H[m] = 0.0f;
   }
   const float Dc = Dv[c], bc = dt_b[c];
-  for (int i = n - 1; i >= 0; --i) {
+  for (int step = 0; step < n; ++step) {
+    const int i = fwd ? step : n - 1 - step;     // fwd: the left-to-right block
     const long long row = (long long)b * L + i;
     const float uu = to_f32(u[row * E + c]);
     const float delta = softplus_f(to_f32(dt_raw[row * E + c]) + bc);

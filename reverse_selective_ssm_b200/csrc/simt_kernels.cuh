@@ -94,10 +94,12 @@ gemm_simt_kernel(const TA* __restrict__ A, int lda, const TW* __restrict__ W, in
 //   u[i, c] = SiLU(conv_b[c] + Σ_{k=0..3} conv_w[c, 3-k] · x[i+k, c]),  x[j] = 0 for j ≥ len.
 // x is read from the in_proj output (row stride ldx).  One thread per (b, i, c).
 // ---------------------------------------------------------------------------
+// fwd = true: the causal conv of the left-to-right block instead,
+//   u[i, c] = SiLU(conv_b[c] + Σ_{k=0..3} conv_w[c, 3-k] · x[i-k, c]),  x[j] = 0 for j < 0.
 template <typename T>
 __global__ void conv_silu_kernel(const T* __restrict__ x, int ldx, T* __restrict__ u, int E,
                                  const float* __restrict__ conv_w, const float* __restrict__ conv_b,
-                                 const int* __restrict__ len, int L) {
+                                 const int* __restrict__ len, int L, bool fwd) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int i = blockIdx.y;
   const int b = blockIdx.z;
@@ -106,8 +108,10 @@ __global__ void conv_silu_kernel(const T* __restrict__ x, int ldx, T* __restrict
   const long long row = (long long)b * L + i;
   float acc = conv_b[c];
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    if (i + k < n) acc = fmaf(conv_w[c * 4 + 3 - k], to_f32(x[(row + k) * ldx + c]), acc);
+  for (int k = 0; k < 4; ++k) {
+    const int j = fwd ? i - k : i + k;
+    if (j >= 0 && j < n) acc = fmaf(conv_w[c * 4 + 3 - k], to_f32(x[((long long)b * L + j) * ldx + c]), acc);
+  }
   u[row * E + c] = from_f32<T>(silu_f(acc));
 }
 

@@ -355,9 +355,29 @@ def pin_stack_composition(O):
     assert np.array_equal(got, cur)
 
 
+def pin_l2r_direction(O):
+    """The left-to-right control equals a forward Mamba block written with
+    torch ops (no flip involved), and a change at position j reaches only
+    positions >= j."""
+    rng = RNG(15)
+    w = tiny_weights(rng)
+    B, L, d = 2, 9, w["W_in"].shape[1]
+    lengths = [9, 5]
+    h = rng.normal(size=(B, L, d))
+    got = O.sidecar_forward(h, w, 0.6, lengths=lengths, direction="l2r")
+    for b, n in enumerate(lengths):
+        want = h[b, :n] + np.tanh(0.6) * forward_mamba_block_l2r(h[b, :n], w)
+        _close(got[b, :n], want, 1e-11, f"l2r b={b}")
+        assert np.array_equal(got[b, n:], h[b, n:])
+    h2 = h.copy()
+    h2[0, 6:] += 1.0
+    out2 = O.sidecar_forward(h2, w, 0.6, lengths=lengths, direction="l2r")
+    assert np.array_equal(out2[0, :6], got[0, :6]), "left-to-right: positions < 6 must not change"
+
+
 ALL_PINS = [
     pin_activations, pin_round_bf16, pin_in_proj_split, pin_x_proj_split, pin_dt,
     pin_conv, pin_scan_bruteforce, pin_scan_special_cases, pin_layer_norm, pin_gate,
     pin_flip_equivalence, pin_s_zero_identity, pin_right_context_only,
-    pin_ragged_isolation, pin_stack_composition,
+    pin_ragged_isolation, pin_stack_composition, pin_l2r_direction,
 ]

@@ -128,3 +128,42 @@ def test_scan_long_sequence_many_chunks():
     whole = run_scan(inp, B, L, E, None, 1 << 20)
     check(auto, want, B, L, None, 5e-3)
     check(whole, want, B, L, None, 5e-3)
+
+
+def oracle_scan_forward(inp, B, L, E, lengths):
+    """The left-to-right scan through the reverse oracle on flipped data."""
+    f = S.to_f64
+    u, z, dt_raw, bc = f(inp["u"]), f(inp["z"])[:, :E], f(inp["dt_raw"]), f(inp["bc"])
+    A = -np.exp(f(inp["A_log"]))
+    delta_all = O.softplus(dt_raw + f(inp["dt_b"]))
+    out = np.full((B * L, E), np.nan)
+    for b in range(B):
+        n = L if lengths is None else int(lengths[b])
+        if n == 0:
+            continue
+        r = slice(b * L, b * L + n)
+        fl = lambda a: a[r][::-1]
+        yf = O.reverse_selective_scan(fl(u), fl(delta_all), A, fl(bc[:, :16]), fl(bc[:, 16:32]), f(inp["D"]), fl(z))
+        out[r] = yf[::-1]
+    return out
+
+
+@pytest.mark.parametrize("chunk_tokens", [0, 48, 100000])
+@pytest.mark.parametrize("structured", [True, False])
+def test_scan_forward_direction(chunk_tokens, structured):
+    """R2L_FLAG_FORWARD_SCAN: the left-to-right scan (Table 4's control)."""
+    B, L, E = 3, 301, 384
+    lengths = [301, 1, 170]
+    inp = make_scan_inputs(B, L, E, seed=71 + structured, structured_A=structured)
+    got = run_scan(inp, B, L, E, lengths, chunk_tokens, flags=bd.R2L_FLAG_FORWARD_SCAN)
+    want = oracle_scan_forward(inp, B, L, E, lengths)
+    check(got, want, B, L, lengths, 5e-3)
+
+
+def test_scan_forward_fp32():
+    B, L, E = 2, 77, 136
+    lengths = [77, 40]
+    inp = make_scan_inputs(B, L, E, seed=81, structured_A=False, dtype=torch.float32)
+    got = run_scan(inp, B, L, E, lengths, 0, dtype=torch.float32, flags=bd.R2L_FLAG_FORWARD_SCAN)
+    want = oracle_scan_forward(inp, B, L, E, lengths)
+    check(got, want, B, L, lengths, 1e-5)
