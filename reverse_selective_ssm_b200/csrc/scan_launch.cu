@@ -40,6 +40,17 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
 
 namespace {
 
+// B|C delivered through tensor memory in the fused-dt_proj scan (0: shared memory).
+#ifndef R2L_SCAN_BCT
+#define R2L_SCAN_BCT 1
+#endif
+
+template <bool FINAL, bool FWD>
+cudaError_t prep_bct_kernel() {
+  return cudaFuncSetAttribute(rscan::chunk_scan_bct_kernel<FINAL, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)rscan::SmemBct::BYTES);
+}
+
 template <bool FINAL, bool DTMMA, bool FWD>
 cudaError_t prep_kernel() {
   return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, DTMMA, FWD>,
@@ -66,8 +77,24 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
     tw = tdt;
   }
   cudaError_t e;
-  if ((e = prep_kernel<true, DTMMA, FWD>()) != cudaSuccess) return e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
+  if (DTMMA && R2L_SCAN_BCT) {
+    using Sb = SmemBct;
+    if ((e = prep_bct_kernel<true, FWD>()) != cudaSuccess) return e;
+    if (nc > 1) {
+      if ((e = prep_bct_kernel<false, FWD>()) != cudaSuccess) return e;
+      chunk_scan_bct_kernel<false, FWD><<<grid, Sb::THREADS, Sb::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+      if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+      chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
+      if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+      if (launches) *launches += 2;
+    }
+    chunk_scan_bct_kernel<true, FWD><<<grid, Sb::THREADS, Sb::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (launches) *launches += 1;
+    return cudaSuccess;
+  }
+  if ((e = prep_kernel<true, DTMMA, FWD>()) != cudaSuccess) return e;
   if (nc > 1) {
     if ((e = prep_kernel<false, DTMMA, FWD>()) != cudaSuccess) return e;
     chunk_scan_kernel<false, DTMMA, FWD><<<grid, Sm::THREADS, Sm::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
