@@ -3,7 +3,8 @@
 // ("Bifocal Diffusion Language Models", arXiv 2606.27732v1, §3.4 steps ❶–❷:
 // the Mamba-1 causal conv seen through the flip).  One thread covers 8
 // channels (16-byte loads and stores) × CT consecutive tokens and keeps the
-// CT + 3 input rows it needs in registers.
+// CT + 3 input rows it needs in registers (as packed bf16, unpacked per use),
+// all requested before the first output is computed.
 #pragma once
 
 #include "common.cuh"
@@ -11,7 +12,7 @@
 namespace r2l {
 namespace conv {
 
-constexpr int CT = 8;        // tokens per thread
+constexpr int CT = 16;       // tokens per thread
 constexpr int THREADS = 128;
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -68,27 +69,27 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
   const long long row0 = (long long)b * L + t0;
   // window rows: token t0 + r (reverse block) or t0 - 3 + r (forward block)
   const int first = FWD ? t0 - 3 : t0;
-  float xw[CT + 3][8];
+  uint4 xr[CT + 3];
 #pragma unroll
   for (int r = 0; r < CT + 3; ++r) {
     const int tok = first + r;
-    if (tok >= 0 && tok < n) {
-      const uint4 v = *reinterpret_cast<const uint4*>(x + ((long long)b * L + tok) * ldx + c0);
-      unpack8(v, xw[r]);
-    } else {
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) xw[r][ch] = 0.0f;
-    }
+    xr[r] = (tok >= 0 && tok < n) ? *reinterpret_cast<const uint4*>(x + ((long long)b * L + tok) * ldx + c0)
+                                  : make_uint4(0u, 0u, 0u, 0u);
   }
+  // rolling window of 4 unpacked rows: win[k] holds window row t + k
+  float win[4][8];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) unpack8(xr[k], win[k]);
 #pragma unroll
   for (int t = 0; t < CT; ++t) {
+    unpack8(xr[t + 3], win[(t + 3) & 3]);
     if (t0 + t >= n) break;
     float o[8];
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
       float acc = bias[ch];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc = fmaf(w[ch][3 - k], xw[FWD ? t + 3 - k : t + k][ch], acc);
+      for (int k = 0; k < 4; ++k) acc = fmaf(w[ch][3 - k], win[((FWD ? 3 - k : k) + t) & 3][ch], acc);
       o[ch] = silu_hw(acc);
     }
     *reinterpret_cast<uint4*>(u + (row0 + t) * E + c0) = pack8(o);

@@ -192,13 +192,23 @@ ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const 
   if ((int)(row - b * L) >= len[b]) return;
   const bf16* orow = o + row * d;
   bf16* hrow = h + row * d;
+  // both rows are requested before any arithmetic, so a warp keeps 8 KB in flight
+  uint4 oraw[NV], hraw_all[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int col = (k * 32 + lane) * 8;
+    if (col < d) {
+      oraw[k] = *reinterpret_cast<const uint4*>(orow + col);
+      hraw_all[k] = *reinterpret_cast<const uint4*>(hrow + col);
+    }
+  }
   float v[NV][8];
   float s = 0.0f;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int col = (k * 32 + lane) * 8;
     if (col < d) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(orow + col);
+      const uint4 raw = oraw[k];
       const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -252,7 +262,7 @@ ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const 
       dst[0] = make_float4(hv[0], hv[1], hv[2], hv[3]);
       dst[1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
     }
-    uint4 hraw = *reinterpret_cast<const uint4*>(hrow + col);
+    uint4 hraw = hraw_all[k];
     __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&hraw);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
