@@ -64,9 +64,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha():
+# The sources each stage's kernel is built from (a profile of that kernel stays
+# valid while these files are unchanged).
+_COMMON = ["common.cuh", "sm100_primitives.cuh", "tmap.cu", "tmap.h"]
+STAGE_SOURCES = {
+    "in_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
+    "x_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
+    "dt_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
+    "out_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
+    "conv": ["conv_fast.cuh"] + _COMMON,
+    "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu"] + _COMMON,
+    "ln_residual": ["simt_kernels.cuh"] + _COMMON,
+}
+
+
+def source_sha(stage=None):
+    """Hash of the kernel sources: of one stage's files, or of all of them."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "reverse_selective_ssm_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "reverse_selective_ssm_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*"))) if stage is None else \
+        [os.path.join(csrc, f) for f in sorted(STAGE_SOURCES[stage])]
+    for f in files:
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
@@ -81,7 +99,7 @@ def read_traffic(stage, workload_tag):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
         if kv.get("stage") == stage and kv.get("workload") == workload_tag and \
-                kv.get("source_sha") == source_sha() and "dram_bytes_per_launch" in kv:
+                kv.get("source_sha") == source_sha(stage) and "dram_bytes_per_launch" in kv:
             try:
                 return float(kv["dram_bytes_per_launch"])
             except ValueError:
@@ -152,15 +170,21 @@ def algorithmic(case, stage):
     if stage == "conv":
         return "hbm", float(T) * E * (a + a), "byte"
     if stage == "scan":
-        # u, z read and y written (act) + B, C read (fp32), plus either the dt_raw
-        # row (act) or, when dt_proj runs inside the scan (bf16, dt_rank 128),
-        # the dt_rank-wide Δr row (bf16)
-        fused = a == 2 and R == 128
-        dt_bytes = R * 2 if fused else E * a
-        return "hbm", float(T) * (E * 3 * a + dt_bytes + 2 * N * 4), "byte"
+        # the step's bytes per token as the scope table counts them: u, z and
+        # dt_raw read, y written (activation dtype) + B, C read (fp32)
+        return "hbm", float(T) * (E * 4 * a + 2 * N * 4), "byte"
     if stage == "ln_residual":  # o read, h read, h written
         return "hbm", float(T) * d * 3 * a, "byte"
     raise KeyError(stage)
+
+
+def scan_kernel_bytes(case):
+    """Bytes the scan kernel itself moves per launch: with dt_proj inside it
+    (bf16, dt_rank 128) it reads the dt_rank-wide Δr row instead of dt_raw."""
+    E, R, N = case.dims.d_inner, case.dims.dt_rank, case.dims.d_state
+    a = 2 if case.dtype.itemsize == 2 else 4
+    dt_bytes = R * 2 if (a == 2 and R == 128) else E * a
+    return float(case.valid_tokens) * (E * 3 * a + dt_bytes + 2 * N * 4)
 
 
 def roofline_obj(case, stage, ms, peaks, peak_kind, workload_tag):
@@ -175,10 +199,15 @@ def roofline_obj(case, stage, ms, peaks, peak_kind, workload_tag):
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
         peak_note = f"{peak_kind} HBM copy"
-    return {"kernel": stage, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "peak_source": peak_note,
-            "algorithmic_per_launch": amount, "ms_per_launch": round(ms, 5),
-            "traffic": read_traffic(stage, workload_tag)}
+    obj = {"kernel": stage, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+           "frac": round(achieved / peak, 4), "peak_source": peak_note,
+           "algorithmic_per_launch": amount, "ms_per_launch": round(ms, 5),
+           "traffic": read_traffic(stage, workload_tag)}
+    if stage == "scan":
+        kb = scan_kernel_bytes(case)
+        obj["kernel_bytes_per_launch"] = kb
+        obj["frac_of_kernel_bytes"] = round(kb / (ms * 1e-3) / 1e9 / peak, 4)
+    return obj
 
 
 # ---------------------------------------------------------------- ranks
