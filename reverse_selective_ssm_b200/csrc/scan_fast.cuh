@@ -230,7 +230,7 @@ __device__ __forceinline__ void scan_sub(const Ctx& cx, float2 (&H)[8], float& s
 // that lies wholly inside the chunk back with a bulk tensor store.  With
 // DTMMA it first loads the CTA's W_dt slice, and streams Δr tiles instead of
 // dt_raw tiles.
-template <class S, bool FINAL, bool DTMMA, bool FWD>
+template <class S, bool FINAL, bool DTMMA, bool FWD, int CHN = CH>
 __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUtensorMap* tm_z,
                                              const CUtensorMap* tm_dt, const CUtensorMap* tm_bc,
                                              const CUtensorMap* tm_y, const CUtensorMap* tm_w, uint8_t* smem,
@@ -250,11 +250,12 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
   }
   if (DTMMA) {
     sm100::prefetch_tmap(tm_w);
-    sm100::mbar_arrive_expect_tx(wfull, W_SLICE);
+    sm100::mbar_arrive_expect_tx(wfull, (uint32_t)(CHN * DT_R * 2));
     for (int a = 0; a < DT_R / 64; ++a)
-      sm100::tma_load_2d(smem + S::W + a * (CH * 128), tm_w, a * 64, cb * CH, wfull);
+      sm100::tma_load_2d(smem + S::W + a * (CHN * 128), tm_w, a * 64, cb * CHN, wfull);
   }
-  constexpr uint32_t bytes = (FINAL ? 2 : 1) * ACT_TILE + BC_TILE + (DTMMA ? DR_TILE : ACT_TILE);
+  constexpr uint32_t act = TS * CHN * 2;
+  constexpr uint32_t bytes = (FINAL ? 2 : 1) * act + BC_TILE + (DTMMA ? DR_TILE : act);
   int issued = 0;
   bool ok = true;
   const int iters = ntiles + (FINAL ? STAGES : 0);
@@ -266,7 +267,7 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
       const int pt = it - STAGES;                     // the tile just finished in this slot
       const int tb = FWD ? s0 + pt * TS : e0 - (pt + 1) * TS;
       if (FWD ? tb + TS <= e0 : tb >= s0) {           // whole tile inside the chunk: y sits in s_y
-        sm100::tma_store_2d(tm_y, s_y + st * TS * CH, cb * CH, b * p.L + tb);
+        sm100::tma_store_2d(tm_y, s_y + st * TS * CHN, cb * CHN, b * p.L + tb);
         sm100::bulk_commit();
         sm100::bulk_wait_read_all();                  // s_y[st] is rewritten STAGES tiles later
       }
@@ -275,14 +276,14 @@ __device__ __forceinline__ void run_producer(const CUtensorMap* tm_u, const CUte
       // may start before row 0 (reverse, b = 0) or run past the last row (FWD): reads zeros
       const int row0 = b * p.L + (FWD ? s0 + it * TS : e0 - (it + 1) * TS);
       sm100::mbar_arrive_expect_tx(&full[st], bytes);
-      sm100::tma_load_2d(s_u + st * TS * CH, tm_u, cb * CH, row0, &full[st]);
+      sm100::tma_load_2d(s_u + st * TS * CHN, tm_u, cb * CHN, row0, &full[st]);
       if (DTMMA) {
         uint8_t* dr = smem + S::DR + st * DR_TILE;
         for (int a = 0; a < DT_R / 64; ++a) sm100::tma_load_2d(dr + a * (TS * 128), tm_dt, a * 64, row0, &full[st]);
       } else {
-        sm100::tma_load_2d(s_dt + st * TS * CH, tm_dt, cb * CH, row0, &full[st]);
+        sm100::tma_load_2d(s_dt + st * TS * CHN, tm_dt, cb * CHN, row0, &full[st]);
       }
-      if (FINAL) sm100::tma_load_2d(s_z + st * TS * CH, tm_z, cb * CH, row0, &full[st]);
+      if (FINAL) sm100::tma_load_2d(s_z + st * TS * CHN, tm_z, cb * CHN, row0, &full[st]);
       sm100::tma_load_2d(s_bc + st * TS * 32, tm_bc, 0, row0, &full[st]);
       ++issued;
     }

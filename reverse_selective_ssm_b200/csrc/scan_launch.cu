@@ -4,6 +4,7 @@
 
 #include "scan_fast.cuh"
 #include "scan_fast.h"
+#include "scan_pair.cuh"
 #include "tmap.h"
 
 namespace r2l {
@@ -45,6 +46,35 @@ namespace {
 #define R2L_SCAN_BCT 1
 #endif
 
+// Two threads per channel for single-pass scans with dt_proj fused (0: off).
+#ifndef R2L_SCAN_PAIR
+#define R2L_SCAN_PAIR 1
+#endif
+
+template <bool FWD>
+cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, cudaStream_t st, int* launches) {
+  using namespace rscan;
+  using Sp = pair::SmemPair;
+  constexpr int CHP = pair::CHP;
+  const long long M = (long long)a.B * a.L;
+  CUtensorMap tu, tz, tdr, tbc, ty, tw;
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CHP, TS, 0) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CHP, TS, 0) ||
+      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, 0) ||
+      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, CHP, TS, 0) ||
+      !make_tmap_2d(&tdr, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, 128) ||
+      !make_tmap_2d(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CHP, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(pair::scan_pair_kernel<FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Sp::BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.E + CHP - 1) / CHP, 1, a.B);
+  pair::scan_pair_kernel<FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaSuccess;
+}
+
 template <bool FINAL, bool FWD>
 cudaError_t prep_bct_kernel() {
   return cudaFuncSetAttribute(rscan::chunk_scan_bct_kernel<FINAL, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -78,6 +108,7 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
   }
   cudaError_t e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
+  if (DTMMA && R2L_SCAN_PAIR && nc == 1) return launch_pair<FWD>(a, p, st, launches);
   if (DTMMA && R2L_SCAN_BCT) {
     using Sb = SmemBct;
     if ((e = prep_bct_kernel<true, FWD>()) != cudaSuccess) return e;
