@@ -18,6 +18,11 @@
 #include "scan_fast.h"
 #include "conv_fast.cuh"
 
+// conv + SiLU fused into the x_proj GEMM on the bf16 path (0: separate kernels).
+#ifndef R2L_CONVX
+#define R2L_CONVX 1
+#endif
+
 #include <type_traits>
 
 using r2l::bf16;
@@ -212,26 +217,42 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
   prof->launches++;
   R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
-  // a2: u = SiLU(anti-causal conv(x))
+  // a2: u = SiLU(anti-causal conv(x)); a3: [Δr | B | C] = u · W_xᵀ (fp32 out).
+  // bf16 with an x_proj of 160 columns: one kernel does both (the conv runs
+  // in x_proj's operand producer and u is written once, for the scan).
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
-  prof->launches++;
+  bool convx_done = false;
   if constexpr (kTC) {
-    namespace cv = r2l::conv;
-    dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
-    if (fwd)
-      cv::conv_silu_bf16_kernel<true><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
-    else
-      cv::conv_silu_bf16_kernel<false><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
-    R2L_LAUNCH_CHECK();
-  } else {
-    dim3 grid((E + 127) / 128, L, B);
-    r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L, fwd);
-    R2L_LAUNCH_CHECK();
+    if (R2L_CONVX && r2l::convx_supported(p.ldd, E)) {
+      R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
+      prof->launches++;
+      r2l::ConvX c{};
+      c.x = (const bf16*)xz; c.ldx = 2LL * E; c.conv_w = w->conv_w; c.conv_b = w->conv_b;
+      c.u = (bf16*)u; c.ldu = E; c.W = (const bf16*)w->x_proj_w; c.C = dbc; c.ldc = p.ldd;
+      c.C2 = dr; c.ldc2 = R; c.c2_cols = R; c.M = (int)M; c.E = E; c.len = len; c.L = L; c.err = err; c.fwd = fwd;
+      if (r2l::convx_gemm(c, st) != cudaSuccess) return R2L_ERR_CUDA;
+      convx_done = true;
+    }
   }
-  // a3: [Δr | B | C] = u · W_xᵀ  (fp32 out)
-  R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
-  prof->launches++;
-  R2L_TRY(proj(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, err, st, dr, R, R));
+  if (!convx_done) {
+    prof->launches++;
+    if constexpr (kTC) {
+      namespace cv = r2l::conv;
+      dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
+      if (fwd)
+        cv::conv_silu_bf16_kernel<true><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+      else
+        cv::conv_silu_bf16_kernel<false><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+      R2L_LAUNCH_CHECK();
+    } else {
+      dim3 grid((E + 127) / 128, L, B);
+      r2l::conv_silu_kernel<T><<<grid, 128, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L, fwd);
+      R2L_LAUNCH_CHECK();
+    }
+    R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
+    prof->launches++;
+    R2L_TRY(proj(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, err, st, dr, R, R));
+  }
   // a4: dt_raw = Δr · W_dtᵀ  (bias + softplus applied in the scan)
   R2L_TRY(prof->mark(R2L_STAGE_DT_PROJ, st));
   prof->launches++;

@@ -2,6 +2,7 @@
 // tile-width choice and the persistent launch (one CTA per SM).
 #include <cuda.h>
 
+#include "gemm_convx.cuh"
 #include "gemm_tc.cuh"
 #include "tc_gemm.h"
 #include "tmap.h"
@@ -45,7 +46,39 @@ cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
   return launch<256, TOut>(g, st);
 }
 
+template <bool FWD>
+cudaError_t launch_convx(const ConvX& g, cudaStream_t st) {
+  namespace cx = convx;
+  CUtensorMap tx, tb, tc, tw4, tcb;
+  if (!make_tmap_2d(&tx, g.x, 2, g.E, g.M, g.ldx * 2, cx::BK, cx::XR, 0) ||
+      !make_tmap_2d(&tb, g.W, 2, g.E, cx::BN, (long long)g.E * 2, cx::BK, cx::BN, 128) ||
+      !make_tmap_2d(&tc, g.C, 4, cx::BN, g.M, (long long)g.ldc * 4, 32, 32, 128) ||
+      !make_tmap_2d(&tw4, g.conv_w, 4, 4, g.E, 16, 4, cx::BK, 0) ||
+      !make_tmap_2d(&tcb, g.conv_b, 4, g.E, 1, (long long)g.E * 4, cx::BK, 1, 0))
+    return cudaErrorInvalidValue;
+  auto kern = cx::gemm_convx_kernel<FWD>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cx::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const long long tiles = (g.M + cx::BM - 1) / cx::BM;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (grid <= 0) return cudaSuccess;
+  cx::Args a;
+  a.x = g.x; a.ldx = g.ldx; a.conv_w = g.conv_w; a.conv_b = g.conv_b; a.u = g.u; a.ldu = g.ldu;
+  a.M = g.M; a.K = g.E; a.C2 = g.C2; a.ldc2 = g.ldc2; a.c2_cols = g.c2_cols; a.len = g.len; a.L = g.L;
+  a.err = g.err;
+  kern<<<grid, cx::THREADS, cx::SMEM_BYTES, st>>>(tx, tb, tc, tw4, tcb, a);
+  return cudaPeekAtLastError();
+}
+
 }  // namespace
+
+bool convx_supported(int N, int E) { return N == convx::BN && E > 0 && E % convx::BK == 0; }
+
+cudaError_t convx_gemm(const ConvX& g, cudaStream_t st) {
+  if (g.M <= 0) return cudaSuccess;
+  if (!convx_supported(160, g.E) || (g.ldx % 8) || (g.ldu % 2) || (g.ldc * 4) % 16) return cudaErrorInvalidValue;
+  return g.fwd ? launch_convx<true>(g, st) : launch_convx<false>(g, st);
+}
 
 cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;

@@ -26,4 +26,30 @@ struct TcGemm {
 // Enqueues the GEMM on `st`.  Requires lda, ldb, K to be multiples of 8.
 cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st);
 
+// conv + SiLU fused into x_proj (gemm_convx.cuh): u = SiLU(conv(x)) written to
+// `u` for the valid rows, and [Δr | B | C] = u·W_xᵀ into C (fp32), Δr also into
+// C2 (bf16).  For N = 160 (dt_rank 128, d_state 16) and E a multiple of 64.
+struct ConvX {
+  const __nv_bfloat16* x;  // [M, E] row stride ldx (the x half of xz)
+  long long ldx;
+  const float* conv_w;     // [E, 4]
+  const float* conv_b;     // [E]
+  __nv_bfloat16* u;        // [M, E] row stride ldu
+  long long ldu;
+  const __nv_bfloat16* W;  // x_proj weight [160, E]
+  float* C;                // [M, 160]
+  int ldc;
+  __nv_bfloat16* C2;       // [M, ldc2], columns < c2_cols
+  int ldc2;
+  int c2_cols;
+  int M, E;
+  const int* len;
+  int L;
+  unsigned* err;
+  bool fwd;                // causal conv of the left-to-right block
+};
+
+bool convx_supported(int N, int E);
+cudaError_t convx_gemm(const ConvX& g, cudaStream_t st);
+
 }  // namespace r2l
