@@ -44,9 +44,16 @@ __device__ __forceinline__ bool rows_have_valid(const int* __restrict__ len, int
   return false;
 }
 
-template <int BN, typename TOut>
+// MB: 128-row MMA blocks per tile.  MB = 1 keeps two accumulators so one
+// tile's epilogue overlaps the next tile's MMAs; MB = 2 (BN = 256) fills all
+// 512 TMEM columns with one 256 × 256 tile, reading a third fewer operand
+// bytes per flop, and its epilogue waits for the tile's MMAs.
+template <int BN, typename TOut, int MB = 1>
 struct TcGemmCfg {
-  static constexpr int BM = 128;
+  static constexpr int BM = 128 * MB;
+  static constexpr int NACC = MB == 1 ? 2 : 1;        // accumulator buffers
+  static constexpr int EPI_WARPS = 4 * MB;             // one warpgroup per 128-row block
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int BK = 64;                       // 128 bytes of bf16: one swizzle row
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
@@ -54,11 +61,12 @@ struct TcGemmCfg {
   // epilogue staging: per epilogue warp two [32 rows × 32 cols] buffers
   static constexpr uint32_t STG_BYTES = 32 * 32 * sizeof(TOut);
   static constexpr int STG_SWIZZLE = 32 * sizeof(TOut);   // 64 (bf16 rows) or 128 (fp32 rows)
-  static constexpr size_t BUDGET = 227 * 1024 - 1024 - 256 - 8 * STG_BYTES;
+  static constexpr size_t BUDGET = 227 * 1024 - 1024 - 256 - 2 * EPI_WARPS * STG_BYTES;
   static constexpr int STAGES_FIT = (int)(BUDGET / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT < 6 ? STAGES_FIT : 6;
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (size_t)STAGE_BYTES + 8 * STG_BYTES + 256;
+  static_assert(MB == 1 || (MB == 2 && BN == 256), "two M blocks only with 256-column tiles");
+  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (size_t)STAGE_BYTES + 2 * EPI_WARPS * STG_BYTES + 256;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128 is a multiple of 16 up to 256");
   static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte swizzle-atom alignment");
   static_assert(STAGES >= 3, "shared memory too small for the pipeline");
@@ -122,19 +130,19 @@ __device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[
 
 // C2 (optional): columns n < c2_cols are also written, rounded to bf16, into
 // C2[m, n] (row stride ldc2).  x_proj uses it to hand Δr to dt_proj in bf16.
-template <int BN, typename TOut>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, typename TOut, int MB = 1>
+__global__ void __launch_bounds__(TcGemmCfg<BN, TOut, MB>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, bf16* __restrict__ C2, int ldc2, int c2_cols,
                int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err) {
-  using Cfg = TcGemmCfg<BN, TOut>;
-  constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES;
+  using Cfg = TcGemmCfg<BN, TOut, MB>;
+  constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES, NACC = Cfg::NACC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint8_t* sStg = sB + STAGES * Cfg::B_BYTES;          // 8 staging buffers (1024-byte aligned)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 8 * Cfg::STG_BYTES);
+  uint8_t* sStg = sB + STAGES * Cfg::B_BYTES;          // 2 staging buffers per epilogue warp (1024-byte aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 2 * Cfg::EPI_WARPS * Cfg::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -155,7 +163,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       sm100::mbar_init(&tfull[a], 1);
-      sm100::mbar_init(&tempty[a], 128);
+      sm100::mbar_init(&tempty[a], 32 * Cfg::EPI_WARPS);
     }
     sm100::mbar_init(drain, 1);
     sm100::fence_barrier_init();
@@ -205,7 +213,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = sm100::idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(128, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -222,16 +230,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t a0 = sm100::smem_u32(sA + stage * Cfg::A_BYTES);
           const uint32_t b0 = sm100::smem_u32(sB + stage * Cfg::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            sm100::mma_bf16(d_tmem, sm100::smem_desc_k128(a0 + k * 32), sm100::smem_desc_k128(b0 + k * 32),
-                            idesc, (kb | k) != 0);
+          for (int k = 0; k < BK / 16; ++k) {
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb)   // rows 128·mb …: accumulator columns [BN·mb, BN·mb + BN)
+              sm100::mma_bf16(d_tmem + (uint32_t)(mb * BN), sm100::smem_desc_k128(a0 + mb * (128 * 128) + k * 32),
+                              sm100::smem_desc_k128(b0 + k * 32), idesc, (kb | k) != 0);
+          }
           sm100::mma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         sm100::mma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) aphase ^= 1u;
+        if (++acc == NACC) { acc = 0; aphase ^= 1u; }
       }
       // all MMAs issued by this thread have retired once `drain` completes
       sm100::mma_commit(drain);
@@ -242,6 +252,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // Each 32 × 32 block goes TMEM -> registers -> swizzled staging buffer ->
     // TMA store (rows past M or columns past N are clipped by the store).
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;   // the 128-row M block this warp drains
     uint8_t* stg = sStg + (warp - 2) * 2 * Cfg::STG_BYTES;
     int acc = 0;
     uint32_t aphase = 0;
@@ -251,38 +262,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!sm100::mbar_wait(&tfull[acc], aphase, err)) break;
       sm100::tc_fence_after();
       const int mb = (int)(t / num_n), nb = (int)(t % num_n);
-      const long long row = (long long)mb * BM + q * 32 + lane;
-      const bool row_ok = row < M && (!len || row_valid(len, L, row));
+      {
+        const int row0 = mb * BM + h * 128 + q * 32;     // this warp's 32 rows of M block h
+        const long long row = (long long)row0 + lane;
+        const bool row_ok = row < M && (!len || row_valid(len, L, row));
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32, ++chunk) {
-        float v[32];
-        sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), v);
-        const int col = nb * BN + c0;
-        uint8_t* buf = stg + (chunk & 1) * Cfg::STG_BYTES;
-        if (lane == 0) sm100::bulk_wait_read_le1();   // the store that used `buf` has read it
-        __syncwarp();
-        stage_row32<TOut>(buf, lane, v);
-        sm100::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && col < N) {
-          sm100::tma_store_2d(&tmC, buf, col, mb * BM + q * 32);
-          sm100::bulk_commit();
-        }
-        if (C2 && row_ok && col < c2_cols) {
-          bf16* d2 = C2 + row * (long long)ldc2 + col;
-          if (col + 32 <= c2_cols) {
-            store_row32<bf16>(d2, v);
-          } else {
+        for (int c0 = 0; c0 < BN; c0 += 32, ++chunk) {
+          float v[32];
+          sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + h * BN + c0), v);
+          const int col = nb * BN + c0;
+          uint8_t* buf = stg + (chunk & 1) * Cfg::STG_BYTES;
+          if (lane == 0) sm100::bulk_wait_read_le1();   // the store that used `buf` has read it
+          __syncwarp();
+          stage_row32<TOut>(buf, lane, v);
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && col < N && row0 < M) {
+            sm100::tma_store_2d(&tmC, buf, col, row0);
+            sm100::bulk_commit();
+          }
+          if (C2 && row_ok && col < c2_cols) {
+            bf16* d2 = C2 + row * (long long)ldc2 + col;
+            if (col + 32 <= c2_cols) {
+              store_row32<bf16>(d2, v);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < c2_cols - col) d2[j] = __float2bfloat16_rn(v[j]);
+              for (int j = 0; j < 32; ++j)
+                if (j < c2_cols - col) d2[j] = __float2bfloat16_rn(v[j]);
+            }
           }
         }
       }
       sm100::tc_fence_before();
       sm100::mbar_arrive(&tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1u;
+      if (++acc == NACC) { acc = 0; aphase ^= 1u; }
     }
     if (lane == 0) sm100::bulk_wait_all();
   }

@@ -2,6 +2,8 @@
 // tile-width choice and the persistent launch (one CTA per SM).
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "gemm_convx.cuh"
 #include "gemm_tc.cuh"
 #include "tc_gemm.h"
@@ -16,21 +18,30 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int BN, typename TOut>
+// 256 × 256 tiles (two M = 128 MMA blocks per CTA) for 256-multiple N (0: 128 × BN only).
+#ifndef R2L_GEMM_MB2
+#define R2L_GEMM_MB2 1
+#endif
+// shortest K for which the 256 × 256 tile pays (its epilogue does not overlap the next tile)
+#ifndef R2L_GEMM_MB2_MIN_K
+#define R2L_GEMM_MB2_MIN_K 0
+#endif
+
+template <int BN, typename TOut, int MB = 1>
 cudaError_t launch(const TcGemm& g, cudaStream_t st) {
-  using Cfg = TcGemmCfg<BN, TOut>;
+  using Cfg = TcGemmCfg<BN, TOut, MB>;
   CUtensorMap ta, tb, tc;
   if (!make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tc, g.C, (int)sizeof(TOut), g.N, g.M, (long long)g.ldc * sizeof(TOut), 32, 32, Cfg::STG_SWIZZLE))
     return cudaErrorInvalidValue;
-  auto kern = gemm_tc_kernel<BN, TOut>;
+  auto kern = gemm_tc_kernel<BN, TOut, MB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, g.C2, g.ldc2, g.c2_cols,
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, g.C2, g.ldc2, g.c2_cols,
                                             g.M, g.N, g.K, g.len, g.L, g.err);
   return cudaPeekAtLastError();
 }
@@ -38,7 +49,11 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
 template <typename TOut>
 cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
   // widest tile that divides N; else the narrowest that covers it; else 256 with a ragged edge
-  if (g.N % 256 == 0) return launch<256, TOut>(g, st);
+  if (g.N % 256 == 0) {
+    if constexpr (std::is_same<TOut, bf16>::value)
+      if (R2L_GEMM_MB2 && g.K >= R2L_GEMM_MB2_MIN_K) return launch<256, TOut, 2>(g, st);
+    return launch<256, TOut>(g, st);
+  }
   if (g.N <= 64) return launch<64, TOut>(g, st);
   if (g.N <= 128) return launch<128, TOut>(g, st);
   if (g.N <= 160) return launch<160, TOut>(g, st);
