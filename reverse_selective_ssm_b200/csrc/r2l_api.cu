@@ -218,12 +218,13 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   prof->launches++;
   R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
   // a2: u = SiLU(anti-causal conv(x)); a3: [Δr | B | C] = u · W_xᵀ (fp32 out).
-  // bf16 with an x_proj of 160 columns: one kernel does both (the conv runs
-  // in x_proj's operand producer and u is written once, for the scan).
+  // bf16 with an x_proj of 160 columns and at least one 128-row tile per SM:
+  // one kernel does both (the conv runs in x_proj's operand producer and u
+  // is written once, for the scan).
   R2L_TRY(prof->mark(R2L_STAGE_CONV, st));
   bool convx_done = false;
   if constexpr (kTC) {
-    if (R2L_CONVX && r2l::convx_supported(p.ldd, E)) {
+    if (R2L_CONVX && r2l::convx_supported(p.ldd, E) && r2l::convx_worthwhile(M)) {
       R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
       prof->launches++;
       r2l::ConvX c{};

@@ -50,8 +50,11 @@ template <typename TOut>
 cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
   // widest tile that divides N; else the narrowest that covers it; else 256 with a ragged edge
   if (g.N % 256 == 0) {
+    // 256 × 256 tiles only when there are enough of them to give every SM one
     if constexpr (std::is_same<TOut, bf16>::value)
-      if (R2L_GEMM_MB2 && g.K >= R2L_GEMM_MB2_MIN_K) return launch<256, TOut, 2>(g, st);
+      if (R2L_GEMM_MB2 && g.K >= R2L_GEMM_MB2_MIN_K &&
+          (long long)((g.M + 255) / 256) * (g.N / 256) >= sm_count())
+        return launch<256, TOut, 2>(g, st);
     return launch<256, TOut>(g, st);
   }
   if (g.N <= 64) return launch<64, TOut>(g, st);
@@ -88,6 +91,8 @@ cudaError_t launch_convx(const ConvX& g, cudaStream_t st) {
 }  // namespace
 
 bool convx_supported(int N, int E) { return N == convx::BN && E > 0 && E % convx::BK == 0; }
+
+bool convx_worthwhile(long long M) { return (M + convx::BM - 1) / convx::BM >= sm_count(); }
 
 cudaError_t convx_gemm(const ConvX& g, cudaStream_t st) {
   if (g.M <= 0) return cudaSuccess;

@@ -50,6 +50,9 @@ struct ConvX {
 };
 
 bool convx_supported(int N, int E);
+// The fused kernel runs one 128-row tile per CTA at a time; below one tile per
+// SM the standalone conv kernel, which spreads over all SMs, is faster.
+bool convx_worthwhile(long long M);
 cudaError_t convx_gemm(const ConvX& g, cudaStream_t st);
 
 }  // namespace r2l
