@@ -40,15 +40,17 @@ namespace pair {
 constexpr int CHP = 256;                          // channels per CTA
 constexpr int PWARPS = 16;                        // compute warps
 constexpr int PTHREADS = PWARPS * 32;
-constexpr int GT = 4;                             // tokens per B|C group and per sub-tile
-constexpr int NG = TS / GT;                       // groups per tile; TMEM region g serves group g
+constexpr int GT = 4;                             // tokens per sub-tile (phase A, then phase B)
+constexpr int GB = 8;                             // tokens per B|C group (one MMA, one handshake)
+constexpr int NG = TS / GB;                       // groups per tile; TMEM region g serves group g
 constexpr uint32_t P_ACT_TILE = TS * CHP * 2;     // one bf16 [TS × CHP] tile
 constexpr uint32_t P_W_SLICE = CHP * DT_R * 2;    // bf16 W_dt [CHP × R]
 constexpr uint32_t P_BC_COL0 = STAGES * 32;       // dt_raw: [stage][block] × 16 columns
 constexpr uint32_t P_TMEM_COLS = 512;
-constexpr uint32_t P_GROUP_COLS = GT * 16;        // 16 columns per token
+constexpr uint32_t P_GROUP_COLS = GB * 16;        // 16 columns per token
+constexpr uint32_t P_OPB_BYTES = GB * 16 * 32;    // GB·16 operand rows of 32 bytes
 static_assert(P_BC_COL0 + NG * P_GROUP_COLS <= P_TMEM_COLS, "TMEM budget");
-static_assert(GT * 16 == 64, "one MMA (N = 64) per group");
+static_assert(GB * 16 <= 256 && GB % GT == 0, "one MMA (N = GB·16) per group");
 
 struct SmemPair {
   static constexpr uint32_t W = 0;
@@ -60,7 +62,7 @@ struct SmemPair {
   static constexpr uint32_t BC = Z + STAGES * P_ACT_TILE;
   static constexpr uint32_t PAT = BC + STAGES * BC_TILE;          // lane-pattern operand
   static constexpr uint32_t OPB = PAT + ONES_BYTES;
-  static constexpr uint32_t BAR = OPB + NG * OPB_BYTES;           // full, empty, dtready [STAGES], wfull, drain, bcready, bcfree [NG]
+  static constexpr uint32_t BAR = OPB + NG * P_OPB_BYTES;           // full, empty, dtready [STAGES], wfull, drain, bcready, bcfree [NG]
   static constexpr uint32_t SLOT = BAR + (3 * STAGES + 2 + 2 * NG) * 8;
   static constexpr size_t BYTES = 1024 + SLOT + 16;
   static constexpr int THREADS = PTHREADS + 64;
@@ -81,15 +83,15 @@ __device__ __forceinline__ void run_mma_pair(uint8_t* smem, uint32_t tmem_base, 
     *reinterpret_cast<float4*>(row) = upper ? make_float4(0.0f, 0.0f, 1.0f, 1.0f) : make_float4(1.0f, 1.0f, 0.0f, 0.0f);
     *reinterpret_cast<float4*>(row + 128) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
-  for (int n = lane; n < NG * 64; n += 32) {
-    uint8_t* row = smem + S::OPB + (n / 64) * OPB_BYTES + opnd_row(n % 64);
+  for (int n = lane; n < NG * GB * 16; n += 32) {
+    uint8_t* row = smem + S::OPB + (n / (GB * 16)) * P_OPB_BYTES + opnd_row(n % (GB * 16));
     *reinterpret_cast<float4*>(row) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     *reinterpret_cast<float4*>(row + 128) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
   sm100::fence_proxy_async_smem();
   __syncwarp();
   constexpr uint32_t idt = sm100::idesc_bf16_f32(128, TS);
-  constexpr uint32_t ibc = sm100::idesc_tf32_f32(128, 64);
+  constexpr uint32_t ibc = sm100::idesc_tf32_f32(128, GB * 16);
   const uint64_t a_pat = sm100::smem_desc_noswz(sm100::smem_u32(smem + S::PAT), 128, 256);
   const uint32_t w0 = sm100::smem_u32(smem + S::W);
   bool ok = sm100::mbar_wait(wfull, 0, err);
@@ -118,12 +120,12 @@ __device__ __forceinline__ void run_mma_pair(uint8_t* smem, uint32_t tmem_base, 
     for (int g = 0; g < NG; ++g) {
       if (!sm100::mbar_wait(&bcfree[g], ((uint32_t)it & 1u) ^ 1u, err)) { ok = false; break; }
       sm100::tc_fence_after();
-      uint8_t* opb = smem + S::OPB + g * OPB_BYTES;
+      uint8_t* opb = smem + S::OPB + g * P_OPB_BYTES;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int row = lane + 32 * half;            // 16·slot + n
+      for (int part = 0; part < GB / 2; ++part) {
+        const int row = lane + 32 * part;            // 16·slot + n
         const int slot = row >> 4, n = row & 15;
-        const int tok = FWD ? GT * g + slot : TS - 1 - GT * g - slot;
+        const int tok = FWD ? GB * g + slot : TS - 1 - GB * g - slot;
         const float v0 = bct[tok * 32 + 2 * n], v1 = bct[tok * 32 + 2 * n + 1];
         const float h0 = __uint_as_float(__float_as_uint(v0) & 0xFFFFE000u);
         const float h1 = __uint_as_float(__float_as_uint(v1) & 0xFFFFE000u);
@@ -172,8 +174,8 @@ __device__ __forceinline__ void pair_decays(const PCtx& cx, float dec, float2 (&
   }
 }
 
-// One tile of 16 tokens as four sub-tiles of GT tokens; sub-tile g is B|C
-// group g (TMEM region g).  Tokens outside [jlo, jhi) (a tile that crosses the
+// One tile of 16 tokens as four sub-tiles of GT tokens; each pair of
+// sub-tiles reads one B|C group (TMEM region g = sub-tile / 2).  Tokens outside [jlo, jhi) (a tile that crosses the
 // sequence's start or end) leave the state untouched and write nothing.
 template <bool POW, bool FULL, bool FWD>
 __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const bf16* su, bf16* sz, bf16* yg,
@@ -183,8 +185,10 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
   const int lane = threadIdx.x & 31;
   const int h = lane >> 4;
 #pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    const int j0 = FWD ? g * GT : TS - GT - g * GT;
+  for (int sb = 0; sb < TS / GT; ++sb) {
+    const int g = sb / (GB / GT);                  // B|C group of this sub-tile
+    const int gs = sb % (GB / GT);                 // sub-tile within the group
+    const int j0 = FWD ? sb * GT : TS - GT - sb * GT;
     // phase A for this thread's tokens t = 2i + h of the sub-tile
     float dec_o[GT / 2], du_o[GT / 2], Du_o[GT / 2], gz_o[GT / 2];
 #pragma unroll
@@ -210,15 +214,17 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
       du_d[i] = __shfl_sync(0xffffffffu, du_o[i], lane | 16);
     }
     float part[GT];     // this thread's half of ⟨C, H⟩ per token of the sub-tile
-    if (!sm100::mbar_wait(&bcready[g], ph, err)) { ok = false; return; }
-    __syncwarp();
-    sm100::tc_fence_after();
+    if (gs == 0) {
+      if (!sm100::mbar_wait(&bcready[g], ph, err)) { ok = false; return; }
+      __syncwarp();
+      sm100::tc_fence_after();
+    }
 #pragma unroll
     for (int slot = 0; slot < GT; ++slot) {
       const int t = FWD ? slot : GT - 1 - slot;
       const int j = j0 + t;
       float bv[16];
-      sm100::tmem_ld16(t_bc + (uint32_t)(g * P_GROUP_COLS + slot * 16), bv);
+      sm100::tmem_ld16(t_bc + (uint32_t)(g * P_GROUP_COLS + (gs * GT + slot) * 16), bv);
       part[t] = 0.0f;
       if (FULL || (j >= jlo && j < jhi)) {
         const float dec = (t & 1) ? dec_d[t >> 1] : dec_e[t >> 1];
@@ -235,9 +241,11 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
         part[t] = acc.x + acc.y;
       }
     }
-    sm100::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) sm100::mbar_arrive(&bcfree[g]);
+    if (gs == GB / GT - 1) {                       // the group's last token is read
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&bcfree[g]);
+    }
     // y of this thread's tokens: its half of ⟨C, H⟩ plus the partner's
 #pragma unroll
     for (int i = 0; i < GT / 2; ++i) {
