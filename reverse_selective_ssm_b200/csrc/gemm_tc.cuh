@@ -130,11 +130,18 @@ __device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[
 
 // C2 (optional): columns n < c2_cols are also written, rounded to bf16, into
 // C2[m, n] (row stride ldc2).  x_proj uses it to hand Δr to dt_proj in bf16.
+// splits > 1 (fp32 C only; C2 unused): each tile's K range is cut into
+// `splits` parts computed by different CTAs; the part s of a tile is stored
+// at rows s·Mp + row of the tensor tmC describes (a partial-sum buffer of
+// `splits` slices of Mp rows, Mp = M rounded up to whole tiles), and a
+// separate kernel adds the slices in a fixed order.  For short, wide-K GEMMs
+// with fewer tiles than SMs.
 template <int BN, typename TOut, int MB = 1>
 __global__ void __launch_bounds__(TcGemmCfg<BN, TOut, MB>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, bf16* __restrict__ C2, int ldc2, int c2_cols,
-               int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err) {
+               int M, int N, int K, const int* __restrict__ len, int L, unsigned* __restrict__ err,
+               int splits) {
   using Cfg = TcGemmCfg<BN, TOut, MB>;
   constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES, NACC = Cfg::NACC;
   extern __shared__ uint8_t smem_raw[];
@@ -154,7 +161,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int num_m = (M + BM - 1) / BM;
   const int num_n = (N + BN - 1) / BN;
   const int num_k = (K + BK - 1) / BK;
-  const long long total = (long long)num_m * num_n;
+  const int kps = (num_k + splits - 1) / splits;       // K blocks per split
+  const long long total = (long long)num_m * num_n * splits;   // work units: (tile, split)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -179,7 +187,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   auto tile_live = [&](long long t) -> bool {
     if (!len) return true;
-    const long long r0 = (t / num_n) * BM;
+    const long long r0 = (t / splits / num_n) * BM;
     const long long r1 = r0 + BM < M ? r0 + BM : M;
     return rows_have_valid(len, L, r0, r1);
   };
@@ -195,8 +203,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool ok = true;
       for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
         if (!tile_live(t)) continue;
-        const int mb = (int)(t / num_n), nb = (int)(t % num_n);
-        for (int kb = 0; kb < num_k; ++kb) {
+        const long long tile = t / splits;
+        const int mb = (int)(tile / num_n), nb = (int)(tile % num_n);
+        const int kb0 = (int)(t % splits) * kps, kb1 = kb0 + kps < num_k ? kb0 + kps : num_k;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, err)) { ok = false; break; }
           sm100::mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           sm100::tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
@@ -224,7 +234,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (!sm100::mbar_wait(&tempty[acc], aphase ^ 1u, err)) { ok = false; break; }
         sm100::tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_k; ++kb) {
+        const int kb0 = (int)(t % splits) * kps, kb1 = kb0 + kps < num_k ? kb0 + kps : num_k;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!sm100::mbar_wait(&full[stage], phase, err)) { ok = false; break; }
           sm100::tc_fence_after();
           const uint32_t a0 = sm100::smem_u32(sA + stage * Cfg::A_BYTES);
@@ -234,7 +245,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
             for (int mb = 0; mb < MB; ++mb)   // rows 128·mb …: accumulator columns [BN·mb, BN·mb + BN)
               sm100::mma_bf16(d_tmem + (uint32_t)(mb * BN), sm100::smem_desc_k128(a0 + mb * (128 * 128) + k * 32),
-                              sm100::smem_desc_k128(b0 + k * 32), idesc, (kb | k) != 0);
+                              sm100::smem_desc_k128(b0 + k * 32), idesc, (kb != kb0) | (k != 0));
           }
           sm100::mma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -261,7 +272,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!tile_live(t)) continue;
       if (!sm100::mbar_wait(&tfull[acc], aphase, err)) break;
       sm100::tc_fence_after();
-      const int mb = (int)(t / num_n), nb = (int)(t % num_n);
+      const long long tile = t / splits;
+      const int mb = (int)(tile / num_n), nb = (int)(tile % num_n);
       {
         const int row0 = mb * BM + h * 128 + q * 32;     // this warp's 32 rows of M block h
         const long long row = (long long)row0 + lane;
@@ -278,10 +290,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           sm100::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && col < N && row0 < M) {
-            sm100::tma_store_2d(&tmC, buf, col, row0);
+            const int prow = splits > 1 ? (int)(t % splits) * (num_m * BM) + row0 : row0;
+            sm100::tma_store_2d(&tmC, buf, col, prow);
             sm100::bulk_commit();
           }
-          if (C2 && row_ok && col < c2_cols) {
+          if (C2 && splits == 1 && row_ok && col < c2_cols) {
             bf16* d2 = C2 + row * (long long)ldc2 + col;
             if (col + 32 <= c2_cols) {
               store_row32<bf16>(d2, v);

@@ -35,7 +35,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Byte offsets of the workspace regions for a [B, L] batch.
 struct Plan {
-  size_t status, len, xz, u, dbc, dr, dt, y, o, carry, total;
+  size_t status, len, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, total;
   int chunk_tokens;  // scan chunk length (bf16 path)
   long long M;
   int E, d, R, N, ldd;
@@ -69,6 +69,10 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, p->E, 0);
   p->carry = off;
   if (dm->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, p->E, p->chunk_tokens), kAlign);
+  // x_proj split-K partial sums (bf16 path, few 128-row tiles)
+  p->xsplit = off;
+  p->xsplit_bytes = dm->dtype == R2L_BF16 ? r2l::tc_gemm_partial_bytes(p->M, p->ldd, p->E) : 0;
+  off = align_up(off + p->xsplit_bytes, kAlign);
   p->total = off;
   return true;
 }
@@ -153,13 +157,14 @@ r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, c
 template <typename T, typename TC>
 r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long long M, int N, int K,
                 const int* len, int L, unsigned* err, cudaStream_t st, bf16* c2 = nullptr, int ldc2 = 0,
-                int c2_cols = 0) {
+                int c2_cols = 0, float* partial = nullptr, size_t partial_bytes = 0) {
   if constexpr (std::is_same<T, bf16>::value) {
     r2l::TcGemm g{};
     g.A = A; g.lda = lda; g.B = W; g.ldb = ldw; g.C = C; g.ldc = ldc;
     g.c_fp32 = std::is_same<TC, float>::value;
     g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols;
     g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
+    g.partial = partial; g.partial_bytes = partial_bytes;
     return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
   } else {
     return gemm(A, lda, W, ldw, C, ldc, M, N, K, len, L, st);
@@ -252,7 +257,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     }
     R2L_TRY(prof->mark(R2L_STAGE_X_PROJ, st));
     prof->launches++;
-    R2L_TRY(proj(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, err, st, dr, R, R));
+    R2L_TRY(proj(u, E, (const T*)w->x_proj_w, E, dbc, p.ldd, M, p.ldd, E, len, L, err, st, dr, R, R,
+                 (float*)(ws + p.xsplit), p.xsplit_bytes));
   }
   // a4: dt_raw = Δr · W_dtᵀ  (bias + softplus applied in the scan)
   R2L_TRY(prof->mark(R2L_STAGE_DT_PROJ, st));

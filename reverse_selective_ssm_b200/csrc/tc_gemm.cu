@@ -22,10 +22,52 @@ int sm_count() {
 #ifndef R2L_GEMM_MB2
 #define R2L_GEMM_MB2 1
 #endif
+// split-K for fp32-output GEMMs with fewer tiles than SMs (0: off)
+#ifndef R2L_GEMM_SPLITK
+#define R2L_GEMM_SPLITK 1
+#endif
 // shortest K for which the 256 × 256 tile pays (its epilogue does not overlap the next tile)
 #ifndef R2L_GEMM_MB2_MIN_K
 #define R2L_GEMM_MB2_MIN_K 0
 #endif
+
+// Split-K: C[m, c] = Σ_s P[s·Mp + m, c], slices added in order s = 0, 1, …
+// (deterministic); C2[m, c] = bf16 of it for c < c2_cols on valid rows.
+__global__ void splitk_sum_kernel(const float* __restrict__ P, int splits, long long Mp, int N,
+                                  float* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols,
+                                  int M, const int* __restrict__ len, int L) {
+  const int m = blockIdx.x;
+  if (m >= M) return;
+  const bool valid = !len || row_valid(len, L, m);
+  for (int c = threadIdx.x; c < N; c += blockDim.x) {
+    float acc = 0.0f;
+    for (int sp = 0; sp < splits; ++sp) acc += P[((long long)sp * Mp + m) * N + c];
+    C[(long long)m * ldc + c] = acc;
+    if (C2 && valid && c < c2_cols) C2[(long long)m * ldc2 + c] = __float2bfloat16_rn(acc);
+  }
+}
+
+int tile_width(int N) {   // the BN dispatch() picks for an fp32-output GEMM of this width
+  if (N % 256 == 0) return 256;
+  if (N <= 64) return 64;
+  if (N <= 128) return 128;
+  if (N <= 160) return 160;
+  if (N % 128 == 0) return 128;
+  return 256;
+}
+
+// K splits for an fp32-output GEMM with fewer tiles than SMs (0 ⇒ none):
+// enough (tile, split) units to cover the SMs, at least 4 K blocks each,
+// every split non-empty.
+int choose_splits(long long tiles, int num_k) {
+  const int sms = sm_count();
+  if (tiles * 2 > sms || num_k < 8) return 1;
+  int want = (int)(sms / tiles);
+  if (want > num_k / 4) want = num_k / 4;
+  if (want < 2) return 1;
+  const int kps = (num_k + want - 1) / want;
+  return (num_k + kps - 1) / kps;
+}
 
 template <int BN, typename TOut, int MB = 1>
 cudaError_t launch(const TcGemm& g, cudaStream_t st) {
@@ -38,11 +80,28 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   auto kern = gemm_tc_kernel<BN, TOut, MB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const long long tiles = (long long)((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  const long long num_m = (g.M + Cfg::BM - 1) / Cfg::BM;
+  const long long tiles = num_m * ((g.N + BN - 1) / BN);
+  int splits = 1;
+  if constexpr (std::is_same<TOut, float>::value) {
+    const int sp = choose_splits(tiles, (g.K + Cfg::BK - 1) / Cfg::BK);
+    const size_t need = (size_t)sp * num_m * Cfg::BM * g.N * sizeof(float);
+    if (R2L_GEMM_SPLITK && sp > 1 && g.partial && g.partial_bytes >= need) {
+      splits = sp;
+      if (!make_tmap_2d(&tc, g.partial, 4, g.N, (long long)sp * num_m * Cfg::BM, (long long)g.N * 4, 32, 32,
+                        Cfg::STG_SWIZZLE))
+        return cudaErrorInvalidValue;
+    }
+  }
+  const long long units = tiles * splits;
+  const int grid = (int)(units < sm_count() ? units : sm_count());
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, g.C2, g.ldc2, g.c2_cols,
-                                            g.M, g.N, g.K, g.len, g.L, g.err);
+                                            g.M, g.N, g.K, g.len, g.L, g.err, splits);
+  cudaError_t e2 = cudaPeekAtLastError();
+  if (e2 != cudaSuccess || splits == 1) return e2;
+  splitk_sum_kernel<<<g.M, 128, 0, st>>>(g.partial, splits, num_m * Cfg::BM, g.N, reinterpret_cast<float*>(g.C),
+                                         g.ldc, g.C2, g.ldc2, g.c2_cols, g.M, g.len, g.L);
   return cudaPeekAtLastError();
 }
 
@@ -55,6 +114,8 @@ cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
       if (R2L_GEMM_MB2 && g.K >= R2L_GEMM_MB2_MIN_K &&
           (long long)((g.M + 255) / 256) * (g.N / 256) >= sm_count())
         return launch<256, TOut, 2>(g, st);
+    // fewer 128 × 256 tiles than SMs: 128-wide tiles give twice as many
+    if ((long long)((g.M + 127) / 128) * (g.N / 256) < sm_count()) return launch<128, TOut>(g, st);
     return launch<256, TOut>(g, st);
   }
   if (g.N <= 64) return launch<64, TOut>(g, st);
@@ -89,6 +150,13 @@ cudaError_t launch_convx(const ConvX& g, cudaStream_t st) {
 }
 
 }  // namespace
+
+size_t tc_gemm_partial_bytes(long long M, int N, int K) {
+  const int BN = tile_width(N);
+  const long long num_m = (M + 127) / 128;
+  const int sp = choose_splits(num_m * ((N + BN - 1) / BN), (K + 63) / 64);
+  return sp > 1 ? (size_t)sp * num_m * 128 * N * sizeof(float) : 0;
+}
 
 bool convx_supported(int N, int E) { return N == convx::BN && E > 0 && E % convx::BK == 0; }
 

@@ -21,7 +21,13 @@ struct TcGemm {
   const int* len;          // device lengths [B] (rows i >= len[b] of each sequence are skipped)
   int L;
   unsigned* err;           // device status word (timeout flag)
+  float* partial;          // optional scratch for split-K partial sums (fp32 C only), or null
+  size_t partial_bytes;
 };
+
+// Scratch an fp32-output GEMM of this shape uses for split-K partial sums
+// (0 when it runs unsplit).  With less, it runs unsplit.
+size_t tc_gemm_partial_bytes(long long M, int N, int K);
 
 // Enqueues the GEMM on `st`.  Requires lda, ldb, K to be multiples of 8.
 cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st);
