@@ -71,10 +71,10 @@ STAGE_SOURCES = {
     "gemm": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "in_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "x_proj": ["gemm_convx.cuh", "gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
+    "conv": ["conv_fast.cuh", "gemm_convx.cuh"] + _COMMON,
     "dt_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "out_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
-    "conv": ["conv_fast.cuh"] + _COMMON,
-    "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu"] + _COMMON,
+    "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh"] + _COMMON,
     "ln_residual": ["simt_kernels.cuh"] + _COMMON,
 }
 
