@@ -66,9 +66,11 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->dt = off;     off = align_up(off + M * p->E * p->act, kAlign);
   p->y = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->o = off;      off = align_up(off + M * p->d * p->act, kAlign);
-  p->chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, p->E, 0);
+  // the bf16 layer with dt_rank 128 runs the scan with dt_proj fused (two threads per channel)
+  const bool pair = dm->dtype == R2L_BF16 && p->R == r2l::kScanFusedDtRank;
+  p->chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, p->E, 0, pair);
   p->carry = off;
-  if (dm->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, p->E, p->chunk_tokens), kAlign);
+  if (dm->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, p->E, p->chunk_tokens, pair), kAlign);
   // x_proj split-K partial sums (bf16 path, few 128-row tiles)
   p->xsplit = off;
   p->xsplit_bytes = dm->dtype == R2L_BF16 ? r2l::tc_gemm_partial_bytes(p->M, p->ldd, p->E) : 0;

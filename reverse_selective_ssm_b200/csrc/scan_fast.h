@@ -31,12 +31,13 @@ struct ScanArgs {
   int forward;                                 // left-to-right block
 };
 
-// Tokens per chunk chosen from the shape alone (deterministic, no device query).
-int scan_auto_chunk_tokens(int B, int L, int E);
+// Tokens per chunk chosen from the shape alone (deterministic, no device
+// query).  `pair`: the scan runs with dt_proj fused (two threads per channel).
+int scan_auto_chunk_tokens(int B, int L, int E, bool pair = false);
 // Chunk length actually used for a request (0 = automatic), a multiple of 16.
-int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens);
+int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens, bool pair = false);
 // Bytes of carry scratch the scan needs for this shape and chunk length.
-size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens);
+size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens, bool pair = false);
 // Enqueue the scan (1 or 3 launches).  Returns the number of kernels launched
 // through *launches when not null.
 cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches);

@@ -9,8 +9,22 @@
 
 namespace r2l {
 
-int scan_auto_chunk_tokens(int B, int L, int E) {
+int scan_auto_chunk_tokens(int B, int L, int E, bool pair) {
   using namespace rscan;
+  if (pair) {
+    // two threads per channel, one 256-channel CTA per SM: split sequences
+    // only when one pass leaves most SMs idle, into as many chunks as one wave
+    // of CTAs holds (each chunk costs a second, state-only pass)
+    const long long ctas1 = (long long)B * ((E + rscan::pair::CHP - 1) / rscan::pair::CHP);
+    const int whole = (L + TS - 1) / TS * TS;
+    if (ctas1 * 3 >= 148LL * 2) return whole;
+    long long nc = 148 / ctas1;
+    if (nc < 2) return whole;
+    long long T = (L + nc - 1) / nc;
+    T = (T + TS - 1) / TS * TS;
+    if (T < 4 * TS) T = 4 * TS;
+    return (int)(T < whole ? T : whole);
+  }
   // Compute warps with one chunk per sequence; below ~6 per SM of a 148-SM
   // part the sequence is split so that about 24 per SM are in flight.
   const long long warps1 = (long long)B * ((E + CTHREADS - 1) / CTHREADS) * CWARPS;
@@ -24,16 +38,16 @@ int scan_auto_chunk_tokens(int B, int L, int E) {
   return (int)(T < whole ? T : whole);
 }
 
-int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens) {
+int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens, bool pair) {
   using namespace rscan;
-  if (chunk_tokens <= 0) return scan_auto_chunk_tokens(B, L, E);
+  if (chunk_tokens <= 0) return scan_auto_chunk_tokens(B, L, E, pair);
   const int T = (chunk_tokens + TS - 1) / TS * TS;
   const int whole = (L + TS - 1) / TS * TS;
   return T < whole ? T : whole;
 }
 
-size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens) {
-  const int T = scan_resolve_chunk_tokens(B, L, E, chunk_tokens);
+size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens, bool pair) {
+  const int T = scan_resolve_chunk_tokens(B, L, E, chunk_tokens, pair);
   const long long nc = (L + T - 1) / T;
   if (nc <= 1) return 0;
   return (size_t)B * nc * E * 17 * sizeof(float);
@@ -52,7 +66,7 @@ namespace {
 #endif
 
 template <bool FWD>
-cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, cudaStream_t st, int* launches) {
+cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
   using namespace rscan;
   using Sp = pair::SmemPair;
   constexpr int CHP = pair::CHP;
@@ -65,11 +79,21 @@ cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, cudaStream_t 
       !make_tmap_2d(&tdr, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, 128) ||
       !make_tmap_2d(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CHP, 128))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(pair::scan_pair_kernel<FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Sp::BYTES);
+  cudaError_t e = cudaFuncSetAttribute(pair::scan_pair_kernel<true, FWD>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sp::BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.E + CHP - 1) / CHP, 1, a.B);
-  pair::scan_pair_kernel<FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+  const dim3 grid((a.E + CHP - 1) / CHP, nc, a.B);
+  if (nc > 1) {
+    if ((e = cudaFuncSetAttribute(pair::scan_pair_kernel<false, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Sp::BYTES)) != cudaSuccess)
+      return e;
+    pair::scan_pair_kernel<false, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (launches) *launches += 2;
+  }
+  pair::scan_pair_kernel<true, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;
@@ -108,7 +132,7 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
   }
   cudaError_t e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
-  if (DTMMA && R2L_SCAN_PAIR && nc == 1) return launch_pair<FWD>(a, p, st, launches);
+  if (DTMMA && R2L_SCAN_PAIR) return launch_pair<FWD>(a, p, nc, st, launches);
   if (DTMMA && R2L_SCAN_BCT) {
     using Sb = SmemBct;
     if ((e = prep_bct_kernel<true, FWD>()) != cudaSuccess) return e;

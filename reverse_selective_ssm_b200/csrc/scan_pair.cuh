@@ -175,13 +175,15 @@ __device__ __forceinline__ void pair_decays(const PCtx& cx, float dec, float2 (&
 }
 
 // One tile of 16 tokens as four sub-tiles of GT tokens; each pair of
-// sub-tiles reads one B|C group (TMEM region g = sub-tile / 2).  Tokens outside [jlo, jhi) (a tile that crosses the
-// sequence's start or end) leave the state untouched and write nothing.
-template <bool POW, bool FULL, bool FWD>
-__device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const bf16* su, bf16* sz, bf16* yg,
-                                          long long ldy, bool store_ok, int jlo, int jhi, const float (&dto)[8],
-                                          uint32_t ph, uint64_t* bcready, uint64_t* bcfree, uint32_t t_bc,
-                                          unsigned* err, bool& ok) {
+// sub-tiles reads one B|C group (TMEM region g = sub-tile / 2).  Tokens
+// outside [jlo, jhi) (a tile that crosses the chunk's start or end) leave the
+// state untouched and write nothing.  Without FINAL (the chunked scheme's
+// first pass) only the state and this thread's Σ Δ over its tokens advance.
+template <bool FINAL, bool POW, bool FULL, bool FWD>
+__device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float& sumd, const bf16* su, bf16* sz,
+                                          bf16* yg, long long ldy, bool store_ok, int jlo, int jhi,
+                                          const float (&dto)[8], uint32_t ph, uint64_t* bcready, uint64_t* bcfree,
+                                          uint32_t t_bc, unsigned* err, bool& ok) {
   const int lane = threadIdx.x & 31;
   const int h = lane >> 4;
 #pragma unroll
@@ -200,8 +202,12 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
       const bool valid = FULL || (j >= jlo && j < jhi);
       dec_o[i] = valid ? (POW ? r : delta) : (POW ? 1.0f : 0.0f);
       du_o[i] = valid ? delta * uu : 0.0f;
-      Du_o[i] = cx.Dc * uu;
-      gz_o[i] = silu_fast(__bfloat162float(sz[j * CHP]));
+      if (FINAL) {
+        Du_o[i] = cx.Dc * uu;
+        gz_o[i] = silu_fast(__bfloat162float(sz[j * CHP]));
+      } else {
+        sumd += valid ? delta : 0.0f;
+      }
     }
     // every thread needs the decay and Δu of all GT tokens: even tokens from
     // lane j, odd tokens from lane j + 16
@@ -235,10 +241,12 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           H[q] = __ffma2_rn(a[q], H[q], __fmul2_rn(du2, make_float2(bv[2 * q], bv[2 * q + 1])));
-        float2 acc = __fmul2_rn(make_float2(bv[8], bv[9]), H[0]);
+        if (FINAL) {
+          float2 acc = __fmul2_rn(make_float2(bv[8], bv[9]), H[0]);
 #pragma unroll
-        for (int q = 1; q < 4; ++q) acc = __ffma2_rn(make_float2(bv[8 + 2 * q], bv[9 + 2 * q]), H[q], acc);
-        part[t] = acc.x + acc.y;
+          for (int q = 1; q < 4; ++q) acc = __ffma2_rn(make_float2(bv[8 + 2 * q], bv[9 + 2 * q]), H[q], acc);
+          part[t] = acc.x + acc.y;
+        }
       }
     }
     if (gs == GB / GT - 1) {                       // the group's last token is read
@@ -248,7 +256,7 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
     }
     // y of this thread's tokens: its half of ⟨C, H⟩ plus the partner's
 #pragma unroll
-    for (int i = 0; i < GT / 2; ++i) {
+    for (int i = 0; i < (FINAL ? GT / 2 : 0); ++i) {
       const float give = h ? part[2 * i] : part[2 * i + 1];       // the partner's token
       const float mine = h ? part[2 * i + 1] : part[2 * i];
       const float other = __shfl_xor_sync(0xffffffffu, give, 16);
@@ -263,8 +271,8 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], const 
   }
 }
 
-template <bool POW, bool FWD>
-__device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], uint8_t* smem, uint64_t* full,
+template <bool FINAL, bool POW, bool FWD>
+__device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], float& sumd, uint8_t* smem, uint64_t* full,
                                              uint64_t* empty, uint64_t* dtready, uint64_t* bcready, uint64_t* bcfree,
                                              uint32_t tmem_base, int ntiles, int s0, int e0, int b, int c, int cl,
                                              bool cvalid, const Params& p) {
@@ -308,21 +316,24 @@ __device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], uin
     bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
     const uint32_t gph = (uint32_t)it & 1u;   // each group region is used once per tile
     if (full_tile)
-      pair_tile<POW, true, FWD>(cx, H, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready, bcfree,
-                                t_lane + P_BC_COL0, p.err, ok);
+      pair_tile<FINAL, POW, true, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready, bcfree,
+                                       t_lane + P_BC_COL0, p.err, ok);
     else
-      pair_tile<POW, false, FWD>(cx, H, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready, bcfree,
-                                 t_lane + P_BC_COL0, p.err, ok);
+      pair_tile<FINAL, POW, false, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready,
+                                        bcfree, t_lane + P_BC_COL0, p.err, ok);
     if (!ok) break;
-    if (full_tile) sm100::fence_proxy_async_smem();   // y tile visible to the TMA store
+    if (FINAL && full_tile) sm100::fence_proxy_async_smem();   // y tile visible to the TMA store
     sm100::tc_fence_before();
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[st]);
   }
 }
 
-// Final pass over whole sequences (one chunk per sequence, zero initial state).
-template <bool FWD>
+// One pass over chunk blockIdx.y of T tokens of every sequence (p.T, p.nc).
+// FINAL: y, starting from the carried state H_in(k) when sequences are split
+// (zero with one chunk).  Otherwise the chunked scheme's first pass: the
+// chunk's end state from a zero start and Σ Δ over it, into the carry buffer.
+template <bool FINAL, bool FWD>
 __global__ void __launch_bounds__(SmemPair::THREADS, 1)
 scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                  const __grid_constant__ CUtensorMap tm_dr, const __grid_constant__ CUtensorMap tm_bc,
@@ -340,12 +351,28 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
   uint64_t* bcfree = bcready + NG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::SLOT);
 
-  const int cb = blockIdx.x, b = blockIdx.z;
+  const int cb = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int n = p.len[b];
-  const int s0 = 0, e0 = n;
-  if (n <= 0) return;                          // nothing to read or write
+  const int s0 = k * p.T;
+  const int e0 = min(s0 + p.T, n);
+  if (s0 >= n) {                               // chunk entirely in the padding
+    if (!FINAL && tid < PTHREADS) {
+      const int q = warp & 3, pp = warp >> 2;
+      const int c = cb * CHP + 128 * (pp >> 1) + 32 * q + 16 * (pp & 1) + (lane & 15);
+      if (c < p.E) {
+        float* dst = p.carry + (((long long)b * p.nc + k) * p.E + c) * 16;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          dst[4 * kk + (lane >> 4)] = 0.0f;
+          dst[4 * kk + 2 + (lane >> 4)] = 0.0f;
+        }
+        if (lane < 16) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
+      }
+    }
+    return;
+  }
   const int ntiles = (e0 - s0 + TS - 1) / TS;
 
   if (tid == 0) {
@@ -370,7 +397,7 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
 
   if (warp == PWARPS) {
     if (lane == 0)
-      run_producer<S, true, true, FWD, CHP>(&tm_u, &tm_z, &tm_dr, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b,
+      run_producer<S, FINAL, true, FWD, CHP>(&tm_u, &tm_z, &tm_dr, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b,
                                             cb, s0, e0, ntiles, p);
     return;
   }
@@ -394,25 +421,41 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
   cx.Dc = cvalid ? p.D[c] : 0.0f;
   bool pow_ok = true;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int m = 4 * k + 2 * e + h;
+      const int m = 4 * kk + 2 * e + h;
       const float a = cvalid ? -expf(p.A_log[c * 16 + m]) : -(float)(m + 1);
-      cx.A2[2 * k + e] = a * LOG2E;
+      cx.A2[2 * kk + e] = a * LOG2E;
       pow_ok = pow_ok && fabsf(a + (float)(m + 1)) <= 1e-5f * (float)(m + 1);
     }
   }
   const bool use_pow = !p.force_general && __all_sync(0xffffffffu, pow_ok);
+  // the thread's states m = 4kk + 2e + h sit at H[kk].x (e = 0) and H[kk].y (e = 1)
   float2 H[4];
+  float* cst = (p.nc > 1 && cvalid) ? p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 : nullptr;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) H[k] = make_float2(0.0f, 0.0f);
+  for (int kk = 0; kk < 4; ++kk)
+    H[kk] = (FINAL && cst) ? make_float2(cst[4 * kk + h], cst[4 * kk + 2 + h]) : make_float2(0.0f, 0.0f);
+  float sumd = 0.0f;
   if (use_pow)
-    pair_compute<true, FWD>(cx, H, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0, e0, b, c, cl,
-                            cvalid, p);
+    pair_compute<FINAL, true, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
+                                   e0, b, c, cl, cvalid, p);
   else
-    pair_compute<false, FWD>(cx, H, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0, e0, b, c, cl,
-                             cvalid, p);
+    pair_compute<FINAL, false, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
+                                    e0, b, c, cl, cvalid, p);
+  if (!FINAL) {
+    // chunk end state S_k and Σ Δ (each thread summed Δ over its own tokens)
+    const float total = sumd + __shfl_xor_sync(0xffffffffu, sumd, 16);
+    if (cst) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        cst[4 * kk + h] = H[kk].x;
+        cst[4 * kk + 2 + h] = H[kk].y;
+      }
+      if (h == 0) p.carry_sum[((long long)b * p.nc + k) * p.E + c] = total;
+    }
+  }
   sm100::tc_fence_before();
   sm100::named_bar_sync(1, PTHREADS + 32);   // release TMEM to the dealloc
 }
