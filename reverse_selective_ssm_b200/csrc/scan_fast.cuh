@@ -22,7 +22,10 @@
 // [128 channels × R] in shared memory and, per tile, issues tcgen05.mma
 // (M = 128 channels, N = 16 tokens, K = R) into a TMEM column block; the
 // accumulator's lane is the channel, so each compute thread reads its 16
-// dt_raw values with one tcgen05.ld.  dt_raw never touches HBM.
+// dt_raw values with one tcgen05.ld.  dt_raw never touches HBM.  The layer
+// itself runs the DTMMA scan as the two-threads-per-channel kernel of
+// scan_pair.cuh; this one-thread DTMMA form is kept as its compile-time
+// alternative (R2L_SCAN_PAIR=0), and the form without DTMMA serves dt_rank ≠ 128.
 //
 // When a sequence is split into several chunks (to give the GPU enough
 // independent work), three launches cooperate through a small carry buffer:
@@ -482,378 +485,15 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constan
   }
 }
 
-// ---------------------------------------------------------------------------
-// B|C through tensor memory (dt_proj fused).  Every compute thread needs all
-// 32 values of B|C for every token; read from shared memory that is a 16-byte
-// broadcast load per four values, and the load/store pipe that serves it is
-// the kernel's busiest unit.  Here the tensor core does the broadcast: per
-// group of two tokens the MMA warp writes the 64 values as 64 rows of a K-major
-// tf32 operand, each value split into hi = its top 11 significant bits and
-// lo = value − hi (both exact tf32 up to the truncation of lo, so hi + lo
-// differs from the value by under 2⁻²¹ of it), and issues one
-// tcgen05.mma (M = 128, N = 64, K = 8) against an operand whose every row is
-// (1, 1, 0, …).  Accumulator lane c, column n then holds value n for every
-// channel c, and a thread reads a token's 32 values with one tcgen05.ld.
-// Groups cycle through NR TMEM regions of 64 columns after the 64 dt_raw
-// columns; bcready/bcfree barriers hand each region between the MMA warp and
-// the 4 compute warps.  y is written into the z tile it replaces (the same
-// thread read that z in phase A), and the TMA store takes it from there.
-constexpr int NR = 3;                                   // B|C regions in TMEM
-constexpr uint32_t BCT_COL0 = TMEM_COLS;                // first B|C column
-constexpr uint32_t BCT_TMEM_COLS = 256;                 // dt_raw 64 + NR × 64
+// Operands of the tensor-core broadcast of B|C (scan_pair.cuh): no-swizzle
+// K-major tf32 tiles with 32-byte rows.
 constexpr uint32_t OPB_BYTES = 64 * 32;                 // 64 rows × (8 tf32)
 constexpr uint32_t ONES_BYTES = 128 * 32;               // 128 rows × (8 tf32)
-static_assert(BCT_COL0 + NR * 64 <= BCT_TMEM_COLS, "TMEM budget");
-
-struct SmemBct {
-  static constexpr uint32_t W = 0;
-  static constexpr uint32_t DR = W_SLICE;
-  static constexpr uint32_t U = DR + STAGES * DR_TILE;
-  static constexpr uint32_t DT = U;                               // unused (dt_proj fused)
-  static constexpr uint32_t Z = U + STAGES * ACT_TILE;
-  static constexpr uint32_t Y = Z;                                // y overwrites z in place
-  static constexpr uint32_t BC = Z + STAGES * ACT_TILE;
-  static constexpr uint32_t ONES = BC + STAGES * BC_TILE;
-  static constexpr uint32_t OPB = ONES + ONES_BYTES;
-  static constexpr uint32_t BAR = OPB + NR * OPB_BYTES;           // full, empty, dtready [STAGES], wfull, drain, bcready, bcfree [NR]
-  static constexpr uint32_t SLOT = BAR + (3 * STAGES + 2 + 2 * NR) * 8;
-  static constexpr size_t BYTES = 1024 + SLOT + 16;
-  static constexpr int THREADS = CTHREADS + 64;
-};
 
 // Byte offset of row n of a no-swizzle K-major operand with 32-byte rows:
 // 8-row core matrices of 16-byte rows, the two 16-byte halves of a row 128
 // bytes apart (lbo), 8-row groups 256 bytes apart (sbo).
 __device__ __forceinline__ uint32_t opnd_row(int n) { return (uint32_t)((n >> 3) * 256 + (n & 7) * 16); }
-
-// The MMA warp: dt_raw per tile as in run_dt_mma, then the tile's eight B|C
-// groups in the order the compute warps consume them.
-template <bool FWD>
-__device__ __forceinline__ void run_mma_bct(uint8_t* smem, uint32_t tmem_base, uint64_t* full, uint64_t* dtready,
-                                            uint64_t* wfull, uint64_t* drain, uint64_t* bcready, uint64_t* bcfree,
-                                            int ntiles, unsigned* err) {
-  using S = SmemBct;
-  const int lane = threadIdx.x & 31;
-  for (int n = lane; n < 128; n += 32) {
-    uint8_t* row = smem + S::ONES + opnd_row(n);
-    *reinterpret_cast<float4*>(row) = make_float4(1.0f, 1.0f, 0.0f, 0.0f);
-    *reinterpret_cast<float4*>(row + 128) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  for (int n = lane; n < NR * 64; n += 32) {
-    uint8_t* row = smem + S::OPB + (n / 64) * OPB_BYTES + opnd_row(n % 64);
-    *reinterpret_cast<float4*>(row) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    *reinterpret_cast<float4*>(row + 128) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  sm100::fence_proxy_async_smem();
-  __syncwarp();
-  constexpr uint32_t idt = sm100::idesc_bf16_f32(128, TS);
-  constexpr uint32_t ibc = sm100::idesc_tf32_f32(128, 64);
-  const uint64_t a_ones = sm100::smem_desc_noswz(sm100::smem_u32(smem + S::ONES), 128, 256);
-  const uint32_t w0 = sm100::smem_u32(smem + S::W);
-  bool ok = sm100::mbar_wait(wfull, 0, err);
-  int r = 0;              // B|C region of the next group
-  uint32_t rph = 0;       // its use count, mod 2
-  for (int it = 0; it < ntiles && ok; ++it) {
-    const int st = it % STAGES;
-    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-    if (!sm100::mbar_wait(&full[st], ph, err)) break;
-    sm100::tc_fence_after();
-    if (lane == 0) {
-      const uint32_t d0 = sm100::smem_u32(smem + S::DR + st * DR_TILE);
-#pragma unroll
-      for (int k = 0; k < DT_R / 16; ++k) {
-        const uint32_t a_addr = w0 + (k / 4) * (CH * 128) + (k % 4) * 32;
-        const uint32_t b_addr = d0 + (k / 4) * (TS * 128) + (k % 4) * 32;
-        sm100::mma_bf16(tmem_base + (uint32_t)(st * TS), sm100::smem_desc_k128(a_addr),
-                        sm100::smem_desc_k128(b_addr), idt, k != 0);
-      }
-      sm100::mma_commit(&dtready[st]);
-    }
-    __syncwarp();
-    const float* bct = reinterpret_cast<const float*>(smem + S::BC + st * BC_TILE);
-    for (int q = 0; q < TS / 2; ++q) {
-      if (!sm100::mbar_wait(&bcfree[r], rph ^ 1u, err)) { ok = false; break; }
-      sm100::tc_fence_after();
-      const int t0 = FWD ? 2 * q : TS - 1 - 2 * q;          // first token the compute warps take
-      const int t1 = FWD ? 2 * q + 1 : TS - 2 - 2 * q;
-      uint8_t* opb = smem + S::OPB + r * OPB_BYTES;
-      const float x0 = bct[t0 * 32 + lane], x1 = bct[t1 * 32 + lane];
-      const float h0 = __uint_as_float(__float_as_uint(x0) & 0xFFFFE000u);
-      const float h1 = __uint_as_float(__float_as_uint(x1) & 0xFFFFE000u);
-      *reinterpret_cast<float2*>(opb + opnd_row(lane)) = make_float2(h0, x0 - h0);
-      *reinterpret_cast<float2*>(opb + opnd_row(32 + lane)) = make_float2(h1, x1 - h1);
-      sm100::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        sm100::mma_tf32(tmem_base + BCT_COL0 + (uint32_t)(r * 64), a_ones,
-                        sm100::smem_desc_noswz(sm100::smem_u32(opb), 128, 256), ibc, 0u);
-        sm100::mma_commit(&bcready[r]);
-      }
-      __syncwarp();
-      if (++r == NR) { r = 0; rph ^= 1u; }
-    }
-  }
-  if (lane == 0) {
-    sm100::mma_commit(drain);
-    sm100::mbar_wait(drain, 0, err, 1000000000ull);
-  }
-  __syncwarp();
-}
-
-// One token of the recurrence from its 32 B|C values in registers.
-template <bool FINAL, bool POW>
-__device__ __forceinline__ void bct_token(const Ctx& cx, float2 (&H)[8], float dec, float du, float Du, float gz,
-                                          const float (&bc)[32], bf16* ydst, bool store_ok) {
-  const float2 du2 = make_float2(du, du);
-  float2 a[8];
-  if (POW) {
-    const float r = dec;
-    const float r2 = r * r;
-    a[0] = make_float2(r, r2);
-    a[1] = __fmul2_rn(a[0], make_float2(r2, r2));
-    const float r4 = a[1].y;
-    a[2] = __fmul2_rn(a[0], make_float2(r4, r4));
-    a[3] = __fmul2_rn(a[1], make_float2(r4, r4));
-    const float r8 = a[3].y;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) a[4 + q] = __fmul2_rn(a[q], make_float2(r8, r8));
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      a[q] = make_float2(ex2_approx(dec * cx.A2[2 * q]), ex2_approx(dec * cx.A2[2 * q + 1]));
-  }
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-    H[q] = __ffma2_rn(a[q], H[q], __fmul2_rn(du2, make_float2(bc[2 * q], bc[2 * q + 1])));
-  if (FINAL) {
-    float2 acc0 = make_float2(Du, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc0 = __ffma2_rn(make_float2(bc[16 + 4 * q], bc[17 + 4 * q]), H[2 * q], acc0);
-      acc1 = __ffma2_rn(make_float2(bc[18 + 4 * q], bc[19 + 4 * q]), H[2 * q + 1], acc1);
-    }
-    const float s = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-    if (store_ok) *ydst = __float2bfloat16_rn(s * gz);
-  }
-}
-
-// One tile of 16 tokens for one compute thread: two sub-tiles of phase A, each
-// followed by its four B|C groups.  Returns false when a wait timed out.
-template <bool FINAL, bool POW, bool FULL, bool FWD>
-__device__ __forceinline__ bool bct_tile(const Ctx& cx, float2 (&H)[8], float& sumd, const bf16* su,
-                                         const float (&dtv)[16], bf16* sz, bf16* yg, long long ldy, bool store_ok,
-                                         int jlo, int jhi, int& r, uint32_t& rph, uint64_t* bcready, uint64_t* bcfree,
-                                         uint32_t t_bc, unsigned* err) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int sb = 0; sb < TS / SUB; ++sb) {
-    const int j0 = FWD ? sb * SUB : TS - SUB - sb * SUB;
-    const bool active = FULL || (j0 + SUB > jlo && j0 < jhi);
-    float dec[SUB], du[SUB], gz[SUB], Du[SUB];
-    if (active) {
-#pragma unroll
-      for (int t = 0; t < SUB; ++t) {
-        const int j = j0 + t;
-        if (!FULL && (j < jlo || j >= jhi)) continue;
-        float delta, r;
-        softplus_and_decay(dtv[j] + cx.dtb, delta, r);
-        const float uu = __bfloat162float(su[j * CH]);
-        dec[t] = POW ? r : delta;
-        du[t] = delta * uu;
-        if (FINAL) {
-          Du[t] = cx.Dc * uu;
-          gz[t] = silu_fast(__bfloat162float(sz[j * CH]));
-        } else {
-          sumd += delta;
-        }
-      }
-    }
-#pragma unroll
-    for (int gq = 0; gq < SUB / 2; ++gq) {
-      if (!sm100::mbar_wait(&bcready[r], rph, err)) return false;
-      __syncwarp();
-      sm100::tc_fence_after();
-#pragma unroll
-      for (int slot = 0; slot < 2; ++slot) {
-        const int t = FWD ? 2 * gq + slot : SUB - 1 - 2 * gq - slot;
-        const int j = j0 + t;
-        if (!active || (!FULL && (j < jlo || j >= jhi))) continue;
-        const uint32_t ta = t_bc + (uint32_t)(r * 64 + slot * 32);
-        float bc[32];
-        if (FINAL) {
-          sm100::tmem_ld32(ta, bc);
-        } else {
-          float b16[16];
-          sm100::tmem_ld16(ta, b16);
-#pragma unroll
-          for (int m = 0; m < 16; ++m) { bc[m] = b16[m]; bc[16 + m] = 0.0f; }
-        }
-        bf16* yd = FULL ? sz + j * CH : yg + (long long)j * ldy;
-        bct_token<FINAL, POW>(cx, H, dec[t], du[t], FINAL ? Du[t] : 0.0f, FINAL ? gz[t] : 0.0f, bc, yd, store_ok);
-      }
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&bcfree[r]);
-      if (++r == NR) { r = 0; rph ^= 1u; }
-    }
-  }
-  return true;
-}
-
-template <bool FINAL, bool POW, bool FWD>
-__device__ __forceinline__ void bct_compute(const Ctx& cx, float2 (&H)[8], float& sumd, uint8_t* smem,
-                                            uint64_t* full, uint64_t* empty, uint64_t* dtready, uint64_t* bcready,
-                                            uint64_t* bcfree, uint32_t tmem_base, int ntiles, int s0, int e0,
-                                            int b, int c, int ch, bool cvalid, const Params& p) {
-  using S = SmemBct;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t t_lane = tmem_base + ((uint32_t)(warp * 32) << 16);
-  float dtv[16];
-  int r = 0;
-  uint32_t rph = 0;
-  for (int it = 0; it < ntiles; ++it) {
-    const int st = it % STAGES;
-    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-    if (!sm100::mbar_wait(&full[st], ph, p.err)) break;
-    if (!sm100::mbar_wait(&dtready[st], ph, p.err)) break;
-    sm100::tc_fence_after();
-    sm100::tmem_ld16(t_lane + (uint32_t)(st * TS), dtv);
-    const int tbase = FWD ? s0 + it * TS : e0 - (it + 1) * TS;
-    const int jlo = (!FWD && s0 > tbase) ? s0 - tbase : 0;
-    const int jhi = (FWD && e0 - tbase < TS) ? e0 - tbase : TS;
-    const bool full_tile = jlo == 0 && jhi == TS;
-    const bf16* su = reinterpret_cast<const bf16*>(smem + S::U) + st * TS * CH + ch;
-    bf16* sz = reinterpret_cast<bf16*>(smem + S::Z) + st * TS * CH + ch;
-    bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
-    const bool ok = full_tile
-        ? bct_tile<FINAL, POW, true, FWD>(cx, H, sumd, su, dtv, sz, yg, p.ldy, cvalid, 0, TS, r, rph, bcready, bcfree,
-                                          t_lane + BCT_COL0, p.err)
-        : bct_tile<FINAL, POW, false, FWD>(cx, H, sumd, su, dtv, sz, yg, p.ldy, cvalid, jlo, jhi, r, rph, bcready,
-                                           bcfree, t_lane + BCT_COL0, p.err);
-    if (!ok) break;
-    if (FINAL && full_tile) sm100::fence_proxy_async_smem();   // y tile visible to the TMA store
-    sm100::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) sm100::mbar_arrive(&empty[st]);
-  }
-}
-
-template <bool FINAL, bool FWD>
-__global__ void __launch_bounds__(SmemBct::THREADS, 2)
-chunk_scan_bct_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
-                      const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_bc,
-                      const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
-                      const Params p) {
-  using S = SmemBct;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR);
-  uint64_t* empty = full + STAGES;
-  uint64_t* dtready = empty + STAGES;
-  uint64_t* wfull = dtready + STAGES;
-  uint64_t* drain = wfull + 1;
-  uint64_t* bcready = drain + 1;
-  uint64_t* bcfree = bcready + NR;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::SLOT);
-
-  const int cb = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const bool compute = tid < CTHREADS;
-  const int ch = compute ? tid : 0;
-  const int c = cb * CH + ch;
-  const bool cvalid = compute && c < p.E;
-  const int n = p.len[b];
-  const int s0 = k * p.T;
-  const int e0 = min(s0 + p.T, n);
-
-  if (s0 >= n) {
-    if (!FINAL && cvalid) {
-      float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      p.carry_sum[((long long)b * p.nc + k) * p.E + c] = 0.0f;
-    }
-    return;
-  }
-  const int ntiles = (e0 - s0 + TS - 1) / TS;
-
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      sm100::mbar_init(&full[s], 1);
-      sm100::mbar_init(&empty[s], CWARPS);
-      sm100::mbar_init(&dtready[s], 1);
-    }
-    sm100::mbar_init(wfull, 1);
-    sm100::mbar_init(drain, 1);
-    for (int r = 0; r < NR; ++r) {
-      sm100::mbar_init(&bcready[r], 1);
-      sm100::mbar_init(&bcfree[r], CWARPS);
-    }
-    sm100::fence_barrier_init();
-  }
-  if (warp == CWARPS + 1) sm100::tmem_alloc(tmem_slot, BCT_TMEM_COLS);
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == CWARPS) {
-    if (lane == 0)
-      run_producer<S, FINAL, true, FWD>(&tm_u, &tm_z, &tm_dt, &tm_bc, &tm_y, &tm_w, smem, full, empty, wfull, b, cb,
-                                        s0, e0, ntiles, p);
-    return;
-  }
-  if (warp == CWARPS + 1) {
-    run_mma_bct<FWD>(smem, tmem_base, full, dtready, wfull, drain, bcready, bcfree, ntiles, p.err);
-    sm100::named_bar_sync(1, CTHREADS + 32);   // every compute warp has finished reading TMEM
-    sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem_base, BCT_TMEM_COLS);
-    return;
-  }
-
-  Ctx cx;
-  cx.dtb = cvalid ? p.dt_b[c] : 0.0f;
-  cx.Dc = cvalid ? p.D[c] : 0.0f;
-  bool pow_ok = true;
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const float a = cvalid ? -expf(p.A_log[c * 16 + m]) : -(float)(m + 1);
-    cx.A2[m] = a * LOG2E;
-    pow_ok = pow_ok && fabsf(a + (float)(m + 1)) <= 1e-5f * (float)(m + 1);
-  }
-  const bool use_pow = !p.force_general && __all_sync(0xffffffffu, pow_ok);
-
-  float2 H[8];
-  if (FINAL && p.nc > 1 && cvalid) {
-    const float4* src = reinterpret_cast<const float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = src[q];
-      H[2 * q] = make_float2(v.x, v.y);
-      H[2 * q + 1] = make_float2(v.z, v.w);
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) H[q] = make_float2(0.0f, 0.0f);
-  }
-  float sumd = 0.0f;
-  if (use_pow)
-    bct_compute<FINAL, true, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
-                                  e0, b, c, ch, cvalid, p);
-  else
-    bct_compute<FINAL, false, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
-                                   e0, b, c, ch, cvalid, p);
-
-  if (!FINAL && cvalid) {
-    float4* dst = reinterpret_cast<float4*>(p.carry + (((long long)b * p.nc + k) * p.E + c) * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_float4(H[2 * q].x, H[2 * q].y, H[2 * q + 1].x, H[2 * q + 1].y);
-    p.carry_sum[((long long)b * p.nc + k) * p.E + c] = sumd;
-  }
-  sm100::tc_fence_before();
-  sm100::named_bar_sync(1, CTHREADS + 32);   // release TMEM to the dealloc
-}
 
 // Per (sequence, channel): turn chunk end states S_k into the states entering
 // each chunk from the right (from the left with fwd), in place (see the

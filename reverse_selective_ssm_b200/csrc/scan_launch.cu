@@ -55,12 +55,8 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens, bool pair) {
 
 namespace {
 
-// B|C delivered through tensor memory in the fused-dt_proj scan (0: shared memory).
-#ifndef R2L_SCAN_BCT
-#define R2L_SCAN_BCT 1
-#endif
-
-// Two threads per channel for single-pass scans with dt_proj fused (0: off).
+// Two threads per channel, B|C broadcast through tensor memory, for scans with
+// dt_proj fused (0: one thread per channel, B|C read from shared memory).
 #ifndef R2L_SCAN_PAIR
 #define R2L_SCAN_PAIR 1
 #endif
@@ -99,12 +95,6 @@ cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaS
   return cudaSuccess;
 }
 
-template <bool FINAL, bool FWD>
-cudaError_t prep_bct_kernel() {
-  return cudaFuncSetAttribute(rscan::chunk_scan_bct_kernel<FINAL, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)rscan::SmemBct::BYTES);
-}
-
 template <bool FINAL, bool DTMMA, bool FWD>
 cudaError_t prep_kernel() {
   return cudaFuncSetAttribute(rscan::chunk_scan_kernel<FINAL, DTMMA, FWD>,
@@ -133,22 +123,6 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
   cudaError_t e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
   if (DTMMA && R2L_SCAN_PAIR) return launch_pair<FWD>(a, p, nc, st, launches);
-  if (DTMMA && R2L_SCAN_BCT) {
-    using Sb = SmemBct;
-    if ((e = prep_bct_kernel<true, FWD>()) != cudaSuccess) return e;
-    if (nc > 1) {
-      if ((e = prep_bct_kernel<false, FWD>()) != cudaSuccess) return e;
-      chunk_scan_bct_kernel<false, FWD><<<grid, Sb::THREADS, Sb::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
-      if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-      chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
-      if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-      if (launches) *launches += 2;
-    }
-    chunk_scan_bct_kernel<true, FWD><<<grid, Sb::THREADS, Sb::BYTES, st>>>(tu, tz, tdt, tbc, ty, tw, p);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-    if (launches) *launches += 1;
-    return cudaSuccess;
-  }
   if ((e = prep_kernel<true, DTMMA, FWD>()) != cudaSuccess) return e;
   if (nc > 1) {
     if ((e = prep_kernel<false, DTMMA, FWD>()) != cudaSuccess) return e;
