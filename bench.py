@@ -109,25 +109,74 @@ def read_traffic(stage, workload_tag):
 
 
 class ClockSampler:
+    """SM clock and clock-event reasons of this rank's GPU, read (never set)
+    every few milliseconds between start() and stop(): through NVML on a
+    thread when pynvml imports, else from an ``nvidia-smi -lms`` child."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): SwPowerCap, HwSlowdown, SwThermal, HwThermal
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                   ("hw_thermal_slowdown", 0x40))
+    PERIOD_S = 0.005
 
     def __init__(self, local_rank):
         vis = os.environ.get("CUDA_VISIBLE_DEVICES")
         self.gpu = vis.split(",")[local_rank].strip() if vis else str(local_rank)
         self.proc = None
+        self.thread = None
+        self.samples = []
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.gpu.startswith("GPU-") or self.gpu.startswith("MIG-"):
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.gpu)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu))
 
     def start(self):
+        import threading
+        try:
+            nv, hnd = self._nvml_handle()
+        except Exception:
+            nv = None
+        if nv is not None:
+            self.stop_event = threading.Event()
+            smax = nv.nvmlDeviceGetMaxClockInfo(hnd, nv.NVML_CLOCK_SM)
+
+            def loop():
+                while not self.stop_event.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(hnd, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(hnd) \
+                            if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons") \
+                            else nv.nvmlDeviceGetCurrentClocksThrottleReasons(hnd)
+                        self.samples.append((float(sm), float(smax), int(rs)))
+                    except Exception:
+                        pass
+                    self.stop_event.wait(self.PERIOD_S)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", self.gpu],
+                 "-lms", "50", "-i", self.gpu],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_event.set()
+            self.thread.join(timeout=5)
+            sm = [x[0] for x in self.samples]
+            smax = [x[1] for x in self.samples]
+            reasons = {n for _, _, r in self.samples for n, bit in self.REASON_BITS if r & bit}
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": max(smax) if smax else None,
+                    "reasons": sorted(reasons), "samples": len(sm), "source": "nvml"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -152,7 +201,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 def algorithmic(case, stage):
