@@ -25,6 +25,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100_primitives.cuh"
 
@@ -47,7 +49,9 @@ __device__ __forceinline__ bool rows_have_valid(const int* __restrict__ len, int
 // MB: 128-row MMA blocks per tile.  MB = 1 keeps two accumulators so one
 // tile's epilogue overlaps the next tile's MMAs; MB = 2 (BN = 256) fills all
 // 512 TMEM columns with one 256 × 256 tile, reading a third fewer operand
-// bytes per flop, and its epilogue waits for the tile's MMAs.
+// bytes per flop; its epilogue copies the accumulator into registers and
+// hands it back before staging and storing, so the next tile's MMAs wait
+// only for the TMEM reads.
 template <int BN, typename TOut, int MB = 1>
 struct TcGemmCfg {
   static constexpr int BM = 128 * MB;
@@ -268,6 +272,55 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0;
     uint32_t aphase = 0;
     int chunk = 0;
+    if constexpr (MB == 2) {
+      // One accumulator: read the thread's whole row (256 columns) out of
+      // TMEM as packed bf16 pairs, hand the accumulator back at once so the
+      // next tile's MMAs start, then stage and store the row from registers
+      // while they run.
+      static_assert(std::is_same<TOut, bf16>::value, "256 x 256 tiles store bf16");
+      for (long long t = blockIdx.x; t < total; t += gridDim.x) {
+        if (!tile_live(t)) continue;
+        if (!sm100::mbar_wait(&tfull[0], aphase, err)) break;
+        sm100::tc_fence_after();
+        const long long tile = t / splits;
+        const int mb = (int)(tile / num_n), nb = (int)(tile % num_n);
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float v[32];
+          sm100::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN + c0), v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            pk[c0 / 2 + j] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        }
+        sm100::tc_fence_before();
+        sm100::mbar_arrive(&tempty[0]);
+        aphase ^= 1u;
+        const int row0 = mb * BM + h * 128 + q * 32;
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32, ++chunk) {
+          uint8_t* buf = stg + (chunk & 1) * Cfg::STG_BYTES;
+          if (lane == 0) sm100::bulk_wait_read_le1();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int pkk = k ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + pkk * 16) =
+                make_uint4(pk[c0 / 2 + 4 * k], pk[c0 / 2 + 4 * k + 1], pk[c0 / 2 + 4 * k + 2], pk[c0 / 2 + 4 * k + 3]);
+          }
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          const int col = nb * BN + c0;
+          if (lane == 0 && col < N && row0 < M) {
+            sm100::tma_store_2d(&tmC, buf, col, row0);
+            sm100::bulk_commit();
+          }
+        }
+      }
+      if (lane == 0) sm100::bulk_wait_all();
+    } else
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       if (!tile_live(t)) continue;
       if (!sm100::mbar_wait(&tfull[acc], aphase, err)) break;
@@ -310,7 +363,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       sm100::mbar_arrive(&tempty[acc]);
       if (++acc == NACC) { acc = 0; aphase ^= 1u; }
     }
-    if (lane == 0) sm100::bulk_wait_all();
+    if (MB == 1 && lane == 0) sm100::bulk_wait_all();
   }
 
   sm100::tc_fence_before();
