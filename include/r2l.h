@@ -247,6 +247,45 @@ R2L_API r2l_status r2l_reverse_scan_noalloc(const void *u, const void *z, int ld
                                             const float *dt_b, void *y, const r2l_dims *dims, int B, int L,
                                             const int32_t *lengths, int chunk_tokens, void *stream);
 
+/* Bytes of device workspace r2l_reverse_scan_backward needs for a [B, L]
+ * batch split into chunks of chunk_tokens positions (0 = automatic, 16).
+ * 0 for invalid or unsupported input (see r2l_reverse_scan_backward).       */
+R2L_API size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims *dims, int B, int L, int chunk_tokens);
+
+/* Gradient of r2l_reverse_scan (the scan of §3.4 step ❷ with its softplus(Δ)
+ * input and SiLU(z) gate), the step that training the sidecar alone
+ * back-propagates through.  For dy = ∂L/∂y it returns, with the forward's
+ * notation (a_i = exp(Δ_i A), G_i = ∂L/∂H_i = a_{i-1} ⊙ G_{i-1} + dp_i C_i,
+ * dp_i = dy_i ⊙ SiLU(z_i)):
+ *
+ *   du      [B·L, E]   D ⊙ dp_i + Δ_i ⊙ Σ_m G_i[:,m] B_i[m]
+ *   ddt_raw [B·L, E]   (Σ_m G_i ⊙ H_{i+1} ⊙ a_i ⊙ A + u_i ⊙ Σ_m G_i B_i) ⊙ softplus'(dt_raw_i + dt_b)
+ *   dz      [B·L, ld_dz] first E columns: dy_i ⊙ p_i ⊙ SiLU'(z_i), p_i = H_i·C_i + D ⊙ u_i
+ *   dbc     [B·L, ld_dbc] columns 0..15 dB_i = Σ_e G_i Δ_i u_i, 16..31 dC_i = Σ_e dp_i H_i
+ *   dA_log  [E, 16]    A ⊙ Σ_i Δ_i ⊙ G_i ⊙ H_{i+1} ⊙ a_i   (summed over the batch)
+ *   dD, ddt_b [E]      Σ_i dp_i ⊙ u_i,  Σ_i ddt_raw_i        (summed over the batch)
+ *
+ * Rows i ≥ len_b of du, ddt_raw, dz and dbc are written with zeros.  Inputs
+ * are those of r2l_reverse_scan (u, z, dt_raw, bc, A_log, D, dt_b, lengths)
+ * plus dy [B·L, E].  Every reduction runs in a fixed order: the results are
+ * bitwise reproducible for a given chunk_tokens.
+ *
+ * Supported: dims->dtype == R2L_FP32 (every activation array is fp32),
+ * d_state == 16, d_inner a multiple of 64, the right-to-left block (the
+ * R2L_FLAG_FORWARD_SCAN flag returns R2L_ERR_UNSUPPORTED); ldz and ldbc
+ * multiples of 4.  chunk_tokens: positions per chunk (1 … 32; larger values are
+ * clamped to 32; 0 = 16).  workspace ≥
+ * r2l_reverse_scan_backward_workspace_size(dims, B, L, chunk_tokens) bytes,
+ * 16-byte aligned; its first 16 bytes are the device status word that
+ * r2l_get_device_status reads.  Device pointers, 16-byte aligned.          */
+R2L_API r2l_status r2l_reverse_scan_backward(const void *u, const void *z, int ldz, const void *dt_raw,
+                                             const float *bc, int ldbc, const float *A_log, const float *D,
+                                             const float *dt_b, const void *dy, void *du, void *dz, int ld_dz,
+                                             void *ddt_raw, float *dbc, int ld_dbc, float *dA_log, float *dD,
+                                             float *ddt_b, const r2l_dims *dims, int B, int L,
+                                             const int32_t *lengths, int chunk_tokens, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
 /* Synchronises `stream`, then reads the device status word that the last
  * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*
  * bits.  Returns R2L_ERR_DEVICE_CHECK if any bit is set, R2L_ERR_CUDA if the

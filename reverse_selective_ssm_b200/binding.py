@@ -27,7 +27,8 @@ STATUS = {0: "R2L_OK", 1: "R2L_ERR_INVALID_ARG", 2: "R2L_ERR_UNSUPPORTED", 3: "R
 EXPORTS = ("r2l_abi_version", "r2l_status_string", "r2l_workspace_size", "r2l_sidecar_forward",
            "r2l_sidecar_forward_debug", "r2l_sidecar_forward_profiled", "r2l_sidecar_stack",
            "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan",
-           "r2l_reverse_scan_noalloc")
+           "r2l_reverse_scan_noalloc", "r2l_reverse_scan_backward_workspace_size",
+           "r2l_reverse_scan_backward")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -98,6 +99,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.r2l_reverse_scan_noalloc.restype = ci
     lib.r2l_reverse_scan_noalloc.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, ctypes.POINTER(Dims), ci,
                                              ci, vp, ci, vp]
+    lib.r2l_reverse_scan_backward_workspace_size.restype = ctypes.c_size_t
+    lib.r2l_reverse_scan_backward_workspace_size.argtypes = [ctypes.POINTER(Dims), ci, ci, ci]
+    lib.r2l_reverse_scan_backward.restype = ci
+    lib.r2l_reverse_scan_backward.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, vp, vp, ci, vp, vp, ci,
+                                              vp, vp, vp, ctypes.POINTER(Dims), ci, ci, vp, ci, vp,
+                                              ctypes.c_size_t, vp]
     lib.r2l_get_device_status.restype = ci
     lib.r2l_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -259,6 +266,33 @@ def reverse_scan_noalloc(u: torch.Tensor, z: torch.Tensor, dt_raw: torch.Tensor,
                                       _ptr(lengths), chunk_tokens, _stream_ptr(stream))
     if check and st != 0:
         raise R2LError(st, "r2l_reverse_scan_noalloc")
+    return st
+
+
+def reverse_scan_backward_workspace_size(dims: Dims, B: int, L: int, chunk_tokens: int = 0) -> int:
+    return int(load().r2l_reverse_scan_backward_workspace_size(ctypes.byref(dims), B, L, chunk_tokens))
+
+
+def reverse_scan_backward(u: torch.Tensor, z: torch.Tensor, dt_raw: torch.Tensor, bc: torch.Tensor,
+                          A_log: torch.Tensor, D: torch.Tensor, dt_b: torch.Tensor, dy: torch.Tensor,
+                          du: torch.Tensor, dz: torch.Tensor, ddt_raw: torch.Tensor, dbc: torch.Tensor,
+                          dA_log: torch.Tensor, dD: torch.Tensor, ddt_b: torch.Tensor, dims: Dims, B: int, L: int,
+                          lengths=None, chunk_tokens: int = 0, workspace: Optional[torch.Tensor] = None,
+                          stream=None, check: bool = True) -> int:
+    """r2l_reverse_scan_backward (fp32).  u, dt_raw, dy, du, ddt_raw: [B·L, E];
+    z, dz: [B·L, ld] (first E columns); bc, dbc: [B·L, ld] with B in columns
+    0..15 and C in 16..31; dA_log [E, 16]; dD, ddt_b [E]."""
+    lib = load()
+    if workspace is None:
+        n = reverse_scan_backward_workspace_size(dims, B, L, chunk_tokens)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=u.device)
+    st = lib.r2l_reverse_scan_backward(_ptr(u), _ptr(z), z.stride(0), _ptr(dt_raw), _ptr(bc), bc.stride(0),
+                                       _ptr(A_log), _ptr(D), _ptr(dt_b), _ptr(dy), _ptr(du), _ptr(dz), dz.stride(0),
+                                       _ptr(ddt_raw), _ptr(dbc), dbc.stride(0), _ptr(dA_log), _ptr(dD),
+                                       _ptr(ddt_b), ctypes.byref(dims), B, L, _ptr(lengths), chunk_tokens,
+                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if check and st != 0:
+        raise R2LError(st, "r2l_reverse_scan_backward")
     return st
 
 

@@ -16,6 +16,7 @@
 #include "scan_simple.cuh"
 #include "tc_gemm.h"
 #include "scan_fast.h"
+#include "scan_bwd.h"
 #include "conv_fast.cuh"
 
 // conv + SiLU fused into the x_proj GEMM on the bf16 path (0: separate kernels).
@@ -495,6 +496,53 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
                                                          (dims->flags & R2L_FLAG_FORWARD_SCAN) != 0);
     R2L_LAUNCH_CHECK();
   }
+  return R2L_OK;
+}
+
+size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims* dims, int B, int L, int chunk_tokens) {
+  if (!dims || B <= 0 || L <= 0 || dims->d_inner <= 0 || chunk_tokens < 0) return 0;
+  if (dims->dtype != R2L_FP32 || dims->d_state != 16 || dims->d_inner % 64) return 0;
+  return align_up(16, kAlign) + align_up(r2l::scan_bwd_scratch_bytes(B, L, dims->d_inner, chunk_tokens), kAlign);
+}
+
+r2l_status r2l_reverse_scan_backward(const void* u, const void* z, int ldz, const void* dt_raw, const float* bc,
+                                     int ldbc, const float* A_log, const float* D, const float* dt_b,
+                                     const void* dy, void* du, void* dz, int ld_dz, void* ddt_raw, float* dbc,
+                                     int ld_dbc, float* dA_log, float* dD, float* ddt_b, const r2l_dims* dims,
+                                     int B, int L, const int32_t* lengths, int chunk_tokens, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!u || !z || !dt_raw || !bc || !A_log || !D || !dt_b || !dy || !du || !dz || !ddt_raw || !dbc || !dA_log ||
+      !dD || !ddt_b || !dims)
+    return R2L_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0 || dims->d_inner <= 0 || chunk_tokens < 0) return R2L_ERR_INVALID_ARG;
+  if (dims->dtype != R2L_BF16 && dims->dtype != R2L_FP32) return R2L_ERR_INVALID_ARG;
+  if (dims->dtype != R2L_FP32 || dims->d_state != 16 || (dims->flags & R2L_FLAG_FORWARD_SCAN))
+    return R2L_ERR_UNSUPPORTED;
+  const int E = dims->d_inner;
+  if (E % 64) return R2L_ERR_UNSUPPORTED;
+  if (ldz < E || ld_dz < E || ldbc < 32 || ld_dbc < 32) return R2L_ERR_INVALID_ARG;
+  if ((ldbc % 4) || (ldz % 4)) return R2L_ERR_ALIGNMENT;
+  if (L > 65535 || B > 65535) return R2L_ERR_UNSUPPORTED;
+  for (const void* q : {u, z, dt_raw, (const void*)bc, (const void*)A_log, (const void*)D, (const void*)dt_b, dy,
+                        (const void*)du, (const void*)dz, (const void*)ddt_raw, (const void*)dbc,
+                        (const void*)dA_log, (const void*)dD, (const void*)ddt_b})
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
+  const size_t need = r2l_reverse_scan_backward_workspace_size(dims, B, L, chunk_tokens);
+  if (!workspace || workspace_bytes < need) return R2L_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return R2L_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  if (cudaMemsetAsync(ws, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
+  r2l::ScanBwdArgs a{};
+  a.u = (const float*)u; a.z = (const float*)z; a.ldz = ldz; a.dt_raw = (const float*)dt_raw;
+  a.bc = bc; a.ldbc = ldbc; a.A_log = A_log; a.D = D; a.dt_b = dt_b; a.dy = (const float*)dy;
+  a.du = (float*)du; a.dz = (float*)dz; a.ld_dz = ld_dz; a.ddt_raw = (float*)ddt_raw;
+  a.dbc = dbc; a.ld_dbc = ld_dbc; a.dA_log = dA_log; a.dD = dD; a.ddt_b = ddt_b;
+  a.B = B; a.L = L; a.E = E; a.chunk_tokens = chunk_tokens;
+  a.lengths = lengths;
+  a.status = (unsigned*)ws;
+  if (r2l::scan_bwd_f32(a, ws + align_up(16, kAlign), st) != cudaSuccess) return R2L_ERR_CUDA;
   return R2L_OK;
 }
 

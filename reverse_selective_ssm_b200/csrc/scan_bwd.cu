@@ -1,0 +1,564 @@
+// Gradient of the reverse selective scan (fp32), the step that training the
+// sidecar alone back-propagates through ("Bifocal Diffusion Language Models",
+// arXiv 2606.27732v1, §3.4 step ❷: the Mamba-1 scan run from each sequence's
+// last valid position to its first, with softplus(Δ) in front and the SiLU(z)
+// gate behind).  Forward, per sequence of n positions:
+//
+//   Δ_i = softplus(v_i), v_i = dt_raw_i + dt_b;   a_i = exp(Δ_i A), A = -exp(A_log)
+//   H_n = 0,  H_i = a_i ⊙ H_{i+1} + Δ_i u_i B_i;   p_i = ⟨C_i, H_i⟩ + D u_i;   y_i = p_i SiLU(z_i)
+//
+// Backward for dy = ∂L/∂y (chain rule):
+//
+//   dp_i = dy_i SiLU(z_i),  dz_i = dy_i p_i SiLU'(z_i)
+//   G_i  = ∂L/∂H_i = a_{i-1} ⊙ G_{i-1} + dp_i C_i,  G_{-1} = 0   (left to right)
+//   dΔ_i = Σ_m G_im H_{i+1,m} a_im A_m + u_i Σ_m G_im B_im,   ddt_raw_i = dΔ_i softplus'(v_i)
+//   du_i = D dp_i + Δ_i Σ_m G_im B_im
+//   dB_i = Σ_c G_i Δ_i u_i,   dC_i = Σ_c dp_i H_i                 (sums over channels)
+//   dA_log = A ⊙ Σ_i Δ_i G_i ⊙ H_{i+1} ⊙ a_i,  dD = Σ_i dp_i u_i,  ddt_b = Σ_i ddt_raw_i
+//
+// The adjoint G runs left to right while H runs right to left, so both are
+// split into chunks of T positions:
+//   1. hstate: each chunk scans H right to left from zero; stores its end
+//      state and Σ Δ over the chunk;
+//   2. hcarry: per (sequence, channel, state), the state entering each chunk
+//      from the right, H_in(k) = S_{k+1} + exp(A Σ_{k+1}Δ) H_in(k+1);
+//   3. gstate: each chunk runs G left to right from zero; stores its end value
+//      and Σ Δ over positions s-1 … e-2 (the decays it crossed);
+//   4. gcarry: G entering each chunk from the left, the same recurrence in
+//      the other direction;
+//   5. final: each chunk recomputes its H from H_in(k) into shared memory,
+//      then walks G from the carried value and writes every gradient;
+//   6. two fixed-order reductions: the per-chunk parameter partials and the
+//      per-block partial sums of dB | dC (deterministic, no atomics).
+//
+// Threads: four per channel, thread q holding states 4q … 4q+3 (float4 loads
+// of B, C and the state rows), 64 channels per 256-thread block.  Sums over
+// the four threads use two xor shuffles; the sum of dB | dC over a warp's 8
+// channels is a 7-shuffle reduce-scatter that leaves each lane one of the 32
+// columns.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "scan_bwd.h"
+
+namespace r2l {
+namespace sbwd {
+
+constexpr int CPB = 64;                   // channels per block
+constexpr int THREADS = CPB * 4;
+constexpr int WARPS = THREADS / 32;
+
+struct Args {
+  const float* u;
+  const float* z;
+  int ldz;
+  const float* dt;
+  const float* bc;
+  int ldbc;
+  const float* A_log;
+  const float* D;
+  const float* dt_b;
+  const float* dy;
+  float* du;
+  float* dz;
+  int ld_dz;
+  float* ddt;
+  float* dbc;
+  int ld_dbc;
+  float* dA_log;
+  float* dD;
+  float* ddt_b;
+  int B, L, E, T, nc;
+  const int* lengths;      // caller's lengths, or null
+  unsigned* status;
+  float* hcar;             // [B][nc][E][16]: chunk end states, then H_in(k)
+  float* hsd;              // [B][nc][E]
+  float* gcar;             // [B][nc][E][16]: chunk end adjoints, then G entering from the left
+  float* gsd;              // [B][nc][E]
+  float* pA;               // [B][nc][E][16] Σ Δ G H_{i+1} a over the chunk
+  float* pD;               // [B][nc][E]
+  float* pb;               // [B][nc][E]
+  float* pbc;              // [E/CPB][B·L][32] per-block partial dB | dC
+};
+
+__device__ __forceinline__ int seq_len(const Args& a, int b) {
+  int n = a.lengths ? a.lengths[b] : a.L;
+  if (n < 0 || n > a.L) {
+    if (a.status && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(a.status, 0x1u);   // R2L_DEVFLAG_LENGTH_CLAMPED
+    n = n < 0 ? 0 : a.L;
+  }
+  return n;
+}
+
+__device__ __forceinline__ float softplus_fwd(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
+__device__ __forceinline__ float softplus_grad(float v) { return v > 20.0f ? 1.0f : 1.0f / (1.0f + expf(-v)); }
+
+// 2^x on the MUFU unit (ex2.approx, relative error about 2^-22): the decays
+// a = exp(Δ A) = 2^(Δ · A log2 e).
+__device__ __forceinline__ float exp2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float get(const float4& v, int j) { return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w; }
+
+__device__ __forceinline__ float sum4(float v) {         // over the channel's four threads
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
+}
+
+struct Lane {
+  int c, q, b, k, s, e, n;
+  float A[4];    // A_m of the thread's states
+  float A2[4];   // A_m · log2 e
+};
+
+__device__ __forceinline__ Lane lane_setup(const Args& a) {
+  Lane l;
+  l.c = blockIdx.x * CPB + (threadIdx.x >> 2);
+  l.q = threadIdx.x & 3;
+  l.k = blockIdx.y;
+  l.b = blockIdx.z;
+  l.n = seq_len(a, l.b);
+  l.s = l.k * a.T;
+  l.e = min(l.s + a.T, l.n);
+  const float4 al = ld4(a.A_log + (size_t)l.c * 16 + 4 * l.q);
+  l.A[0] = -expf(al.x); l.A[1] = -expf(al.y); l.A[2] = -expf(al.z); l.A[3] = -expf(al.w);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) l.A2[j] = l.A[j] * kLog2e;
+  return l;
+}
+
+__device__ __forceinline__ size_t carry_idx(const Args& a, const Lane& l) {
+  return (((size_t)l.b * a.nc + l.k) * a.E + l.c);
+}
+
+// Per-(position, channel) scalars of a chunk for the block's 64 channels,
+// rows [s, e): computed once per element by the whole block from coalesced
+// float4 reads (instead of once per state-holding thread), so the
+// per-position loops below read shared memory only.  Arrays are [T][64]
+// (row r = position s + r); bc is the raw [T][32] B | C rows.
+//   U = u, DL = Δ, DU = Δ u, DP = dp = dy SiLU(z), FZ = dy SiLU'(z) (dz = p FZ),
+//   SG = softplus'(v)
+enum : unsigned { S_U = 1, S_DL = 2, S_DU = 4, S_DP = 8, S_FZ = 16, S_SG = 32 };
+constexpr int NSTAGE = 6;
+
+struct Stage {
+  float* arr[NSTAGE];
+  float* bc;
+};
+
+__device__ __forceinline__ Stage stage_layout(float* base, int T) {
+  Stage st;
+#pragma unroll
+  for (int k = 0; k < NSTAGE; ++k) st.arr[k] = base + (size_t)k * T * CPB;
+  st.bc = base + (size_t)NSTAGE * T * CPB;
+  return st;
+}
+
+constexpr size_t stage_floats(int T) { return (size_t)T * (NSTAGE * CPB + 32); }
+
+template <unsigned WANT>
+__device__ __forceinline__ void stage_chunk(const Args& a, const Lane& l, const Stage& st) {
+  const int nrows = l.e - l.s;
+  if (nrows <= 0) return;
+  const long long row0 = (long long)l.b * a.L + l.s;
+  const int col0 = blockIdx.x * CPB;
+  constexpr bool NEED_U = WANT & (S_U | S_DU);
+  constexpr bool NEED_Z = WANT & (S_DP | S_FZ);
+  for (int t = threadIdx.x; t < nrows * (CPB / 4); t += THREADS) {
+    const int r = t / (CPB / 4), q4 = t % (CPB / 4);
+    const long long row = row0 + r;
+    const int col = col0 + 4 * q4;
+    const float4 dtb = ld4(a.dt_b + col);
+    const float4 v4 = ld4(a.dt + row * a.E + col);
+    float4 u4 = make_float4(0.f, 0.f, 0.f, 0.f), z4 = u4, dy4 = u4;
+    if (NEED_U) u4 = ld4(a.u + row * a.E + col);
+    if (NEED_Z) {
+      z4 = ld4(a.z + row * a.ldz + col);
+      dy4 = ld4(a.dy + row * a.E + col);
+    }
+    float o[NSTAGE][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float v = get(v4, j) + get(dtb, j);
+      const float delta = softplus_fwd(v);
+      const float uu = get(u4, j), zz = get(z4, j), dyy = get(dy4, j);
+      const float sg = 1.0f / (1.0f + expf(-zz));
+      o[0][j] = uu;
+      o[1][j] = delta;
+      o[2][j] = delta * uu;
+      o[3][j] = dyy * zz * sg;
+      o[4][j] = dyy * sg * (1.0f + zz * (1.0f - sg));
+      o[5][j] = (WANT & S_SG) ? softplus_grad(v) : 0.0f;
+    }
+    const int off = r * CPB + 4 * q4;
+#pragma unroll
+    for (int k = 0; k < NSTAGE; ++k)
+      if (WANT & (1u << k)) st4(st.arr[k] + off, make_float4(o[k][0], o[k][1], o[k][2], o[k][3]));
+  }
+  for (int t = threadIdx.x; t < nrows * 8; t += THREADS) {
+    const int r = t >> 3, q4 = t & 7;
+    st4(st.bc + r * 32 + 4 * q4, ld4(a.bc + (row0 + r) * a.ldbc + 4 * q4));
+  }
+}
+
+// 1. H right to left over the chunk from zero.
+__global__ void __launch_bounds__(THREADS) hstate_kernel(const Args a) {
+  extern __shared__ float4 sm4[];
+  const Lane l = lane_setup(a);
+  const Stage sg = stage_layout(reinterpret_cast<float*>(sm4), a.T);
+  stage_chunk<S_DL | S_DU>(a, l, sg);
+  __syncthreads();
+  const size_t ci = carry_idx(a, l);
+  const int ch = threadIdx.x >> 2;
+  float H[4] = {0.f, 0.f, 0.f, 0.f};
+  float sd = 0.0f;
+  for (int i = l.e - 1; i >= l.s; --i) {
+    const int r = i - l.s;
+    const float delta = sg.arr[1][r * CPB + ch];
+    const float du = sg.arr[2][r * CPB + ch];
+    const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+    sd += delta;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) H[j] = fmaf(exp2_mufu(delta * l.A2[j]), H[j], du * get(Bq, j));
+  }
+  st4(a.hcar + ci * 16 + 4 * l.q, make_float4(H[0], H[1], H[2], H[3]));
+  if (l.q == 0) a.hsd[ci] = sd;
+}
+
+// 2. / 4. Carries over the chunks of one (sequence, channel, state): right to
+// left for H (rev), left to right for G.  buf[k] ← value entering chunk k,
+// running = buf_old[k] + exp(A·sd[k]) · running.
+__global__ void carry_kernel(const Args a, float* buf, const float* sd, bool rev) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // c·16 + m
+  const int b = blockIdx.y;
+  if (t >= (long long)a.E * 16) return;
+  const int c = (int)(t >> 4), m = (int)(t & 15);
+  const float A = -expf(a.A_log[(size_t)c * 16 + m]);
+  float run = 0.0f;
+  constexpr int PF = 8;                    // chunks whose loads are issued together
+  for (int s0 = 0; s0 < a.nc; s0 += PF) {
+    float old[PF], dec[PF];
+#pragma unroll
+    for (int j = 0; j < PF; ++j) {
+      const int step = s0 + j;
+      const int k = rev ? a.nc - 1 - step : step;
+      const size_t ci = ((size_t)b * a.nc + (step < a.nc ? k : 0)) * a.E + c;
+      old[j] = step < a.nc ? buf[ci * 16 + m] : 0.0f;
+      dec[j] = step < a.nc ? sd[ci] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < PF; ++j) {
+      const int step = s0 + j;
+      if (step < a.nc) {
+        const int k = rev ? a.nc - 1 - step : step;
+        buf[(((size_t)b * a.nc + k) * a.E + c) * 16 + m] = run;
+        run = fmaf(expf(A * dec[j]), run, old[j]);
+      }
+    }
+  }
+}
+
+// 3. G left to right over the chunk from zero.
+__global__ void __launch_bounds__(THREADS) gstate_kernel(const Args a) {
+  extern __shared__ float4 sm4[];
+  const Lane l = lane_setup(a);
+  const Stage sg = stage_layout(reinterpret_cast<float*>(sm4), a.T);
+  stage_chunk<S_DL | S_DP>(a, l, sg);
+  const size_t ci = carry_idx(a, l);
+  const int ch = threadIdx.x >> 2;
+  float G[4] = {0.f, 0.f, 0.f, 0.f};
+  float sd = 0.0f, prev = 0.0f;
+  if (l.s > 0 && l.s < l.e) prev = softplus_fwd(a.dt[((size_t)l.b * a.L + l.s - 1) * a.E + l.c] + a.dt_b[l.c]);
+  __syncthreads();
+  for (int i = l.s; i < l.e; ++i) {
+    const int r = i - l.s;
+    const float delta = sg.arr[1][r * CPB + ch];
+    const float dp = sg.arr[3][r * CPB + ch];
+    const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
+    if (i > l.s) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) G[j] *= exp2_mufu(prev * l.A2[j]);
+    }
+    if (i > l.s || l.s > 0) sd += prev;                  // decays crossed: positions s-1 … e-2
+#pragma unroll
+    for (int j = 0; j < 4; ++j) G[j] = fmaf(dp, get(Cq, j), G[j]);
+    prev = delta;
+  }
+  st4(a.gcar + ci * 16 + 4 * l.q, make_float4(G[0], G[1], G[2], G[3]));
+  if (l.q == 0) a.gsd[ci] = sd;
+}
+
+// 5. Per chunk: H from H_in(k) into shared memory (right to left), then G
+// from the carried value (left to right) with every gradient.
+__global__ void __launch_bounds__(THREADS) final_kernel(const Args a) {
+  extern __shared__ float4 sm4[];
+  float4* Hs = sm4;                                              // [T][THREADS]
+  float* red = reinterpret_cast<float*>(sm4 + (size_t)a.T * THREADS);   // [WARPS][T][32]
+  const Lane l = lane_setup(a);
+  const Stage sg = stage_layout(red + (size_t)WARPS * a.T * 32, a.T);
+  stage_chunk<S_U | S_DL | S_DU | S_DP | S_FZ | S_SG>(a, l, sg);
+  const size_t ci = carry_idx(a, l);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ch = threadIdx.x >> 2;
+  const float Dc = a.D[l.c];
+  const float4 Hr = ld4(a.hcar + ci * 16 + 4 * l.q);             // H_e, entering from the right
+  const float4 Gin = ld4(a.gcar + ci * 16 + 4 * l.q);            // G_{s-1}, entering from the left
+  float aprev[4] = {0.f, 0.f, 0.f, 0.f};                         // G_{-1} = 0 at s = 0
+  if (l.s > 0 && l.s < l.e) {
+    const float dprev = softplus_fwd(a.dt[((size_t)l.b * a.L + l.s - 1) * a.E + l.c] + a.dt_b[l.c]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) aprev[j] = exp2_mufu(dprev * l.A2[j]);
+  }
+  __syncthreads();
+
+  // H over the chunk
+  {
+    float H[4] = {Hr.x, Hr.y, Hr.z, Hr.w};
+    for (int i = l.e - 1; i >= l.s; --i) {
+      const int r = i - l.s;
+      const float delta = sg.arr[1][r * CPB + ch];
+      const float du = sg.arr[2][r * CPB + ch];
+      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) H[j] = fmaf(exp2_mufu(delta * l.A2[j]), H[j], du * get(Bq, j));
+      Hs[r * THREADS + threadIdx.x] = make_float4(H[0], H[1], H[2], H[3]);
+    }
+  }
+
+  // G from the left
+  float G[4] = {Gin.x, Gin.y, Gin.z, Gin.w};
+  float dA[4] = {0.f, 0.f, 0.f, 0.f};
+  float dDacc = 0.0f, dbacc = 0.0f;
+  const int T = a.T;
+  const int rows_end = min(l.s + T, a.L);                        // rows of this chunk in the padded batch
+  const int col = [&] {
+    // this lane's column of dB | dC after the reduce-scatter below: value
+    // index vi = 4·bit4 + 2·bit3 + bit2 of the lane → (vi < 4 ? 0 : 16) + 4q + (vi & 3)
+    const int vi = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+    return (vi < 4 ? 0 : 16) + 4 * l.q + (vi & 3);
+  }();
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  for (int i = l.s; i < rows_end; ++i) {
+    const size_t row = (size_t)l.b * a.L + i;
+    const int r = i - l.s;
+    float vred = 0.0f;
+    if (i < l.e) {
+      const float uu = sg.arr[0][r * CPB + ch];
+      const float delta = sg.arr[1][r * CPB + ch];
+      const float du_ = sg.arr[2][r * CPB + ch];
+      const float dp = sg.arr[3][r * CPB + ch];
+      const float fz = sg.arr[4][r * CPB + ch];
+      const float spg = sg.arr[5][r * CPB + ch];
+      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+      const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
+      const float4 Hi = Hs[r * THREADS + threadIdx.x];
+      const float4 Hn = (i + 1 < l.e) ? Hs[(r + 1) * THREADS + threadIdx.x] : Hr;
+      float ai[4], pc = 0.0f, sa = 0.0f, sb = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        G[j] = fmaf(aprev[j], G[j], dp * get(Cq, j));
+        ai[j] = exp2_mufu(delta * l.A2[j]);
+        pc = fmaf(get(Hi, j), get(Cq, j), pc);
+        const float gha = G[j] * get(Hn, j) * ai[j];
+        sa = fmaf(gha, l.A[j], sa);
+        sb = fmaf(G[j], get(Bq, j), sb);
+        dA[j] = fmaf(delta, gha, dA[j]);
+      }
+      pc = sum4(pc);
+      sa = sum4(sa);
+      sb = sum4(sb);
+      const float p = fmaf(Dc, uu, pc);
+      const float ddt = fmaf(sb, uu, sa) * spg;
+      dDacc = fmaf(dp, uu, dDacc);
+      dbacc += ddt;
+      if (l.q == 0) a.du[row * a.E + l.c] = fmaf(Dc, dp, delta * sb);
+      if (l.q == 1) a.ddt[row * a.E + l.c] = ddt;
+      if (l.q == 2) a.dz[row * a.ld_dz + l.c] = p * fz;
+      // dB (values 0-3) and dC (values 4-7) of states 4q … 4q+3, summed over
+      // the warp's 8 channels by a reduce-scatter on lane bits 4, 3, 2
+      float vv[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        vv[j] = G[j] * du_;
+        vv[4 + j] = dp * get(Hi, j);
+      }
+      float w[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float send = b4 ? vv[t] : vv[t + 4];
+        const float keep = b4 ? vv[t + 4] : vv[t];
+        w[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+      }
+      float x[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float send = b3 ? w[t] : w[t + 2];
+        const float keep = b3 ? w[t + 2] : w[t];
+        x[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+      {
+        const float send = b2 ? x[0] : x[1];
+        const float keep = b2 ? x[1] : x[0];
+        vred = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) aprev[j] = ai[j];
+    } else {
+      if (l.q == 0) a.du[row * a.E + l.c] = 0.0f;
+      if (l.q == 1) a.ddt[row * a.E + l.c] = 0.0f;
+      if (l.q == 2) a.dz[row * a.ld_dz + l.c] = 0.0f;
+    }
+    red[((size_t)warp * T + r) * 32 + col] = vred;
+  }
+  __syncthreads();
+  // fixed-order sum over the block's warps → per-block partial of dB | dC
+  const int nrows = rows_end - l.s;
+  for (int t = threadIdx.x; t < nrows * 32; t += THREADS) {
+    const int rr = t >> 5, cc = t & 31;
+    float acc = 0.0f;
+    for (int w = 0; w < WARPS; ++w) acc += red[((size_t)w * T + rr) * 32 + cc];
+    a.pbc[((size_t)blockIdx.x * a.B * a.L + (size_t)l.b * a.L + l.s + rr) * 32 + cc] = acc;
+  }
+  st4(a.pA + ci * 16 + 4 * l.q, make_float4(dA[0], dA[1], dA[2], dA[3]));
+  if (l.q == 0) {
+    a.pD[ci] = dDacc;
+    a.pb[ci] = dbacc;
+  }
+}
+
+// 6a. dA_log, dD, ddt_b: sums over the B·nc (sequence, chunk) partials in a
+// fixed order, in two levels: segment g of RSEG consecutive partials is
+// summed by block row g into seg[g], then the segments in order.
+constexpr int RSEG = 32;
+
+__global__ void reduce_params_seg_kernel(const Args a, float* seg) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // c·16 + m
+  if (t >= (long long)a.E * 16) return;
+  const int c = (int)(t >> 4), m = (int)(t & 15);
+  const long long cells = (long long)a.B * a.nc;
+  const long long p0 = (long long)blockIdx.y * RSEG;
+  float sA = 0.0f, sD = 0.0f, sb = 0.0f;
+#pragma unroll 8
+  for (int j = 0; j < RSEG; ++j) {
+    const long long p = p0 + j;                 // p = b·nc + k
+    if (p < cells) {
+      const size_t ci = (size_t)p * a.E + c;
+      sA += a.pA[ci * 16 + m];
+      if (m == 0) {
+        sD += a.pD[ci];
+        sb += a.pb[ci];
+      }
+    }
+  }
+  const size_t o = ((size_t)blockIdx.y * a.E * 16 + t) * 3;
+  seg[o] = sA;
+  seg[o + 1] = sD;
+  seg[o + 2] = sb;
+}
+
+__global__ void reduce_params_kernel(const Args a, const float* seg, int nseg) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // c·16 + m
+  if (t >= (long long)a.E * 16) return;
+  const int c = (int)(t >> 4), m = (int)(t & 15);
+  float sA = 0.0f, sD = 0.0f, sb = 0.0f;
+  for (int g = 0; g < nseg; ++g) {
+    const size_t o = ((size_t)g * a.E * 16 + t) * 3;
+    sA += seg[o];
+    sD += seg[o + 1];
+    sb += seg[o + 2];
+  }
+  a.dA_log[(size_t)c * 16 + m] = sA * -expf(a.A_log[(size_t)c * 16 + m]);
+  if (m == 0) {
+    a.dD[c] = sD;
+    a.ddt_b[c] = sb;
+  }
+}
+
+// 6b. dB | dC: sum of the per-block partials in block order.
+__global__ void reduce_bc_kernel(const Args a) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // row·32 + col
+  const long long M = (long long)a.B * a.L;
+  if (t >= M * 32) return;
+  const long long row = t >> 5;
+  const int col = (int)(t & 31);
+  const int nb = a.E / CPB;
+  float acc = 0.0f;
+  for (int cb = 0; cb < nb; ++cb) acc += a.pbc[((size_t)cb * M + row) * 32 + col];
+  a.dbc[row * a.ld_dbc + col] = acc;
+}
+
+}  // namespace sbwd
+
+int scan_bwd_chunk_tokens(int chunk_tokens) {
+  if (chunk_tokens <= 0) return 16;
+  return chunk_tokens > SCAN_BWD_MAX_CHUNK ? SCAN_BWD_MAX_CHUNK : chunk_tokens;
+}
+
+size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens) {
+  const int T = scan_bwd_chunk_tokens(chunk_tokens);
+  const size_t nc = (size_t)((L + T - 1) / T);
+  const size_t cells = (size_t)B * nc * E;
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  const size_t nseg = (cells / E + sbwd::RSEG - 1) / sbwd::RSEG;
+  return al(cells * 16 * 4) * 3 + al(cells * 4) * 4 + al((size_t)(E / sbwd::CPB) * B * L * 32 * 4) +
+         al(nseg * E * 16 * 3 * 4);
+}
+
+cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
+  using namespace sbwd;
+  Args a{};
+  a.u = g.u; a.z = g.z; a.ldz = g.ldz; a.dt = g.dt_raw; a.bc = g.bc; a.ldbc = g.ldbc;
+  a.A_log = g.A_log; a.D = g.D; a.dt_b = g.dt_b; a.dy = g.dy;
+  a.du = g.du; a.dz = g.dz; a.ld_dz = g.ld_dz; a.ddt = g.ddt_raw; a.dbc = g.dbc; a.ld_dbc = g.ld_dbc;
+  a.dA_log = g.dA_log; a.dD = g.dD; a.ddt_b = g.ddt_b;
+  a.B = g.B; a.L = g.L; a.E = g.E;
+  a.T = scan_bwd_chunk_tokens(g.chunk_tokens);
+  a.nc = (g.L + a.T - 1) / a.T;
+  a.lengths = g.lengths;
+  a.status = g.status;
+  const size_t cells = (size_t)g.B * a.nc * g.E;
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  char* p = (char*)scratch;
+  a.hcar = (float*)p; p += al(cells * 16 * 4);
+  a.gcar = (float*)p; p += al(cells * 16 * 4);
+  a.pA = (float*)p;   p += al(cells * 16 * 4);
+  a.hsd = (float*)p;  p += al(cells * 4);
+  a.gsd = (float*)p;  p += al(cells * 4);
+  a.pD = (float*)p;   p += al(cells * 4);
+  a.pb = (float*)p;   p += al(cells * 4);
+  a.pbc = (float*)p;  p += al((size_t)(g.E / CPB) * g.B * g.L * 32 * 4);
+  float* seg = (float*)p;
+  const int nseg = (int)(((size_t)g.B * a.nc + RSEG - 1) / RSEG);
+
+  const dim3 grid(g.E / CPB, a.nc, g.B);
+  const dim3 cgrid((unsigned)((g.E * 16 + 255) / 256), g.B);
+  const size_t ssmem = stage_floats(a.T) * sizeof(float);
+  const size_t fsmem = (size_t)a.T * THREADS * sizeof(float4) + (size_t)WARPS * a.T * 32 * sizeof(float) + ssmem;
+  cudaError_t e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(hstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
+      cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(gstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
+      cudaSuccess)
+    return e;
+  hstate_kernel<<<grid, THREADS, ssmem, st>>>(a);
+  carry_kernel<<<cgrid, 256, 0, st>>>(a, a.hcar, a.hsd, true);
+  gstate_kernel<<<grid, THREADS, ssmem, st>>>(a);
+  carry_kernel<<<cgrid, 256, 0, st>>>(a, a.gcar, a.gsd, false);
+  final_kernel<<<grid, THREADS, fsmem, st>>>(a);
+  reduce_params_seg_kernel<<<dim3((unsigned)((g.E * 16 + 255) / 256), nseg), 256, 0, st>>>(a, seg);
+  reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a, seg, nseg);
+  const long long M = (long long)g.B * g.L;
+  reduce_bc_kernel<<<(unsigned)((M * 32 + 255) / 256), 256, 0, st>>>(a);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace r2l

@@ -1,0 +1,25 @@
+// Host interface of the fp32 reverse-scan gradient (scan_bwd.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace r2l {
+
+constexpr int SCAN_BWD_MAX_CHUNK = 32;   // positions per chunk (shared memory: 5 KB each)
+
+struct ScanBwdArgs {
+  const float *u, *z, *dt_raw, *bc, *A_log, *D, *dt_b, *dy;
+  int ldz, ldbc;
+  float *du, *dz, *ddt_raw, *dbc, *dA_log, *dD, *ddt_b;
+  int ld_dz, ld_dbc;
+  int B, L, E, chunk_tokens;
+  const int* lengths;   // device [B] or null
+  unsigned* status;     // device status word (R2L_DEVFLAG_* bits)
+};
+
+int scan_bwd_chunk_tokens(int chunk_tokens);
+size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens);
+cudaError_t scan_bwd_f32(const ScanBwdArgs& a, void* scratch, cudaStream_t st);
+
+}  // namespace r2l

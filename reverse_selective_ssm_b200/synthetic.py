@@ -200,3 +200,33 @@ def to_f64(t):
 
 def weights_f64(w: Dict[str, Optional[torch.Tensor]]) -> Dict[str, object]:
     return {k: to_f64(v) for k, v in w.items()}
+
+
+def make_scan_bwd_case(B: int, L: int, E: int, seed: int, lengths: Optional[torch.Tensor] = None,
+                       dt_min: float = 1e-3, dt_max: float = 1e-1) -> Dict[str, torch.Tensor]:
+    """Inputs of the scan-gradient entry point, fp32 on the host: the scan's
+    own inputs with the distributions they have inside the layer (u, z ~
+    N(0, 1); B, C ~ N(0, 1); dt_raw ~ N(0, 0.1) around the per-channel bias
+    of a logUniform[dt_min, dt_max] step; A_log = log(1..16); D = 1) and an
+    upstream gradient dy ~ N(0, 1).  Rows at or past a sequence's length are
+    NaN in every per-position input (they must not be read)."""
+    g = torch.Generator().manual_seed(seed)
+    M = B * L
+    c = {
+        "u": torch.randn((M, E), generator=g),
+        "z": torch.randn((M, E), generator=g),
+        "dt_raw": torch.randn((M, E), generator=g) * 0.1,
+        "bc": torch.randn((M, 32), generator=g),
+        "dy": torch.randn((M, E), generator=g),
+    }
+    u01 = torch.rand((E,), generator=g, dtype=torch.float64)
+    dt0 = torch.exp(u01 * (math.log(dt_max) - math.log(dt_min)) + math.log(dt_min))
+    c["dt_b"] = (dt0 + torch.log(-torch.expm1(-dt0))).to(torch.float32)
+    c["A_log"] = torch.log(torch.arange(1, 17, dtype=torch.float32)).repeat(E, 1).contiguous()
+    c["D"] = torch.ones(E)
+    if lengths is not None:
+        for b, n in enumerate(lengths.tolist()):
+            if n < L:
+                for k in ("u", "z", "dt_raw", "bc", "dy"):
+                    c[k][b * L + n:(b + 1) * L] = float("nan")
+    return c

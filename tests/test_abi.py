@@ -129,3 +129,42 @@ def test_stack_and_debug_argument_checks(lib):
                                          n, None, None) == 1
     st = lib.r2l_get_device_status(None, None, None)
     assert st == 1
+
+
+def _bwd(lib, dims=None, B=2, L=40, ldz=128, ldbc=32, lengths=None, ws=FAKE, ws_bytes=None, chunk=0, bad=None):
+    dims = dims or bd.make_dims(64, 128, dtype=torch.float32)
+    if ws_bytes is None:
+        ws_bytes = bd.reverse_scan_backward_workspace_size(dims, B, L, chunk) or 1
+    p = [FAKE] * 19
+    if bad is not None:
+        p[bad[0]] = bad[1]
+    return lib.r2l_reverse_scan_backward(p[0], p[1], ldz, p[2], p[3], ldbc, p[4], p[5], p[6], p[7], p[8], p[9],
+                                         128, p[10], p[11], 32, p[12], p[13], p[14], ctypes.byref(dims), B, L,
+                                         lengths, chunk, ws, ws_bytes, None)
+
+
+def test_scan_backward_argument_checks(lib):
+    """r2l_reverse_scan_backward rejects bad arguments on the host (no GPU
+    needed): null pointers, unsupported dtype / direction / widths,
+    misalignment and a short workspace."""
+    f32 = bd.make_dims(64, 128, dtype=torch.float32)
+    n = bd.reverse_scan_backward_workspace_size(f32, 2, 40, 0)
+    assert n >= 3 * (2 * 3 * 128 * 16 * 4)              # three [B][chunks][E][16] fp32 arrays (T = 16: 3 chunks)
+    assert bd.reverse_scan_backward_workspace_size(f32, 2, 40, 8) > n   # shorter chunks, more carries
+    assert bd.reverse_scan_backward_workspace_size(bd.make_dims(64, 128), 2, 40, 0) == 0      # bf16
+    assert bd.reverse_scan_backward_workspace_size(bd.make_dims(64, 96, dtype=torch.float32), 2, 40, 0) == 0
+    assert _bwd(lib, bad=(0, None)) == 1
+    assert _bwd(lib, bad=(14, None)) == 1
+    assert _bwd(lib, B=0) == 1
+    assert _bwd(lib, chunk=-1) == 1
+    assert _bwd(lib, dims=bd.make_dims(64, 128)) == 2                                  # bf16: not yet
+    assert _bwd(lib, dims=bd.make_dims(64, 96, dtype=torch.float32), ldz=96) == 2      # E % 64
+    assert _bwd(lib, dims=bd.make_dims(64, 128, dtype=torch.float32, flags=bd.R2L_FLAG_FORWARD_SCAN)) == 2
+    assert _bwd(lib, ldz=64) == 1
+    assert _bwd(lib, ldbc=34) == 3
+    assert _bwd(lib, ldz=130) == 3
+    assert _bwd(lib, bad=(7, FAKE + 4)) == 3
+    assert _bwd(lib, lengths=FAKE + 2) == 3
+    assert _bwd(lib, ws=None) == 4
+    assert _bwd(lib, ws_bytes=16) == 4
+    assert _bwd(lib, ws=FAKE + 8) == 3
