@@ -51,6 +51,9 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays (no per-stage times)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--scan-backward", action="store_true",
+                    help="time the fp32 reverse-scan gradient (r2l_reverse_scan_backward) at B=8, L=4096, "
+                         "d_inner=4096 instead of the forward")
     return ap.parse_args(argv)
 
 
@@ -76,6 +79,7 @@ STAGE_SOURCES = {
     "out_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh"] + _COMMON,
     "ln_residual": ["simt_kernels.cuh"] + _COMMON,
+    "scan_bwd": ["scan_bwd.cu", "scan_bwd.h"] + _COMMON,
 }
 
 
@@ -535,6 +539,173 @@ def cpu_baseline(case, sample_seqs=(0, 1)):
                       f"numpy float64 oracle, {dt:.1f} s"}
 
 
+# ---------------------------------------------------------------- scan gradient
+
+BWD_METRIC = "R2L reverse-scan backward tokens/sec at B=8,L=4096,E=4096 (fp32)"
+BWD_LAUNCHES = 8          # kernels one r2l_reverse_scan_backward call launches
+
+
+def bwd_bytes_per_token(E):
+    """Bytes the gradient must move per position: u, z, dt_raw, dy read and du,
+    dz, ddt_raw written (fp32, E channels each), B | C read and dB | dC written
+    (32 fp32 each)."""
+    return E * 7 * 4 + 2 * 32 * 4
+
+
+def run_scan_backward(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from reverse_selective_ssm_b200 import binding as bd
+    from reverse_selective_ssm_b200 import synthetic as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bd.load()
+    B, L, E = args.batch or 8, args.seq or 4096, 4096
+    host = S.make_scan_bwd_case(B, L, E, seed=64 + rank)
+    d = {k: v.to(dev) for k, v in host.items()}
+    M = B * L
+    out = {k: torch.empty((M, E), device=dev) for k in ("du", "dz", "ddt_raw")}
+    out["dbc"] = torch.empty((M, 32), device=dev)
+    out["dA_log"] = torch.empty((E, 16), device=dev)
+    out["dD"] = torch.empty(E, device=dev)
+    out["ddt_b"] = torch.empty(E, device=dev)
+    dims = bd.make_dims(64, E, dtype=torch.float32)
+    ws = torch.empty(bd.reverse_scan_backward_workspace_size(dims, B, L, 0), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        bd.reverse_scan_backward(d["u"], d["z"], d["dt_raw"], d["bc"], d["A_log"], d["D"], d["dt_b"], d["dy"],
+                                 out["du"], out["dz"], out["ddt_raw"], out["dbc"], out["dA_log"], out["dD"],
+                                 out["ddt_b"], dims, B, L, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    st, fl = bd.get_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} flags {fl}")
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for _ in range(K):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        ins = {k: host[k].pin_memory() for k in ("u", "z", "dt_raw", "bc", "dy")}
+        outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+        h2d = sum(v.numel() * v.element_size() for v in ins.values())
+        d2h = sum(v.numel() * v.element_size() for v in outs.values())
+
+        def e2e_step():
+            for k, v in ins.items():
+                d[k].copy_(v, non_blocking=True)
+            call()
+            for k, v in outs.items():
+                v.copy_(out[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(1, min(K, 5))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": round(whole_job_rate(M, world, ke, ms_e), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
+               "api": "r2l_reverse_scan_backward via binding, pinned host inputs and gradients"}
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    per_call = ms / K
+    nbytes = bwd_bytes_per_token(E) * M
+    achieved = nbytes / (per_call * 1e-3) / 1e9
+    tag = f"scanbwd-B{B}-L{L}-E{E}"
+    line = {
+        "metric": BWD_METRIC, "value": round(whole_job_rate(M, world, K, ms), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(per_call, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded: u, z, dy ~ N(0,1); B, C ~ N(0,1); dt_raw ~ N(0,0.1) around a "
+                "logUniform[1e-3,1e-1] step; A=-(1..16); D=1)",
+        "config": {"workload": f"reverse-scan gradient fp32 B={B} L={L} E={E} N=16", "B": B, "L": L,
+                   "d_inner": E, "d_state": 16, "chunk_tokens": 16,
+                   "l2": "inputs larger than L2 (~4 GB read and written per step), no flush",
+                   "parallelism": f"dp{world}: one independent batch per GPU, no collective"},
+        "roofline": {"kernel": f"r2l_reverse_scan_backward (the {BWD_LAUNCHES} launches of one call)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": f"{peak_kind} HBM copy", "algorithmic_per_launch": nbytes,
+                     "bytes_per_token": bwd_bytes_per_token(E), "ms_per_launch": round(per_call, 4),
+                     "traffic": read_traffic("scan_bwd", tag)},
+        "gpu_launches": BWD_LAUNCHES * K, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_backward(host, B, L, E)
+    return line
+
+
+def cpu_baseline_backward(host, B, L, E, n=256):
+    """The float64 gradient oracle, as it stands, on a bounded sample: the
+    first n positions of sequence 0, all channels."""
+    import oracle as O
+    from reverse_selective_ssm_b200 import synthetic as S
+    f = lambda k: S.to_f64(host[k][:n])
+    bc = f("bc")
+    t = time.perf_counter()
+    O.reverse_scan_backward(f("u"), f("dt_raw"), S.to_f64(host["dt_b"]), S.to_f64(host["A_log"]), bc[:, :16],
+                            bc[:, 16:], S.to_f64(host["D"]), f("z"), f("dy"))
+    dt = time.perf_counter() - t
+    return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"positions 0..{n - 1} of sequence 0, all {E} channels, numpy float64 gradient oracle, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference_backward(args, rank, world):
+    """The gradient oracle timed on the host cores, each step a bounded sample
+    (the first 256 positions of one sequence, all channels)."""
+    if rank != 0:
+        return None
+    from reverse_selective_ssm_b200 import synthetic as S
+    B, L, E = args.batch or 8, args.seq or 4096, 4096
+    host = S.make_scan_bwd_case(B, L, E, seed=64)
+    for _ in range(args.warmup):
+        cpu_baseline_backward(host, B, L, E)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline_backward(host, B, L, E)
+    dt = time.perf_counter() - t
+    v = round(256 * args.steps / dt, 2)
+    cb = {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+          "sample": "per step positions 0..255 of sequence 0, all 4096 channels, numpy float64 gradient oracle"}
+    return {"metric": BWD_METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"reverse-scan gradient B={B} L={L} E={E} N=16"}, "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -586,7 +757,7 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = run_reference_backward(args, rank, world) if args.scan_backward else run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return 0
@@ -597,7 +768,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_scan_backward if args.scan_backward else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
