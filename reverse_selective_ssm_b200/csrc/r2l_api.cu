@@ -521,7 +521,7 @@ r2l_status r2l_reverse_scan_backward(const void* u, const void* z, int ldz, cons
   const int E = dims->d_inner;
   if (E % 64) return R2L_ERR_UNSUPPORTED;
   if (ldz < E || ld_dz < E || ldbc < 32 || ld_dbc < 32) return R2L_ERR_INVALID_ARG;
-  if ((ldbc % 4) || (ldz % 4)) return R2L_ERR_ALIGNMENT;
+  if ((ldbc % 4) || (ldz % 4) || (ld_dz % 4)) return R2L_ERR_ALIGNMENT;
   if (L > 65535 || B > 65535) return R2L_ERR_UNSUPPORTED;
   for (const void* q : {u, z, dt_raw, (const void*)bc, (const void*)A_log, (const void*)D, (const void*)dt_b, dy,
                         (const void*)du, (const void*)dz, (const void*)ddt_raw, (const void*)dbc,

@@ -116,6 +116,8 @@ struct Lane {
   int c, q, b, k, s, e, n;
   float A[4];    // A_m of the thread's states
   float A2[4];   // A_m · log2 e
+  float2 Ap[2];  // A as (states 0,1), (2,3) pairs for the packed f32x2 arithmetic
+  float2 A2p[2];
 };
 
 __device__ __forceinline__ Lane lane_setup(const Args& a) {
@@ -131,7 +133,24 @@ __device__ __forceinline__ Lane lane_setup(const Args& a) {
   l.A[0] = -expf(al.x); l.A[1] = -expf(al.y); l.A[2] = -expf(al.z); l.A[3] = -expf(al.w);
 #pragma unroll
   for (int j = 0; j < 4; ++j) l.A2[j] = l.A[j] * kLog2e;
+  l.Ap[0] = make_float2(l.A[0], l.A[1]);
+  l.Ap[1] = make_float2(l.A[2], l.A[3]);
+  l.A2p[0] = make_float2(l.A2[0], l.A2[1]);
+  l.A2p[1] = make_float2(l.A2[2], l.A2[3]);
   return l;
+}
+
+__device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+
+// The decays of the thread's 4 states for step Δ: exp(Δ A) = 2^(Δ A log2 e).
+__device__ __forceinline__ void decays(const Lane& l, float delta, float2 (&a)[2]) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float2 t = __fmul2_rn(dup2(delta), l.A2p[k]);
+    a[k] = make_float2(exp2_mufu(t.x), exp2_mufu(t.y));
+  }
 }
 
 __device__ __forceinline__ size_t carry_idx(const Args& a, const Lane& l) {
@@ -217,18 +236,25 @@ __global__ void __launch_bounds__(THREADS) hstate_kernel(const Args a) {
   __syncthreads();
   const size_t ci = carry_idx(a, l);
   const int ch = threadIdx.x >> 2;
-  float H[4] = {0.f, 0.f, 0.f, 0.f};
+  float2 H[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float sd = 0.0f;
-  for (int i = l.e - 1; i >= l.s; --i) {
-    const int r = i - l.s;
+  auto step = [&](int r) {
     const float delta = sg.arr[1][r * CPB + ch];
-    const float du = sg.arr[2][r * CPB + ch];
+    const float2 du = dup2(sg.arr[2][r * CPB + ch]);
     const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
     sd += delta;
+    float2 ad[2];
+    decays(l, delta, ad);
+    H[0] = __ffma2_rn(ad[0], H[0], __fmul2_rn(du, lo2(Bq)));
+    H[1] = __ffma2_rn(ad[1], H[1], __fmul2_rn(du, hi2(Bq)));
+  };
+  if (a.T == 16 && l.e - l.s == 16) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) H[j] = fmaf(exp2_mufu(delta * l.A2[j]), H[j], du * get(Bq, j));
+    for (int rr = 0; rr < 16; ++rr) step(15 - rr);
+  } else {
+    for (int r = l.e - l.s - 1; r >= 0; --r) step(r);
   }
-  st4(a.hcar + ci * 16 + 4 * l.q, make_float4(H[0], H[1], H[2], H[3]));
+  st4(a.hcar + ci * 16 + 4 * l.q, make_float4(H[0].x, H[0].y, H[1].x, H[1].y));
   if (l.q == 0) a.hsd[ci] = sd;
 }
 
@@ -273,30 +299,156 @@ __global__ void __launch_bounds__(THREADS) gstate_kernel(const Args a) {
   stage_chunk<S_DL | S_DP>(a, l, sg);
   const size_t ci = carry_idx(a, l);
   const int ch = threadIdx.x >> 2;
-  float G[4] = {0.f, 0.f, 0.f, 0.f};
+  float2 G[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float sd = 0.0f, prev = 0.0f;
   if (l.s > 0 && l.s < l.e) prev = softplus_fwd(a.dt[((size_t)l.b * a.L + l.s - 1) * a.E + l.c] + a.dt_b[l.c]);
   __syncthreads();
-  for (int i = l.s; i < l.e; ++i) {
-    const int r = i - l.s;
+  // decays crossed: positions s-1 … e-2 (G_{s-1} multiplies a_{s-1})
+  auto step = [&](int r) {
     const float delta = sg.arr[1][r * CPB + ch];
     const float dp = sg.arr[3][r * CPB + ch];
     const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
-    if (i > l.s) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) G[j] *= exp2_mufu(prev * l.A2[j]);
+    if (r > 0) {
+      float2 ad[2];
+      decays(l, prev, ad);
+      G[0] = __fmul2_rn(G[0], ad[0]);
+      G[1] = __fmul2_rn(G[1], ad[1]);
     }
-    if (i > l.s || l.s > 0) sd += prev;                  // decays crossed: positions s-1 … e-2
-#pragma unroll
-    for (int j = 0; j < 4; ++j) G[j] = fmaf(dp, get(Cq, j), G[j]);
+    if (r > 0 || l.s > 0) sd += prev;
+    G[0] = __ffma2_rn(dup2(dp), lo2(Cq), G[0]);
+    G[1] = __ffma2_rn(dup2(dp), hi2(Cq), G[1]);
     prev = delta;
+  };
+  if (a.T == 16 && l.e - l.s == 16) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) step(r);
+  } else {
+    for (int r = 0; r < l.e - l.s; ++r) step(r);
   }
-  st4(a.gcar + ci * 16 + 4 * l.q, make_float4(G[0], G[1], G[2], G[3]));
+  st4(a.gcar + ci * 16 + 4 * l.q, make_float4(G[0].x, G[0].y, G[1].x, G[1].y));
   if (l.q == 0) a.gsd[ci] = sd;
 }
 
 // 5. Per chunk: H from H_in(k) into shared memory (right to left), then G
-// from the carried value (left to right) with every gradient.
+// from the carried value (left to right) with every gradient.  TF = 16: a
+// chunk of 16 valid positions, unrolled with static shared-memory offsets;
+// TF = 0: any chunk (ragged ends, other chunk lengths).
+template <int TF>
+__device__ __forceinline__ void final_body(const Args& a, const Lane& l, const Stage& sg, float4* Hs, float* red,
+                                           float4 Hr, float4 Gin, float (&aprev)[4], float (&dA)[4],
+                                           float& dDacc, float& dbacc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ch = threadIdx.x >> 2;
+  const int T = TF ? TF : a.T;
+  const int nvalid = TF ? TF : l.e - l.s;                   // positions s … e-1
+  const int nrows = TF ? TF : min(l.s + a.T, a.L) - l.s;    // rows of this chunk in the padded batch
+  const float Dc = a.D[l.c];
+
+  // H over the chunk, right to left
+  {
+    float2 H[2] = {lo2(Hr), hi2(Hr)};
+    auto hstep = [&](int r) {
+      const float delta = sg.arr[1][r * CPB + ch];
+      const float2 du = dup2(sg.arr[2][r * CPB + ch]);
+      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+      float2 ad[2];
+      decays(l, delta, ad);
+      H[0] = __ffma2_rn(ad[0], H[0], __fmul2_rn(du, lo2(Bq)));
+      H[1] = __ffma2_rn(ad[1], H[1], __fmul2_rn(du, hi2(Bq)));
+      Hs[r * THREADS + threadIdx.x] = make_float4(H[0].x, H[0].y, H[1].x, H[1].y);
+    };
+    if constexpr (TF > 0) {
+#pragma unroll
+      for (int rr = 0; rr < TF; ++rr) hstep(TF - 1 - rr);
+    } else {
+      for (int r = nvalid - 1; r >= 0; --r) hstep(r);
+    }
+  }
+
+  float2 G[2] = {lo2(Gin), hi2(Gin)};
+  float2 ap[2] = {make_float2(aprev[0], aprev[1]), make_float2(aprev[2], aprev[3])};
+  float2 dAp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  // this lane's column of dB | dC after the reduce-scatter: value index
+  // vi = 4·bit4 + 2·bit3 + bit2 of the lane → (vi < 4 ? 0 : 16) + 4q + (vi & 3)
+  const int vi = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+  const int col = (vi < 4 ? 0 : 16) + 4 * l.q + (vi & 3);
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float* redw = red + (size_t)warp * T * 32 + col;
+  // thread q of a channel leaves one per-position gradient in shared memory,
+  // over the staged input it no longer needs: du over Δu (q = 0), ddt_raw
+  // over softplus' (q = 1), dz over the dz factor (q = 2)
+  float* outq = l.q == 0 ? sg.arr[2] : l.q == 1 ? sg.arr[5] : sg.arr[4];
+  auto gstep = [&](int r) {
+    const float uu = sg.arr[0][r * CPB + ch];
+    const float delta = sg.arr[1][r * CPB + ch];
+    const float du_ = sg.arr[2][r * CPB + ch];
+    const float dp = sg.arr[3][r * CPB + ch];
+    const float fz = sg.arr[4][r * CPB + ch];
+    const float spg = sg.arr[5][r * CPB + ch];
+    const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+    const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
+    const float4 Hi = Hs[r * THREADS + threadIdx.x];
+    const float4 Hn = (r + 1 < nvalid) ? Hs[(r + 1) * THREADS + threadIdx.x] : Hr;
+    const float2 dp2 = dup2(dp);
+    G[0] = __ffma2_rn(ap[0], G[0], __fmul2_rn(dp2, lo2(Cq)));
+    G[1] = __ffma2_rn(ap[1], G[1], __fmul2_rn(dp2, hi2(Cq)));
+    float2 ai[2];
+    decays(l, delta, ai);
+    const float2 pc2 = __ffma2_rn(hi2(Hi), hi2(Cq), __fmul2_rn(lo2(Hi), lo2(Cq)));
+    const float2 gh0 = __fmul2_rn(__fmul2_rn(G[0], lo2(Hn)), ai[0]);
+    const float2 gh1 = __fmul2_rn(__fmul2_rn(G[1], hi2(Hn)), ai[1]);
+    const float2 sa2 = __ffma2_rn(gh1, l.Ap[1], __fmul2_rn(gh0, l.Ap[0]));
+    const float2 sb2 = __ffma2_rn(G[1], hi2(Bq), __fmul2_rn(G[0], lo2(Bq)));
+    const float2 d2 = dup2(delta);
+    dAp[0] = __ffma2_rn(d2, gh0, dAp[0]);
+    dAp[1] = __ffma2_rn(d2, gh1, dAp[1]);
+    const float pc = sum4(pc2.x + pc2.y);
+    const float sa = sum4(sa2.x + sa2.y);
+    const float sb = sum4(sb2.x + sb2.y);
+    const float p = fmaf(Dc, uu, pc);
+    const float ddt = fmaf(sb, uu, sa) * spg;
+    dDacc = fmaf(dp, uu, dDacc);
+    dbacc += ddt;
+    // dB (values 0-3) and dC (values 4-7) of states 4q … 4q+3, summed over
+    // the warp's 8 channels by a reduce-scatter on lane bits 4, 3, 2
+    const float2 gb0 = __fmul2_rn(G[0], dup2(du_)), gb1 = __fmul2_rn(G[1], dup2(du_));
+    const float2 hc0 = __fmul2_rn(dp2, lo2(Hi)), hc1 = __fmul2_rn(dp2, hi2(Hi));
+    const float vv[8] = {gb0.x, gb0.y, gb1.x, gb1.y, hc0.x, hc0.y, hc1.x, hc1.y};
+    float w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float send = b4 ? vv[t] : vv[t + 4];
+      const float keep = b4 ? vv[t + 4] : vv[t];
+      w[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float x[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const float send = b3 ? w[t] : w[t + 2];
+      const float keep = b3 ? w[t + 2] : w[t];
+      x[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float send = b2 ? x[0] : x[1];
+    const float keep = b2 ? x[1] : x[0];
+    redw[r * 32] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    const float outv = l.q == 0 ? fmaf(Dc, dp, delta * sb) : l.q == 1 ? ddt : p * fz;
+    if (l.q < 3) outq[r * CPB + ch] = outv;
+    ap[0] = ai[0];
+    ap[1] = ai[1];
+  };
+  if constexpr (TF > 0) {
+#pragma unroll
+    for (int r = 0; r < TF; ++r) gstep(r);
+  } else {
+    for (int r = 0; r < nvalid; ++r) gstep(r);
+    for (int r = nvalid > 0 ? nvalid : 0; r < nrows; ++r) {   // padding rows of the chunk
+      if (l.q < 3) outq[r * CPB + ch] = 0.0f;
+      redw[r * 32] = 0.0f;
+    }
+  }
+  dA[0] = dAp[0].x; dA[1] = dAp[0].y; dA[2] = dAp[1].x; dA[3] = dAp[1].y;
+}
+
 __global__ void __launch_bounds__(THREADS) final_kernel(const Args a) {
   extern __shared__ float4 sm4[];
   float4* Hs = sm4;                                              // [T][THREADS]
@@ -305,9 +457,6 @@ __global__ void __launch_bounds__(THREADS) final_kernel(const Args a) {
   const Stage sg = stage_layout(red + (size_t)WARPS * a.T * 32, a.T);
   stage_chunk<S_U | S_DL | S_DU | S_DP | S_FZ | S_SG>(a, l, sg);
   const size_t ci = carry_idx(a, l);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int ch = threadIdx.x >> 2;
-  const float Dc = a.D[l.c];
   const float4 Hr = ld4(a.hcar + ci * 16 + 4 * l.q);             // H_e, entering from the right
   const float4 Gin = ld4(a.gcar + ci * 16 + 4 * l.q);            // G_{s-1}, entering from the left
   float aprev[4] = {0.f, 0.f, 0.f, 0.f};                         // G_{-1} = 0 at s = 0
@@ -317,112 +466,33 @@ __global__ void __launch_bounds__(THREADS) final_kernel(const Args a) {
     for (int j = 0; j < 4; ++j) aprev[j] = exp2_mufu(dprev * l.A2[j]);
   }
   __syncthreads();
-
-  // H over the chunk
-  {
-    float H[4] = {Hr.x, Hr.y, Hr.z, Hr.w};
-    for (int i = l.e - 1; i >= l.s; --i) {
-      const int r = i - l.s;
-      const float delta = sg.arr[1][r * CPB + ch];
-      const float du = sg.arr[2][r * CPB + ch];
-      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) H[j] = fmaf(exp2_mufu(delta * l.A2[j]), H[j], du * get(Bq, j));
-      Hs[r * THREADS + threadIdx.x] = make_float4(H[0], H[1], H[2], H[3]);
-    }
-  }
-
-  // G from the left
-  float G[4] = {Gin.x, Gin.y, Gin.z, Gin.w};
   float dA[4] = {0.f, 0.f, 0.f, 0.f};
   float dDacc = 0.0f, dbacc = 0.0f;
-  const int T = a.T;
-  const int rows_end = min(l.s + T, a.L);                        // rows of this chunk in the padded batch
-  const int col = [&] {
-    // this lane's column of dB | dC after the reduce-scatter below: value
-    // index vi = 4·bit4 + 2·bit3 + bit2 of the lane → (vi < 4 ? 0 : 16) + 4q + (vi & 3)
-    const int vi = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-    return (vi < 4 ? 0 : 16) + 4 * l.q + (vi & 3);
-  }();
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  for (int i = l.s; i < rows_end; ++i) {
-    const size_t row = (size_t)l.b * a.L + i;
-    const int r = i - l.s;
-    float vred = 0.0f;
-    if (i < l.e) {
-      const float uu = sg.arr[0][r * CPB + ch];
-      const float delta = sg.arr[1][r * CPB + ch];
-      const float du_ = sg.arr[2][r * CPB + ch];
-      const float dp = sg.arr[3][r * CPB + ch];
-      const float fz = sg.arr[4][r * CPB + ch];
-      const float spg = sg.arr[5][r * CPB + ch];
-      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
-      const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
-      const float4 Hi = Hs[r * THREADS + threadIdx.x];
-      const float4 Hn = (i + 1 < l.e) ? Hs[(r + 1) * THREADS + threadIdx.x] : Hr;
-      float ai[4], pc = 0.0f, sa = 0.0f, sb = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        G[j] = fmaf(aprev[j], G[j], dp * get(Cq, j));
-        ai[j] = exp2_mufu(delta * l.A2[j]);
-        pc = fmaf(get(Hi, j), get(Cq, j), pc);
-        const float gha = G[j] * get(Hn, j) * ai[j];
-        sa = fmaf(gha, l.A[j], sa);
-        sb = fmaf(G[j], get(Bq, j), sb);
-        dA[j] = fmaf(delta, gha, dA[j]);
-      }
-      pc = sum4(pc);
-      sa = sum4(sa);
-      sb = sum4(sb);
-      const float p = fmaf(Dc, uu, pc);
-      const float ddt = fmaf(sb, uu, sa) * spg;
-      dDacc = fmaf(dp, uu, dDacc);
-      dbacc += ddt;
-      if (l.q == 0) a.du[row * a.E + l.c] = fmaf(Dc, dp, delta * sb);
-      if (l.q == 1) a.ddt[row * a.E + l.c] = ddt;
-      if (l.q == 2) a.dz[row * a.ld_dz + l.c] = p * fz;
-      // dB (values 0-3) and dC (values 4-7) of states 4q … 4q+3, summed over
-      // the warp's 8 channels by a reduce-scatter on lane bits 4, 3, 2
-      float vv[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        vv[j] = G[j] * du_;
-        vv[4 + j] = dp * get(Hi, j);
-      }
-      float w[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float send = b4 ? vv[t] : vv[t + 4];
-        const float keep = b4 ? vv[t + 4] : vv[t];
-        w[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-      }
-      float x[2];
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float send = b3 ? w[t] : w[t + 2];
-        const float keep = b3 ? w[t + 2] : w[t];
-        x[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-      }
-      {
-        const float send = b2 ? x[0] : x[1];
-        const float keep = b2 ? x[1] : x[0];
-        vred = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) aprev[j] = ai[j];
-    } else {
-      if (l.q == 0) a.du[row * a.E + l.c] = 0.0f;
-      if (l.q == 1) a.ddt[row * a.E + l.c] = 0.0f;
-      if (l.q == 2) a.dz[row * a.ld_dz + l.c] = 0.0f;
-    }
-    red[((size_t)warp * T + r) * 32 + col] = vred;
-  }
+  if (a.T == 16 && l.e - l.s == 16)
+    final_body<16>(a, l, sg, Hs, red, Hr, Gin, aprev, dA, dDacc, dbacc);
+  else
+    final_body<0>(a, l, sg, Hs, red, Hr, Gin, aprev, dA, dDacc, dbacc);
   __syncthreads();
+  // the per-position gradients, [rows × 64 channels] each, as float4 rows
+  const int T = a.T;
+  const int nrows = min(l.s + T, a.L) - l.s;
+  {
+    const size_t row0 = (size_t)l.b * a.L + l.s;
+    const int col0 = blockIdx.x * CPB;
+    for (int t = threadIdx.x; t < nrows * (CPB / 4); t += THREADS) {
+      const int r = t / (CPB / 4), q4 = t % (CPB / 4);
+      const int off = r * CPB + 4 * q4;
+      const size_t row = row0 + r;
+      st4(a.du + row * a.E + col0 + 4 * q4, ld4(sg.arr[2] + off));
+      st4(a.ddt + row * a.E + col0 + 4 * q4, ld4(sg.arr[5] + off));
+      st4(a.dz + row * a.ld_dz + col0 + 4 * q4, ld4(sg.arr[4] + off));
+    }
+  }
   // fixed-order sum over the block's warps → per-block partial of dB | dC
-  const int nrows = rows_end - l.s;
   for (int t = threadIdx.x; t < nrows * 32; t += THREADS) {
     const int rr = t >> 5, cc = t & 31;
     float acc = 0.0f;
+#pragma unroll
     for (int w = 0; w < WARPS; ++w) acc += red[((size_t)w * T + rr) * 32 + cc];
     a.pbc[((size_t)blockIdx.x * a.B * a.L + (size_t)l.b * a.L + l.s + rr) * 32 + cc] = acc;
   }
