@@ -401,29 +401,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        h_host = case.h.pin_memory()
-        out_host = torch.empty_like(h_host).pin_memory()
-        for _ in range(max(1, args.warmup // 2)):
-            h.copy_(h_host, non_blocking=True)
-            step()
-            out_host.copy_(h, non_blocking=True)
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K):
-            h.copy_(h_host, non_blocking=True)
-            step()
-            out_host.copy_(h, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        nbytes = h_host.numel() * h_host.element_size()
-        e2e = {"value": round(whole_job_rate(case.valid_tokens, world, K, ms_e2e), 1), "unit": "tokens/s",
-               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
-               "api": "r2l_sidecar_forward via binding, pinned host hidden in/out"}
+        e2e = run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
 
     if rank != 0:
         return None
@@ -537,6 +515,95 @@ def cpu_baseline(case, sample_seqs=(0, 1)):
             "cores": _blas_threads(), "kind": "oracle",
             "sample": f"sequences {list(sample_seqs)} of the workload in full ({tokens} tokens), "
                       f"numpy float64 oracle, {dt:.1f} s"}
+
+
+def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev):
+    """Tokens/s through r2l_sidecar_forward with the hidden states coming from
+    and going back to pinned host memory every step.
+
+    value: a pipelined serving loop. Step k's host-to-device copy runs on one
+    stream, its forward on another and its device-to-host copy on a third, over
+    two device buffers. So the inbound copy of step k+1 and the outbound copy
+    of step k-1 overlap the forward of step k. The forward calls stay ordered
+    on one stream, so they share one workspace.
+    serial_value: copy in, forward, copy out, one after the other on one stream."""
+    import torch
+    from reverse_selective_ssm_b200 import binding as bd
+    K = args.steps
+    hooks = len(wdev)
+    h_host = case.h.pin_memory()
+    out_host = torch.empty_like(h_host).pin_memory()
+    nbytes = h_host.numel() * h_host.element_size()
+
+    def forward(buf, st):
+        for k in range(hooks):
+            bd.sidecar_forward(buf, wdev[k], dims, case.s[k], lengths, ws, st)
+
+    # serial
+    for _ in range(max(1, args.warmup // 2)):
+        h.copy_(h_host, non_blocking=True)
+        forward(h, stream)
+        out_host.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        h.copy_(h_host, non_blocking=True)
+        forward(h, stream)
+        out_host.copy_(h, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_serial = max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    # pipelined
+    bufs = [h, torch.empty_like(h)]
+    s_in, s_fw, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_fw = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def pipelined(n, t_start=None, t_end=None):
+        if t_start is not None:
+            t_start.record(s_in)
+            s_fw.wait_event(t_start)
+            s_out.wait_event(t_start)
+        for k in range(n):
+            i = k & 1
+            if k >= 2:
+                s_in.wait_event(ev_out[i])          # buffer i is free once step k-2 is copied out
+            with torch.cuda.stream(s_in):
+                bufs[i].copy_(h_host, non_blocking=True)
+            ev_in[i].record(s_in)
+            s_fw.wait_event(ev_in[i])
+            forward(bufs[i], s_fw)
+            ev_fw[i].record(s_fw)
+            s_out.wait_event(ev_fw[i])
+            with torch.cuda.stream(s_out):
+                out_host.copy_(bufs[i], non_blocking=True)
+            ev_out[i].record(s_out)
+        if t_end is not None:
+            s_out.wait_stream(s_in)
+            s_out.wait_stream(s_fw)
+            t_end.record(s_out)
+
+    pipelined(max(2, args.warmup))
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipelined(K, p0, p1)
+    torch.cuda.synchronize()
+    barrier()
+    ms_pipe = max_over_ranks(p0.elapsed_time(p1), world, dev)
+    return {"value": round(whole_job_rate(case.valid_tokens, world, K, ms_pipe), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+            "serial_value": round(whole_job_rate(case.valid_tokens, world, K, ms_serial), 1),
+            "api": "r2l_sidecar_forward via binding, pinned host hidden in/out",
+            "schedule": "pipelined: copy-in, forward and copy-out of successive steps on three streams over "
+                        "two device buffers (serial_value: one stream, no overlap)"}
 
 
 # ---------------------------------------------------------------- scan gradient
