@@ -172,15 +172,20 @@ struct Stage {
   float* bc;
 };
 
+// Arrays sit 8 words apart in bank order (stride T·64 + 8 floats), so the
+// three gradient rows that a channel's threads q = 0, 1, 2 leave in arrays
+// 2, 5 and 4 fall in different banks.
+constexpr int STAGE_PAD = 8;
+
 __device__ __forceinline__ Stage stage_layout(float* base, int T) {
   Stage st;
 #pragma unroll
-  for (int k = 0; k < NSTAGE; ++k) st.arr[k] = base + (size_t)k * T * CPB;
-  st.bc = base + (size_t)NSTAGE * T * CPB;
+  for (int k = 0; k < NSTAGE; ++k) st.arr[k] = base + (size_t)k * (T * CPB + STAGE_PAD);
+  st.bc = base + (size_t)NSTAGE * (T * CPB + STAGE_PAD);
   return st;
 }
 
-constexpr size_t stage_floats(int T) { return (size_t)T * (NSTAGE * CPB + 32); }
+constexpr size_t stage_floats(int T) { return (size_t)NSTAGE * (T * CPB + STAGE_PAD) + (size_t)T * 32; }
 
 template <unsigned WANT>
 __device__ __forceinline__ void stage_chunk(const Args& a, const Lane& l, const Stage& st) {
@@ -329,12 +334,15 @@ __global__ void __launch_bounds__(THREADS) gstate_kernel(const Args a) {
   if (l.q == 0) a.gsd[ci] = sd;
 }
 
-// 5. Per chunk: H from H_in(k) into shared memory (right to left), then G
-// from the carried value (left to right) with every gradient.  TF = 16: a
-// chunk of 16 valid positions, unrolled with static shared-memory offsets;
-// TF = 0: any chunk (ragged ends, other chunk lengths).
+// 5. Per chunk: H from H_in(k), right to left, keeping it at every second
+// position (shared memory); then G from the carried value, left to right,
+// two positions at a time: their H is recomputed in registers from the
+// checkpoint on their right (with the decays the G steps reuse), and every
+// gradient is formed.  TF = 16: a chunk of 16 valid positions, unrolled with
+// static shared-memory offsets; TF = 0: any chunk (ragged ends, other chunk
+// lengths).
 template <int TF>
-__device__ __forceinline__ void final_body(const Args& a, const Lane& l, const Stage& sg, float4* Hs, float* red,
+__device__ __forceinline__ void final_body(const Args& a, const Lane& l, const Stage& sg, float4* Hck, float* red,
                                            float4 Hr, float4 Gin, float (&aprev)[4], float (&dA)[4],
                                            float& dDacc, float& dbacc) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -344,24 +352,29 @@ __device__ __forceinline__ void final_body(const Args& a, const Lane& l, const S
   const int nrows = TF ? TF : min(l.s + a.T, a.L) - l.s;    // rows of this chunk in the padded batch
   const float Dc = a.D[l.c];
 
-  // H over the chunk, right to left
+  auto hcalc = [&](int r, const float4& Hright, float4& Hout, float2 (&ad)[2]) {
+    const float delta = sg.arr[1][r * CPB + ch];
+    const float2 du = dup2(sg.arr[2][r * CPB + ch]);
+    const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+    decays(l, delta, ad);
+    const float2 h0 = __ffma2_rn(ad[0], lo2(Hright), __fmul2_rn(du, lo2(Bq)));
+    const float2 h1 = __ffma2_rn(ad[1], hi2(Hright), __fmul2_rn(du, hi2(Bq)));
+    Hout = make_float4(h0.x, h0.y, h1.x, h1.y);
+  };
+
+  // H over the chunk, right to left, kept at the even positions 2, 4, …
   {
-    float2 H[2] = {lo2(Hr), hi2(Hr)};
+    float4 H = Hr;
     auto hstep = [&](int r) {
-      const float delta = sg.arr[1][r * CPB + ch];
-      const float2 du = dup2(sg.arr[2][r * CPB + ch]);
-      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
       float2 ad[2];
-      decays(l, delta, ad);
-      H[0] = __ffma2_rn(ad[0], H[0], __fmul2_rn(du, lo2(Bq)));
-      H[1] = __ffma2_rn(ad[1], H[1], __fmul2_rn(du, hi2(Bq)));
-      Hs[r * THREADS + threadIdx.x] = make_float4(H[0].x, H[0].y, H[1].x, H[1].y);
+      hcalc(r, H, H, ad);
+      if ((r & 1) == 0) Hck[(r >> 1) * THREADS + threadIdx.x] = H;
     };
     if constexpr (TF > 0) {
 #pragma unroll
-      for (int rr = 0; rr < TF; ++rr) hstep(TF - 1 - rr);
+      for (int rr = 0; rr < TF - 2; ++rr) hstep(TF - 1 - rr);
     } else {
-      for (int r = nvalid - 1; r >= 0; --r) hstep(r);
+      for (int r = nvalid - 1; r >= 2; --r) hstep(r);
     }
   }
 
@@ -378,7 +391,7 @@ __device__ __forceinline__ void final_body(const Args& a, const Lane& l, const S
   // over the staged input it no longer needs: du over Δu (q = 0), ddt_raw
   // over softplus' (q = 1), dz over the dz factor (q = 2)
   float* outq = l.q == 0 ? sg.arr[2] : l.q == 1 ? sg.arr[5] : sg.arr[4];
-  auto gstep = [&](int r) {
+  auto gstep = [&](int r, const float4& Hi, const float4& Hn, const float2 (&ai)[2]) {
     const float uu = sg.arr[0][r * CPB + ch];
     const float delta = sg.arr[1][r * CPB + ch];
     const float du_ = sg.arr[2][r * CPB + ch];
@@ -387,13 +400,9 @@ __device__ __forceinline__ void final_body(const Args& a, const Lane& l, const S
     const float spg = sg.arr[5][r * CPB + ch];
     const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
     const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
-    const float4 Hi = Hs[r * THREADS + threadIdx.x];
-    const float4 Hn = (r + 1 < nvalid) ? Hs[(r + 1) * THREADS + threadIdx.x] : Hr;
     const float2 dp2 = dup2(dp);
     G[0] = __ffma2_rn(ap[0], G[0], __fmul2_rn(dp2, lo2(Cq)));
     G[1] = __ffma2_rn(ap[1], G[1], __fmul2_rn(dp2, hi2(Cq)));
-    float2 ai[2];
-    decays(l, delta, ai);
     const float2 pc2 = __ffma2_rn(hi2(Hi), hi2(Cq), __fmul2_rn(lo2(Hi), lo2(Cq)));
     const float2 gh0 = __fmul2_rn(__fmul2_rn(G[0], lo2(Hn)), ai[0]);
     const float2 gh1 = __fmul2_rn(__fmul2_rn(G[1], hi2(Hn)), ai[1]);
@@ -436,11 +445,23 @@ __device__ __forceinline__ void final_body(const Args& a, const Lane& l, const S
     ap[0] = ai[0];
     ap[1] = ai[1];
   };
+  // positions r0 and r0 + 1 (the latter if valid): H_{r0+2} from the
+  // checkpoint (H entering the chunk from the right past its end)
+  auto pair = [&](int r0) {
+    const bool two = r0 + 1 < nvalid;
+    const float4 Hright = (r0 + 2 < nvalid) ? Hck[((r0 + 2) >> 1) * THREADS + threadIdx.x] : Hr;
+    float4 H1 = Hright, H0;
+    float2 a1[2], a0[2];
+    if (two) hcalc(r0 + 1, Hright, H1, a1);
+    hcalc(r0, H1, H0, a0);
+    gstep(r0, H0, H1, a0);
+    if (two) gstep(r0 + 1, H1, Hright, a1);
+  };
   if constexpr (TF > 0) {
 #pragma unroll
-    for (int r = 0; r < TF; ++r) gstep(r);
+    for (int r0 = 0; r0 < TF; r0 += 2) pair(r0);
   } else {
-    for (int r = 0; r < nvalid; ++r) gstep(r);
+    for (int r0 = 0; r0 < nvalid; r0 += 2) pair(r0);
     for (int r = nvalid > 0 ? nvalid : 0; r < nrows; ++r) {   // padding rows of the chunk
       if (l.q < 3) outq[r * CPB + ch] = 0.0f;
       redw[r * 32] = 0.0f;
@@ -449,10 +470,10 @@ __device__ __forceinline__ void final_body(const Args& a, const Lane& l, const S
   dA[0] = dAp[0].x; dA[1] = dAp[0].y; dA[2] = dAp[1].x; dA[3] = dAp[1].y;
 }
 
-__global__ void __launch_bounds__(THREADS) final_kernel(const Args a) {
+__global__ void __launch_bounds__(THREADS, 3) final_kernel(const Args a) {
   extern __shared__ float4 sm4[];
-  float4* Hs = sm4;                                              // [T][THREADS]
-  float* red = reinterpret_cast<float*>(sm4 + (size_t)a.T * THREADS);   // [WARPS][T][32]
+  float4* Hs = sm4;                            // [(T+1)/2][THREADS]: H at positions 2, 4, … (index r/2)
+  float* red = reinterpret_cast<float*>(sm4 + (size_t)((a.T + 1) / 2) * THREADS);   // [WARPS][T][32]
   const Lane l = lane_setup(a);
   const Stage sg = stage_layout(red + (size_t)WARPS * a.T * 32, a.T);
   stage_chunk<S_U | S_DL | S_DU | S_DP | S_FZ | S_SG>(a, l, sg);
@@ -610,7 +631,8 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   const dim3 grid(g.E / CPB, a.nc, g.B);
   const dim3 cgrid((unsigned)((g.E * 16 + 255) / 256), g.B);
   const size_t ssmem = stage_floats(a.T) * sizeof(float);
-  const size_t fsmem = (size_t)a.T * THREADS * sizeof(float4) + (size_t)WARPS * a.T * 32 * sizeof(float) + ssmem;
+  const size_t fsmem =
+      (size_t)((a.T + 1) / 2) * THREADS * sizeof(float4) + (size_t)WARPS * a.T * 32 * sizeof(float) + ssmem;
   cudaError_t e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
   if (e != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(hstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
