@@ -609,7 +609,7 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
 # ---------------------------------------------------------------- scan gradient
 
 BWD_METRIC = "R2L reverse-scan backward tokens/sec at B=8,L=4096,E=4096 (fp32)"
-BWD_LAUNCHES = 8          # kernels one r2l_reverse_scan_backward call launches
+BWD_LAUNCHES = 6          # kernels one r2l_reverse_scan_backward call launches
 
 
 def bwd_bytes_per_token(E):

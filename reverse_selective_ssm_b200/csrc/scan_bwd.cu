@@ -17,19 +17,19 @@
 //   dA_log = A ⊙ Σ_i Δ_i G_i ⊙ H_{i+1} ⊙ a_i,  dD = Σ_i dp_i u_i,  ddt_b = Σ_i ddt_raw_i
 //
 // The adjoint G runs left to right while H runs right to left, so both are
-// split into chunks of T positions:
-//   1. hstate: each chunk scans H right to left from zero; stores its end
-//      state and Σ Δ over the chunk;
-//   2. hcarry: per (sequence, channel, state), the state entering each chunk
-//      from the right, H_in(k) = S_{k+1} + exp(A Σ_{k+1}Δ) H_in(k+1);
-//   3. gstate: each chunk runs G left to right from zero; stores its end value
-//      and Σ Δ over positions s-1 … e-2 (the decays it crossed);
-//   4. gcarry: G entering each chunk from the left, the same recurrence in
-//      the other direction;
-//   5. final: each chunk recomputes its H from H_in(k) into shared memory,
-//      then walks G from the carried value and writes every gradient;
-//   6. two fixed-order reductions: the per-chunk parameter partials and the
-//      per-block partial sums of dB | dC (deterministic, no atomics).
+// split into chunks of T positions, in 6 launches:
+//   1. state: each chunk scans H right to left from zero (its end state and
+//      Σ Δ over the chunk) and G left to right from zero (its end value and
+//      Σ Δ over positions s-1 … e-2, the decays it crossed);
+//   2. carry: per (sequence, channel, state), the state entering each chunk
+//      from the right, H_in(k) = S_{k+1} + exp(A Σ_{k+1}Δ) H_in(k+1), and G
+//      entering each chunk from the left, the same recurrence the other way;
+//   3. final: each chunk recomputes its H from H_in(k), keeping every second
+//      position, then walks G from the carried value two positions at a
+//      time and writes every gradient;
+//   4.-6. fixed-order reductions: the per-chunk parameter partials (two
+//      levels) and the per-block partial sums of dB | dC (deterministic, no
+//      atomics).
 //
 // Threads: four per channel, thread q holding states 4q … 4q+3 (float4 loads
 // of B, C and the state rows), 64 channels per 256-thread block.  Sums over
@@ -232,43 +232,80 @@ __device__ __forceinline__ void stage_chunk(const Args& a, const Lane& l, const 
   }
 }
 
-// 1. H right to left over the chunk from zero.
-__global__ void __launch_bounds__(THREADS) hstate_kernel(const Args a) {
+// 1. + 3. Per chunk, from zero: H right to left (its end state and Σ Δ over
+// the chunk) and G left to right (its end value and Σ Δ over positions
+// s-1 … e-2, the decays it crosses), from one staging of the chunk.
+__global__ void __launch_bounds__(THREADS) state_kernel(const Args a) {
   extern __shared__ float4 sm4[];
   const Lane l = lane_setup(a);
   const Stage sg = stage_layout(reinterpret_cast<float*>(sm4), a.T);
-  stage_chunk<S_DL | S_DU>(a, l, sg);
-  __syncthreads();
+  stage_chunk<S_DL | S_DU | S_DP>(a, l, sg);
   const size_t ci = carry_idx(a, l);
   const int ch = threadIdx.x >> 2;
-  float2 H[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  float sd = 0.0f;
-  auto step = [&](int r) {
-    const float delta = sg.arr[1][r * CPB + ch];
-    const float2 du = dup2(sg.arr[2][r * CPB + ch]);
-    const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
-    sd += delta;
-    float2 ad[2];
-    decays(l, delta, ad);
-    H[0] = __ffma2_rn(ad[0], H[0], __fmul2_rn(du, lo2(Bq)));
-    H[1] = __ffma2_rn(ad[1], H[1], __fmul2_rn(du, hi2(Bq)));
-  };
-  if (a.T == 16 && l.e - l.s == 16) {
+  const bool full = a.T == 16 && l.e - l.s == 16;
+  float prev = 0.0f;                                   // Δ_{s-1}
+  if (l.s > 0 && l.s < l.e) prev = softplus_fwd(a.dt[((size_t)l.b * a.L + l.s - 1) * a.E + l.c] + a.dt_b[l.c]);
+  __syncthreads();
+  {
+    float2 H[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float sd = 0.0f;
+    auto step = [&](int r) {
+      const float delta = sg.arr[1][r * CPB + ch];
+      const float2 du = dup2(sg.arr[2][r * CPB + ch]);
+      const float4 Bq = ld4(sg.bc + r * 32 + 4 * l.q);
+      sd += delta;
+      float2 ad[2];
+      decays(l, delta, ad);
+      H[0] = __ffma2_rn(ad[0], H[0], __fmul2_rn(du, lo2(Bq)));
+      H[1] = __ffma2_rn(ad[1], H[1], __fmul2_rn(du, hi2(Bq)));
+    };
+    if (full) {
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) step(15 - rr);
-  } else {
-    for (int r = l.e - l.s - 1; r >= 0; --r) step(r);
+      for (int rr = 0; rr < 16; ++rr) step(15 - rr);
+    } else {
+      for (int r = l.e - l.s - 1; r >= 0; --r) step(r);
+    }
+    st4(a.hcar + ci * 16 + 4 * l.q, make_float4(H[0].x, H[0].y, H[1].x, H[1].y));
+    if (l.q == 0) a.hsd[ci] = sd;
   }
-  st4(a.hcar + ci * 16 + 4 * l.q, make_float4(H[0].x, H[0].y, H[1].x, H[1].y));
-  if (l.q == 0) a.hsd[ci] = sd;
+  {
+    float2 G[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float sd = 0.0f;
+    auto step = [&](int r) {
+      const float delta = sg.arr[1][r * CPB + ch];
+      const float dp = sg.arr[3][r * CPB + ch];
+      const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
+      if (r > 0) {
+        float2 ad[2];
+        decays(l, prev, ad);
+        G[0] = __fmul2_rn(G[0], ad[0]);
+        G[1] = __fmul2_rn(G[1], ad[1]);
+      }
+      if (r > 0 || l.s > 0) sd += prev;
+      G[0] = __ffma2_rn(dup2(dp), lo2(Cq), G[0]);
+      G[1] = __ffma2_rn(dup2(dp), hi2(Cq), G[1]);
+      prev = delta;
+    };
+    if (full) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) step(r);
+    } else {
+      for (int r = 0; r < l.e - l.s; ++r) step(r);
+    }
+    st4(a.gcar + ci * 16 + 4 * l.q, make_float4(G[0].x, G[0].y, G[1].x, G[1].y));
+    if (l.q == 0) a.gsd[ci] = sd;
+  }
 }
 
-// 2. / 4. Carries over the chunks of one (sequence, channel, state): right to
-// left for H (rev), left to right for G.  buf[k] ← value entering chunk k,
-// running = buf_old[k] + exp(A·sd[k]) · running.
-__global__ void carry_kernel(const Args a, float* buf, const float* sd, bool rev) {
+// 2. + 4. Carries over the chunks of one (sequence, channel, state), for H
+// (blockIdx.z = 0: right to left) and G (blockIdx.z = 1: left to right):
+// buf[k] ← the value entering chunk k, running = buf_old[k] + exp(A·sd[k])·running.
+__global__ void carry_kernel(const Args a) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // c·16 + m
   const int b = blockIdx.y;
+  const bool rev = blockIdx.z == 0;
+  float* buf = rev ? a.hcar : a.gcar;
+  const float* sd = rev ? a.hsd : a.gsd;
   if (t >= (long long)a.E * 16) return;
   const int c = (int)(t >> 4), m = (int)(t & 15);
   const float A = -expf(a.A_log[(size_t)c * 16 + m]);
@@ -294,44 +331,6 @@ __global__ void carry_kernel(const Args a, float* buf, const float* sd, bool rev
       }
     }
   }
-}
-
-// 3. G left to right over the chunk from zero.
-__global__ void __launch_bounds__(THREADS) gstate_kernel(const Args a) {
-  extern __shared__ float4 sm4[];
-  const Lane l = lane_setup(a);
-  const Stage sg = stage_layout(reinterpret_cast<float*>(sm4), a.T);
-  stage_chunk<S_DL | S_DP>(a, l, sg);
-  const size_t ci = carry_idx(a, l);
-  const int ch = threadIdx.x >> 2;
-  float2 G[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  float sd = 0.0f, prev = 0.0f;
-  if (l.s > 0 && l.s < l.e) prev = softplus_fwd(a.dt[((size_t)l.b * a.L + l.s - 1) * a.E + l.c] + a.dt_b[l.c]);
-  __syncthreads();
-  // decays crossed: positions s-1 … e-2 (G_{s-1} multiplies a_{s-1})
-  auto step = [&](int r) {
-    const float delta = sg.arr[1][r * CPB + ch];
-    const float dp = sg.arr[3][r * CPB + ch];
-    const float4 Cq = ld4(sg.bc + r * 32 + 16 + 4 * l.q);
-    if (r > 0) {
-      float2 ad[2];
-      decays(l, prev, ad);
-      G[0] = __fmul2_rn(G[0], ad[0]);
-      G[1] = __fmul2_rn(G[1], ad[1]);
-    }
-    if (r > 0 || l.s > 0) sd += prev;
-    G[0] = __ffma2_rn(dup2(dp), lo2(Cq), G[0]);
-    G[1] = __ffma2_rn(dup2(dp), hi2(Cq), G[1]);
-    prev = delta;
-  };
-  if (a.T == 16 && l.e - l.s == 16) {
-#pragma unroll
-    for (int r = 0; r < 16; ++r) step(r);
-  } else {
-    for (int r = 0; r < l.e - l.s; ++r) step(r);
-  }
-  st4(a.gcar + ci * 16 + 4 * l.q, make_float4(G[0].x, G[0].y, G[1].x, G[1].y));
-  if (l.q == 0) a.gsd[ci] = sd;
 }
 
 // 5. Per chunk: H from H_in(k), right to left, keeping it at every second
@@ -629,22 +628,17 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   const int nseg = (int)(((size_t)g.B * a.nc + RSEG - 1) / RSEG);
 
   const dim3 grid(g.E / CPB, a.nc, g.B);
-  const dim3 cgrid((unsigned)((g.E * 16 + 255) / 256), g.B);
+  const dim3 cgrid((unsigned)((g.E * 16 + 255) / 256), g.B, 2);
   const size_t ssmem = stage_floats(a.T) * sizeof(float);
   const size_t fsmem =
       (size_t)((a.T + 1) / 2) * THREADS * sizeof(float4) + (size_t)WARPS * a.T * 32 * sizeof(float) + ssmem;
   cudaError_t e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
   if (e != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(hstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
+  if ((e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
       cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(gstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem)) !=
-      cudaSuccess)
-    return e;
-  hstate_kernel<<<grid, THREADS, ssmem, st>>>(a);
-  carry_kernel<<<cgrid, 256, 0, st>>>(a, a.hcar, a.hsd, true);
-  gstate_kernel<<<grid, THREADS, ssmem, st>>>(a);
-  carry_kernel<<<cgrid, 256, 0, st>>>(a, a.gcar, a.gsd, false);
+  state_kernel<<<grid, THREADS, ssmem, st>>>(a);
+  carry_kernel<<<cgrid, 256, 0, st>>>(a);
   final_kernel<<<grid, THREADS, fsmem, st>>>(a);
   reduce_params_seg_kernel<<<dim3((unsigned)((g.E * 16 + 255) / 256), nseg), 256, 0, st>>>(a, seg);
   reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a, seg, nseg);
