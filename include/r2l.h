@@ -271,7 +271,8 @@ R2L_API size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims *dims, in
  * bitwise reproducible for a given chunk_tokens.
  *
  * Supported: dims->dtype == R2L_FP32 (every activation array is fp32),
- * d_state == 16, d_inner a multiple of 64, the right-to-left block (the
+ * d_state == 16, d_inner a multiple of 64, B and L up to 65535 with
+ * B·⌈L / chunk⌉ ≤ 2,097,120 (grid limits), the right-to-left block (the
  * R2L_FLAG_FORWARD_SCAN flag returns R2L_ERR_UNSUPPORTED); ldz, ld_dz and
  * ldbc multiples of 4.  chunk_tokens: positions per chunk (1 … 32; larger values are
  * clamped to 32; 0 = 16).  workspace ≥

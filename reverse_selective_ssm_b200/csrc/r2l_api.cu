@@ -502,6 +502,7 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
 size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims* dims, int B, int L, int chunk_tokens) {
   if (!dims || B <= 0 || L <= 0 || dims->d_inner <= 0 || chunk_tokens < 0) return 0;
   if (dims->dtype != R2L_FP32 || dims->d_state != 16 || dims->d_inner % 64) return 0;
+  if (!r2l::scan_bwd_supported(B, L, dims->d_inner, chunk_tokens)) return 0;
   return align_up(16, kAlign) + align_up(r2l::scan_bwd_scratch_bytes(B, L, dims->d_inner, chunk_tokens), kAlign);
 }
 
@@ -522,7 +523,7 @@ r2l_status r2l_reverse_scan_backward(const void* u, const void* z, int ldz, cons
   if (E % 64) return R2L_ERR_UNSUPPORTED;
   if (ldz < E || ld_dz < E || ldbc < 32 || ld_dbc < 32) return R2L_ERR_INVALID_ARG;
   if ((ldbc % 4) || (ldz % 4) || (ld_dz % 4)) return R2L_ERR_ALIGNMENT;
-  if (L > 65535 || B > 65535) return R2L_ERR_UNSUPPORTED;
+  if (L > 65535 || B > 65535 || !r2l::scan_bwd_supported(B, L, E, chunk_tokens)) return R2L_ERR_UNSUPPORTED;
   for (const void* q : {u, z, dt_raw, (const void*)bc, (const void*)A_log, (const void*)D, (const void*)dt_b, dy,
                         (const void*)du, (const void*)dz, (const void*)ddt_raw, (const void*)dbc,
                         (const void*)dA_log, (const void*)dD, (const void*)ddt_b})

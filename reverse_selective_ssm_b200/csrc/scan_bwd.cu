@@ -595,6 +595,13 @@ int scan_bwd_chunk_tokens(int chunk_tokens) {
   return chunk_tokens > SCAN_BWD_MAX_CHUNK ? SCAN_BWD_MAX_CHUNK : chunk_tokens;
 }
 
+bool scan_bwd_supported(int B, int L, int E, int chunk_tokens) {
+  const int T = scan_bwd_chunk_tokens(chunk_tokens);
+  const long long nc = (L + T - 1) / T;
+  const long long nseg = ((long long)B * nc + sbwd::RSEG - 1) / sbwd::RSEG;
+  return E % sbwd::CPB == 0 && nc <= 65535 && B <= 65535 && nseg <= 65535;
+}
+
 size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens) {
   const int T = scan_bwd_chunk_tokens(chunk_tokens);
   const size_t nc = (size_t)((L + T - 1) / T);

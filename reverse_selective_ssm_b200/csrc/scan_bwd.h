@@ -19,6 +19,7 @@ struct ScanBwdArgs {
 };
 
 int scan_bwd_chunk_tokens(int chunk_tokens);
+bool scan_bwd_supported(int B, int L, int E, int chunk_tokens);   // grid limits of the launches
 size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens);
 cudaError_t scan_bwd_f32(const ScanBwdArgs& a, void* scratch, cudaStream_t st);
 

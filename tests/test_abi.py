@@ -168,3 +168,6 @@ def test_scan_backward_argument_checks(lib):
     assert _bwd(lib, ws=None) == 4
     assert _bwd(lib, ws_bytes=16) == 4
     assert _bwd(lib, ws=FAKE + 8) == 3
+    big = bd.make_dims(64, 128, dtype=torch.float32)
+    assert bd.reverse_scan_backward_workspace_size(big, 65535, 65535, 1) == 0     # beyond the launch grid
+    assert _bwd(lib, B=65535, L=65535, chunk=1, ws_bytes=1 << 40) == 2
