@@ -22,7 +22,7 @@ below are that block: in_proj -> depthwise conv of width d_conv -> SiLU ->
 data-dependent (Δ, B, C) projections -> softplus(Δ) -> selective scan with
 Ā = exp(ΔA), B̄u = ΔBu -> + D·u -> ·SiLU(z) -> out_proj.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * the flip of step ❶ and the un-flip of step ❸ are applied per sequence to
     its valid prefix [0, len_b) of a right-padded row; in original coordinates
     the block therefore runs from position len_b-1 down to 0 with a zero
