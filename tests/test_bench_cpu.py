@@ -1,0 +1,62 @@
+"""bench.py's JSON line on the CPU: the reference arm (the oracle timed on the
+host cores) prints one line with the contract's keys, for the forward
+workload and for the scan gradient, and a non-zero rank prints nothing."""
+import contextlib
+import io
+import json
+
+import bench
+
+
+def _run(argv, env=None, monkeypatch=None):
+    if env and monkeypatch:
+        for k, v in env.items():
+            monkeypatch.setenv(k, v)
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.main(argv)
+    assert rc == 0
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
+    return [json.loads(ln) for ln in lines]
+
+
+KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e")
+
+
+def _check(line, metric):
+    for k in KEYS:
+        assert k in line, k
+    assert line["metric"] == metric
+    assert line["impl"] == "reference"
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert "workload" in line["config"]
+
+
+def test_reference_arm_forward_line():
+    out = _run(["--impl", "reference", "--steps", "1", "--warmup", "0", "--seq", "64"])
+    assert len(out) == 1
+    _check(out[0], bench.METRIC)
+
+
+def test_reference_arm_scan_backward_line():
+    out = _run(["--impl", "reference", "--scan-backward", "--steps", "1", "--warmup", "0"])
+    assert len(out) == 1
+    _check(out[0], bench.BWD_METRIC)
+    assert out[0]["dtype"] == "f64"
+
+
+def test_reference_arm_other_ranks_print_nothing(monkeypatch):
+    out = _run(["--impl", "reference", "--steps", "1", "--warmup", "0", "--seq", "64"],
+               env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, monkeypatch=monkeypatch)
+    assert out == []
+
+
+def test_scan_backward_algorithmic_bytes():
+    """114,944 B per position at d_inner 4096: 7 fp32 arrays of E channels
+    (u, z, dt_raw, dy read; du, dz, ddt_raw written) and B | C read, dB | dC
+    written (32 fp32 each)."""
+    assert bench.bwd_bytes_per_token(4096) == 4096 * 7 * 4 + 2 * 32 * 4 == 114944
