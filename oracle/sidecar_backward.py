@@ -45,7 +45,7 @@ import numpy as np
 from .r2l_oracle import LN_EPS, silu, sidecar_sequence
 from .scan_backward import reverse_scan_backward, sigmoid
 
-__all__ = ["sidecar_sequence_backward"]
+__all__ = ["sidecar_sequence_backward", "sidecar_backward_batch"]
 
 
 def _silu_grad(v):
@@ -136,3 +136,25 @@ def sidecar_sequence_backward(h, w, s, dh_out, length=None):
     out["dW_in"] = np.matmul(dxz.T, hv)
     assert np.allclose(silu(pre), u)
     return out
+
+
+def sidecar_backward_batch(h, w, s, dh_out, lengths=None):
+    """The same over a right-padded batch: h, dh_out [B, L, d_model].  Each
+    sequence b uses its first lengths[b] positions; padding rows pass dh_out
+    through unchanged (the hook neither reads nor writes them), and the
+    parameter gradients and ds are summed over the sequences."""
+    Bt, L, _ = h.shape
+    lens = [L] * Bt if lengths is None else [int(x) for x in lengths]
+    total = None
+    dh = np.empty_like(np.asarray(dh_out, dtype=np.float64))
+    for b in range(Bt):
+        g = sidecar_sequence_backward(h[b], w, s, dh_out[b], lens[b])
+        dh[b] = g.pop("dh")
+        if total is None:
+            total = g
+        else:
+            for k, v in g.items():
+                if v is not None:
+                    total[k] = total[k] + v
+    total["dh"] = dh
+    return total

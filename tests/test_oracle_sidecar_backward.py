@@ -102,3 +102,27 @@ def test_finite_difference_pin_catches_planted_mistake(monkeypatch):
     g = SB.sidecar_sequence_backward(h, w, 0.7, dh)
     fd = _fd_array(lambda: _loss(h, w, 0.7, dh, 6), w["conv_b"])
     assert _rel(g["dconv_b"], fd) > 1e-3
+
+
+def test_batched_backward_padding_and_sums():
+    """Ragged batch: each sequence's gradient is the single-sequence one on its
+    valid prefix, padding rows pass dh⁺ through, parameter gradients add up;
+    and a whole batch still matches finite differences of the batched forward."""
+    from oracle.sidecar_backward import sidecar_backward_batch
+    rng = np.random.default_rng(21)
+    Bt, L = 3, 6
+    lens = [6, 0, 3]
+    h = rng.standard_normal((Bt, L, D_MODEL))
+    dh = rng.standard_normal((Bt, L, D_MODEL))
+    w = _weights(6)
+    s = -0.4
+    g = sidecar_backward_batch(h, w, s, dh, lens)
+    for b, n in enumerate(lens):
+        one = sidecar_sequence_backward(h[b], w, s, dh[b], n)
+        assert np.array_equal(g["dh"][b], one["dh"])
+        assert np.array_equal(g["dh"][b, n:], dh[b, n:])
+    fd = _fd_array(lambda: float(np.sum(dh * O.sidecar_forward(h, w, s, np.array(lens)))), w["W_x"])
+    assert _rel(g["dW_x"], fd) < 1e-6
+    sv = np.array([s])
+    fds = _fd_array(lambda: float(np.sum(dh * O.sidecar_forward(h, w, sv[0], np.array(lens)))), sv)[0]
+    assert abs(g["ds"] - fds) <= 1e-6 * max(1.0, abs(fds))
