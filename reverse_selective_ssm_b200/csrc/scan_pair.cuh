@@ -1,7 +1,9 @@
 // Reverse selective scan with two threads per channel ("Bifocal Diffusion
 // Language Models", arXiv 2606.27732v1, §3.4 step ❷; the recurrence and its
-// terms are those of scan_fast.cuh), for the final pass over whole sequences
-// with dt_proj fused (bf16, dt_rank 128).
+// terms are those of scan_fast.cuh) with dt_proj fused (bf16, dt_rank 128):
+// one pass over whole sequences, or, when sequences are split into chunks,
+// the state-only first pass (FINAL = false) and the final pass from the
+// carried states (FINAL = true).
 //
 // Why: at batch 8 a sequence-length scan has only B·E = 32,768 independent
 // channel chains, about 7 warps per SM with one thread per channel, and each
