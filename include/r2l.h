@@ -69,7 +69,19 @@ typedef enum {
   R2L_FP32 = 1    /* fp32 everywhere, true fp32 arithmetic (no TF32) */
 } r2l_dtype;
 
-/* r2l_dims.flags */
+/* r2l_dims.flags
+ *
+ * The scan's power path (bf16 path only).  When A is the S4D-real
+ * initialisation A[c][m] = -(m+1), the 16 decays exp(Δ·A[c][m]) of a (position,
+ * channel) are the powers r, r², …, r¹⁶ of r = exp(-Δ), so the scan needs one
+ * reciprocal instead of 16 exponentials.  The choice is made once per call
+ * (per hook of r2l_sidecar_stack), on the device, by an exact test: the power
+ * path is taken when every A_log[c][m] equals, bit for bit, the float nearest
+ * ln(m+1), and the scan then uses A[c][m] = -(m+1) exactly (it differs from
+ * -exp(A_log[c][m]) by less than 2e-7 relative).  Any other A_log, even one
+ * entry, sends the whole call down the general path (one exponential per
+ * state).  R2L_FLAG_GENERAL_A skips the test and always takes the general
+ * path.  The fp32 path always evaluates exp(Δ·A) directly.                   */
 #define R2L_FLAG_GENERAL_A 0x1u     /* never take the A = -(1..16) power fast path of the scan    */
 #define R2L_FLAG_FORWARD_SCAN 0x2u  /* run the block left to right instead: causal conv and a
                                        forward scan (the "L2R Mamba" control of Table 4); every
@@ -230,9 +242,11 @@ R2L_API r2l_status r2l_reverse_scan(const void *u, const void *z, int ldz, const
  * of R2L_NOALLOC_SCRATCH_BYTES that the library's device code declares; every
  * device that loads the library holds it until the process exits.  The entry
  * point calls no cudaMalloc, cudaFree or other allocating routine.
- *   - The first call on a device looks up the array's device address with
- *     that device current and caches it; make that first call before any
- *     stream capture.
+ *   - Every call looks up the array's device address in the current device's
+ *     context (cudaGetSymbolAddress; nothing is allocated), so the address
+ *     stays right after cudaDeviceReset.  The first call on a device also
+ *     loads the library's device image into that context; make that first
+ *     call before any stream capture.
  *   - All calls share the one array, which keeps the last call's contents
  *     (each call rewrites what it reads).  Calls whose work overlaps on the
  *     GPU (for instance on two streams) race on it; order them.

@@ -2,8 +2,6 @@
 // device status word, the clamped lengths and the chunk carries) held in a
 // fixed-size array that is part of the library's device image, for callers
 // that must not allocate device memory at run time.
-#include <mutex>
-
 #include "r2l.h"
 
 namespace {
@@ -14,23 +12,19 @@ namespace {
 // cudaGetSymbolAddress returns for the current device.
 static __device__ __align__(256) unsigned char g_scan_scratch[R2L_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_scan_scratch on the current device, looked up on the
-// first call for that device (with that device current) and cached.
+// Device address of g_scan_scratch in the current device's context, looked up
+// on every call.  The lookup allocates nothing; not caching it means a call
+// after cudaDeviceReset (or after the primary context was destroyed and made
+// again) gets the array's address in the new context instead of a dangling
+// one.  The very first lookup on a device loads the library's device image
+// into that context.
 r2l_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return R2L_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return R2L_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess || !p) return R2L_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return R2L_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return R2L_OK;
 }
 

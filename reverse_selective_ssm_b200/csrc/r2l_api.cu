@@ -64,11 +64,12 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->u = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->dbc = off;    off = align_up(off + M * p->ldd * sizeof(float), kAlign);
   p->dr = off;     off = align_up(off + M * p->R * 2, kAlign);   // Δr in bf16 (tensor-core path)
-  p->dt = off;     off = align_up(off + M * p->E * p->act, kAlign);
+  // the bf16 layer with dt_rank 128 runs dt_proj inside the scan: dt_raw never
+  // reaches memory, so its region is only reserved for the other paths
+  const bool pair = dm->dtype == R2L_BF16 && p->R == r2l::kScanFusedDtRank;
+  p->dt = off;     if (!pair) off = align_up(off + M * p->E * p->act, kAlign);
   p->y = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->o = off;      off = align_up(off + M * p->d * p->act, kAlign);
-  // the bf16 layer with dt_rank 128 runs the scan with dt_proj fused (two threads per channel)
-  const bool pair = dm->dtype == R2L_BF16 && p->R == r2l::kScanFusedDtRank;
   p->chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, p->E, 0, pair);
   p->carry = off;
   if (dm->dtype == R2L_BF16) off = align_up(off + r2l::scan_carry_bytes(B, L, p->E, p->chunk_tokens, pair), kAlign);
@@ -145,6 +146,29 @@ r2l_status prep(const Plan& p, char* ws, const int32_t* lengths, int B, int L, c
   if (cudaMemsetAsync(ws + p.status, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
   r2l::prep_lengths_kernel<<<(B + 127) / 128, 128, 0, st>>>(
       lengths, (int*)(ws + p.len), B, L, (unsigned*)(ws + p.status));
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+// The float nearest ln(m+1) for m = 0..15: the A_log of the S4D-real
+// initialisation A = −(1..16), against which a_log_check_kernel compares.
+r2l::LnTable ln_table() {
+  r2l::LnTable t;
+  for (int m = 0; m < 16; ++m) {
+    const float v = (float)std::log((double)(m + 1));
+    std::memcpy(&t.bits[m], &v, sizeof(v));
+  }
+  return t;
+}
+
+// Decide the scan's power path for this call (see a_log_check_kernel): writes
+// 0 or 1 into the second word of the status region.  With force_general the
+// scan never reads it.
+r2l_status check_a_log(const float* A_log, int E, unsigned* status, bool force_general, cudaStream_t st,
+                       Prof* prof) {
+  if (force_general) return R2L_OK;
+  if (prof) prof->launches++;
+  r2l::a_log_check_kernel<<<1, 1024, 0, st>>>(A_log, E, ln_table(), status + 1);
   R2L_LAUNCH_CHECK();
   return R2L_OK;
 }
@@ -278,6 +302,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
   prof->launches++;
   if constexpr (kTC) {
+    R2L_TRY(check_a_log(w->A_log, E, err, (p.flags & R2L_FLAG_GENERAL_A) != 0, st, prof));
     r2l::ScanArgs sa{};
     sa.u = u; sa.ldu = E;
     sa.z = xz + E; sa.ldz = 2 * E;
@@ -290,6 +315,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.carry = (float*)(ws + p.carry);
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
+    sa.a_general = err + 1;
     sa.dt_mma = dt_fused ? 1 : 0;
     sa.forward = fwd ? 1 : 0;
     sa.dr = dr; sa.lddr = R;
@@ -474,6 +500,8 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
   r2l::prep_lengths_kernel<<<(B + 127) / 128, 128, 0, st>>>(lengths, len, B, L, status);
   R2L_LAUNCH_CHECK();
   if (dims->dtype == R2L_BF16) {
+    const bool force_general = (dims->flags & R2L_FLAG_GENERAL_A) != 0;
+    R2L_TRY(check_a_log(A_log, E, status, force_general, st, nullptr));
     r2l::ScanArgs sa{};
     sa.u = (const bf16*)u; sa.ldu = E;
     sa.z = (const bf16*)z; sa.ldz = ldz;
@@ -485,7 +513,8 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
     sa.chunk_tokens = r2l::scan_resolve_chunk_tokens(B, L, E, chunk_tokens);
     sa.carry = carry;
     sa.err = status;
-    sa.force_general = (int)(dims->flags & R2L_FLAG_GENERAL_A);
+    sa.force_general = force_general ? 1 : 0;
+    sa.a_general = status + 1;
     sa.forward = (dims->flags & R2L_FLAG_FORWARD_SCAN) ? 1 : 0;
     if (r2l::scan_bf16(sa, st, nullptr) != cudaSuccess) return R2L_ERR_CUDA;
   } else {

@@ -27,6 +27,8 @@ struct ScanArgs {
   float* carry;                                // scan_carry_bytes() of device scratch (may be null if 1 chunk)
   unsigned* err;                               // device status word
   int force_general;                           // never use the A = -(1..16) power path
+  const unsigned* a_general;                   // device flag of a_log_check_kernel (0: power path); read
+                                               // unless force_general
   int dt_mma;                                  // compute dt_raw = Δr·W_dtᵀ inside the scan (dt_rank 128)
   int forward;                                 // left-to-right block
 };

@@ -165,6 +165,8 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.carry_sum = a.carry ? a.carry + (size_t)a.B * nc * a.E * 16 : nullptr;
   p.err = a.err;
   p.force_general = a.force_general;
+  p.a_general = a.a_general;
+  if (!a.force_general && !a.a_general) return cudaErrorInvalidValue;
   p.fwd = a.forward;
   if (a.dt_mma) {
     if (!a.dr || !a.wdt || (a.lddr % 8)) return cudaErrorInvalidValue;

@@ -421,7 +421,6 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
   cx.upper = h != 0;
   cx.dtb = cvalid ? p.dt_b[c] : 0.0f;
   cx.Dc = cvalid ? p.D[c] : 0.0f;
-  bool pow_ok = true;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
@@ -429,10 +428,9 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
       const int m = 4 * kk + 2 * e + h;
       const float a = cvalid ? -expf(p.A_log[c * 16 + m]) : -(float)(m + 1);
       cx.A2[2 * kk + e] = a * LOG2E;
-      pow_ok = pow_ok && fabsf(a + (float)(m + 1)) <= 1e-5f * (float)(m + 1);
     }
   }
-  const bool use_pow = !p.force_general && __all_sync(0xffffffffu, pow_ok);
+  const bool use_pow = !p.force_general && *p.a_general == 0u;
   // the thread's states m = 4kk + 2e + h sit at H[kk].x (e = 0) and H[kk].y (e = 1)
   float2 H[4];
   float* cst = (p.nc > 1 && cvalid) ? p.carry + (((long long)b * p.nc + k) * p.E + c) * 16 : nullptr;

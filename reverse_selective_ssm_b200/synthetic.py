@@ -107,14 +107,37 @@ def make_weights(dims: Dims, dtype: torch.dtype, seed: int, *, std: float = 0.02
     return w
 
 
-def make_hidden(B: int, L: int, d: int, dtype: torch.dtype, seed: int) -> torch.Tensor:
-    g = torch.Generator().manual_seed(seed)
-    return torch.randn((B, L, d), generator=g, dtype=torch.float32).to(dtype)
+def _sequence_generator(seed: int, index: int) -> torch.Generator:
+    """The generator of global sequence ``index`` of a batch drawn with ``seed``."""
+    return torch.Generator().manual_seed(seed * 1_000_003 + index)
 
 
-def make_lengths(B: int, lo: int, hi: int, seed: int) -> torch.Tensor:
-    g = torch.Generator().manual_seed(seed)
-    return torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+def make_hidden(B: int, L: int, d: int, dtype: torch.dtype, seed: int, first: int = 0) -> torch.Tensor:
+    """Hidden states [B, L, d] ~ N(0, 1).  Row b is global sequence first + b
+    and depends on (seed, first + b) only, so a contiguous slice of a global
+    batch (one rank's shard) is drawn with the same bits as the whole."""
+    out = torch.empty((B, L, d), dtype=torch.float32)
+    for b in range(B):
+        out[b] = torch.randn((L, d), generator=_sequence_generator(seed, first + b), dtype=torch.float32)
+    return out.to(dtype)
+
+
+def make_lengths(B: int, lo: int, hi: int, seed: int, first: int = 0) -> torch.Tensor:
+    """Valid lengths ~ U{lo..hi}, one draw per global sequence (as make_hidden)."""
+    vals = [int(torch.randint(lo, hi + 1, (1,), generator=_sequence_generator(seed + 7919, first + b)))
+            for b in range(B)]
+    return torch.tensor(vals, dtype=torch.int32)
+
+
+def shard_first(B: int, shard) -> int:
+    """First global sequence of a rank's shard: rank r of n takes sequences
+    [r·B, (r+1)·B) of a global batch of n·B (B sequences per rank)."""
+    if shard is None:
+        return 0
+    rank, world = shard
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world {world}")
+    return rank * B
 
 
 def poison_padding(h: torch.Tensor, lengths: torch.Tensor) -> torch.Tensor:
@@ -141,53 +164,70 @@ CONFIG_NAMES = {
 }
 
 
+def _meta(first: int, B: int, shard) -> dict:
+    world = 1 if shard is None else shard[1]
+    return {"first_sequence": first, "global_batch": B * world}
+
+
 def make_case(cfg: int, *, B: Optional[int] = None, L: Optional[int] = None,
-              weights: bool = True) -> Case:
-    """Build one of the five workloads (``B``/``L`` override for smaller runs)."""
+              weights: bool = True, shard=None) -> Case:
+    """Build one of the workloads (``B``/``L`` override for smaller runs).
+
+    ``shard`` = (rank, world): the case holds rank's contiguous slice of a
+    global batch of world·B sequences (B per rank); the weights are the same
+    on every rank, and the slice's hidden states and lengths are bit for bit
+    the rows of the global batch."""
     if cfg == 0:
         dims, dt = TINY, torch.float32
         Bv, Lv = (B or 1), (L or 64)
-        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=0)
+        first = shard_first(Bv, shard)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=0, first=first)
         ws = [make_weights(dims, dt, seed=100)] if weights else []
-        return Case(CONFIG_NAMES[0], dims, dt, Bv, Lv, h, ws, [0.5])
+        return Case(CONFIG_NAMES[0], dims, dt, Bv, Lv, h, ws, [0.5], meta=_meta(first, Bv, shard))
     if cfg == 1:
         dims, dt = BIG, torch.bfloat16
         Bv, Lv = (B or 1), (L or 2048)
-        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=1)
+        first = shard_first(Bv, shard)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=1, first=first)
         ws = [make_weights(dims, dt, seed=101)] if weights else []
-        return Case(CONFIG_NAMES[1], dims, dt, Bv, Lv, h, ws, [1.0])
+        return Case(CONFIG_NAMES[1], dims, dt, Bv, Lv, h, ws, [1.0], meta=_meta(first, Bv, shard))
     if cfg == 2:
         dims, dt = BIG, torch.bfloat16
         Bv, Lv = (B or 8), (L or 4096)
-        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=2)
+        first = shard_first(Bv, shard)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=2, first=first)
         ws = [make_weights(dims, dt, seed=102)] if weights else []
-        return Case(CONFIG_NAMES[2], dims, dt, Bv, Lv, h, ws, [0.3])
+        return Case(CONFIG_NAMES[2], dims, dt, Bv, Lv, h, ws, [0.3], meta=_meta(first, Bv, shard))
     if cfg == 3:
         dims, dt = BIG, torch.bfloat16
         Bv, Lv = (B or 4), (L or 8192)
-        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=3)
+        first = shard_first(Bv, shard)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=3, first=first)
         g = torch.Generator().manual_seed(3)
         s = (torch.rand((7,), generator=g, dtype=torch.float64) * 2.0 - 1.0).tolist()
         ws = [make_weights(dims, dt, seed=300 + k) for k in range(7)] if weights else []
-        return Case(CONFIG_NAMES[3], dims, dt, Bv, Lv, h, ws, s)
+        return Case(CONFIG_NAMES[3], dims, dt, Bv, Lv, h, ws, s, meta=_meta(first, Bv, shard))
     if cfg == 4:
         dims, dt = BIG, torch.bfloat16
         Bv, Lv = (B or 256), (L or 512)
-        lengths = make_lengths(Bv, min(64, Lv), Lv, seed=4)
-        h = poison_padding(make_hidden(Bv, Lv, dims.d_model, dt, seed=4), lengths)
+        first = shard_first(Bv, shard)
+        lengths = make_lengths(Bv, min(64, Lv), Lv, seed=4, first=first)
+        h = poison_padding(make_hidden(Bv, Lv, dims.d_model, dt, seed=4, first=first), lengths)
         ws = [make_weights(dims, dt, seed=104)] if weights else []
-        return Case(CONFIG_NAMES[4], dims, dt, Bv, Lv, h, ws, [0.7], lengths=lengths)
+        return Case(CONFIG_NAMES[4], dims, dt, Bv, Lv, h, ws, [0.7], lengths=lengths,
+                    meta=_meta(first, Bv, shard))
     if cfg == 5:
         # one denoising step of cached parallel decoding (§3.5, "Inference with
         # prefix KV cache"): the 7 hooks run over the generation block alone,
         # G = 128 positions of each of B = 8 requests (§4.1 throughput setup)
         dims, dt = BIG, torch.bfloat16
         Bv, Lv = (B or 8), (L or 128)
-        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=5)
+        first = shard_first(Bv, shard)
+        h = make_hidden(Bv, Lv, dims.d_model, dt, seed=5, first=first)
         g = torch.Generator().manual_seed(5)
         s = (torch.rand((7,), generator=g, dtype=torch.float64) * 2.0 - 1.0).tolist()
         ws = [make_weights(dims, dt, seed=500 + k) for k in range(7)] if weights else []
-        return Case(CONFIG_NAMES[5], dims, dt, Bv, Lv, h, ws, s)
+        return Case(CONFIG_NAMES[5], dims, dt, Bv, Lv, h, ws, s, meta=_meta(first, Bv, shard))
     raise ValueError(f"unknown config {cfg}")
 
 

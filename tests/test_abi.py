@@ -46,7 +46,11 @@ def test_abi_version_and_status_strings(lib):
 def test_workspace_size(lib):
     d = bd.make_dims(2048, 4096)
     a = bd.workspace_size(d, 8, 4096)
-    assert a > 8 * 4096 * 4096 * 2 * 5          # xz, u, dt, y at least
+    assert a > 8 * 4096 * 4096 * 2 * 4          # xz, u, y at least
+    # dt_rank 128 runs dt_proj inside the scan: no [M, d_inner] dt_raw region
+    assert a < 8 * 4096 * 4096 * 2 * 5
+    # dt_rank 64 (dt_proj as its own GEMM) adds the dt_raw region back; its Δr|B|C rows are 384 B shorter
+    assert bd.workspace_size(bd.make_dims(2048, 4096, dt_rank=64), 8, 4096) >= a + 8 * 4096 * (4096 * 2 - 384)
     assert bd.workspace_size(d, 8, 4096) == a     # deterministic
     assert bd.workspace_size(d, 16, 4096) > a
     assert bd.workspace_size(d, 0, 4096) == 0

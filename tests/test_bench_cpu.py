@@ -60,3 +60,21 @@ def test_scan_backward_algorithmic_bytes():
     (u, z, dt_raw, dy read; du, dz, ddt_raw written) and B | C read, dB | dC
     written (32 fp32 each)."""
     assert bench.bwd_bytes_per_token(4096) == 4096 * 7 * 4 + 2 * 32 * 4 == 114944
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """A short timed region at full clock with no power cap is measured against
+    the burst cuBLAS peak; a power-capped, long or low-clock run against the
+    sustained one; the note says which."""
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1370.0}
+    fast = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    p, note = bench.tensor_peak(peaks, "measured", fast, 40.0)
+    assert p == 1650.0 and "burst" in note
+    p, note = bench.tensor_peak(peaks, "measured", dict(fast, reasons=["sw_power_cap"]), 40.0)
+    assert p == 1370.0 and "power cap" in note
+    p, _ = bench.tensor_peak(peaks, "measured", fast, 4000.0)
+    assert p == 1370.0
+    p, _ = bench.tensor_peak(peaks, "measured", dict(fast, sm_mhz=1400.0), 40.0)
+    assert p == 1370.0
+    p, _ = bench.tensor_peak(peaks, "measured", None, 40.0)
+    assert p == 1370.0

@@ -55,12 +55,14 @@ def test_stack_in_cuda_graph_matches_direct_calls():
 
 
 def test_denoise_block_against_oracle():
-    """The full denoise-step shape (B=8, G=128, 7 hooks) against the oracle on
-    two requests."""
+    """The full denoise-step shape (B=8, G=128, 7 hooks): the final h⁺ against
+    the oracle's stack on requests 0 and 7; and the last hook, run through the
+    debug entry point on the GPU's hidden state after six hooks, against the
+    oracle's hook on that input (h⁺, pre-gate ĥ and y, requests 0 and 7)."""
     case = S.make_case(5)
-    got, _, flags = G.run_gpu(case)
-    assert flags == 0
+    before, got, dbg = G.run_gpu_stack_last_debug(case)
     want = G.run_oracle(case, [0, 7])
     for b in (0, 7):
         e = G.err_bf16(S.to_f64(got[b]), want[b])
         assert e <= G.TOL_BF16, f"b={b}: {e:.3e}"
+    G.check_sampled_rows(case, got, dbg, full=(0, 7), hook=6, h_in=before)

@@ -194,44 +194,92 @@ def test_lengths_out_of_range_are_clamped_and_flagged():
 
 
 # ----------------------------------------------------------------- full sizes
+#
+# At the full sizes every check covers h⁺ and, through the debug entry point,
+# the pre-gate ĥ and the scan output y: for small |s| a check on h⁺ alone
+# would admit a large error in ĥ, and with the workloads' N(0, 0.02) weights
+# and D = 1 the state term is a small part of y, so one case makes the scan
+# dominate (D = 0, O(1) B and C).
 
 def test_cfg2_serving_shape():
-    """B=8, L=4096: sequences 0 and 7 in full, the last 384 positions of the others."""
+    """B=8, L=4096: h⁺, ĥ and y for sequences 0 and 7 in full and the last
+    384 positions of the others (exact by right-context-only)."""
     case = S.make_case(2)
-    got, _, _ = G.run_gpu(case)
-    full = G.run_oracle(case, [0, 7])
-    for b in (0, 7):
-        _check_seq(case, got, full, b, "full")
-    suf = G.run_oracle(case, [1, 2, 3, 4, 5, 6], suffix=384)
-    for b in (1, 2, 3, 4, 5, 6):
-        n = case.L
-        e = G.err_bf16(S.to_f64(got[b, n - 384:]), suf[b, n - 384:])
-        assert e <= G.TOL_BF16, f"suffix b={b}: {e:.3e}"
+    got, dbg, flags = G.run_gpu(case, debug=True, keys=("y", "hhat"))
+    assert flags == 0
+    G.check_sampled_rows(case, got, dbg, full=(0, 7), suffix=384)
+
+
+def test_cfg2_serving_shape_scan_visible():
+    """The serving shape with the scan's state term dominating y (D = 0,
+    x_proj std 0.8, seeded LayerNorm): u, y, ĥ and h⁺ for sequences 0 and 7
+    in full and the last 384 positions of the others."""
+    case = S.make_case(2)
+    case.weights = [S.make_weights(case.dims, torch.bfloat16, seed=205, x_proj_std=0.8, D_value=0.0,
+                                   ln="seeded")]
+    got, dbg, flags = G.run_gpu(case, debug=True, keys=("u", "y", "hhat"))
+    assert flags == 0
+    G.check_sampled_rows(case, got, dbg, full=(0, 7), suffix=384, keys=("u", "y", "hhat"))
 
 
 def test_cfg3_stack_of_seven():
-    """B=4, L=8192, 7 hooks: sequence 3 in full, the last 256 positions of 0..2."""
+    """B=4, L=8192, 7 hooks.  The final h⁺ against the oracle's stack on
+    sequence 3 in full and the last 256 positions of 0..2; and the last hook,
+    run through the debug entry point on the GPU's hidden state after six
+    hooks, against the oracle's hook on that same input (h⁺, ĥ, y; sequence 3
+    in full and the last 256 positions of the others)."""
     case = S.make_case(3)
-    got, _, _ = G.run_gpu(case)
+    before, got, dbg = G.run_gpu_stack_last_debug(case)
     full = G.run_oracle(case, [3])
     _check_seq(case, got, full, 3, "stack full")
     suf = G.run_oracle(case, [0, 1, 2], suffix=256)
     for b in (0, 1, 2):
         e = G.err_bf16(S.to_f64(got[b, -256:]), suf[b, -256:])
         assert e <= G.TOL_BF16, f"stack suffix b={b}: {e:.3e}"
+    G.check_sampled_rows(case, got, dbg, full=(3,), suffix=256, hook=6, h_in=before)
 
 
 def test_cfg4_ragged_batch():
-    """B=256, L=512, lengths ~ U[64, 512], NaN padding: the shortest, the longest
-    and six random sequences against the oracle; all padding untouched."""
+    """B=256, L=512, lengths ~ U[64, 512], NaN padding: h⁺, ĥ and y of the
+    shortest, the longest and six random sequences against the oracle; all
+    padding untouched."""
     case = S.make_case(4)
-    got, _, flags = G.run_gpu(case)
+    got, dbg, flags = G.run_gpu(case, debug=True, keys=("y", "hhat"))
     assert flags == 0
     lens = case.lengths.numpy()
     rng = np.random.default_rng(4)
     pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens))] + rng.choice(256, 6, replace=False).tolist()))
-    want = G.run_oracle(case, pick)
-    for b in pick:
-        _check_seq(case, got, want, b, "ragged")
+    G.check_sampled_rows(case, got, dbg, full=pick)
     _padding_untouched(case, got)
     assert torch.isfinite(torch.cat([got[b, :int(n)].float().flatten() for b, n in enumerate(lens)])).all()
+
+
+# ----------------------------------------------------------------- the power path
+
+def test_power_path_is_decided_once_per_call_exactly():
+    """A_log one ulp away from ln(m+1) in a single (channel, state) sends the
+    whole call down the general path: its output equals, bit for bit, the
+    output of the same call with R2L_FLAG_GENERAL_A, while the unmodified
+    A_log takes the power path (a different rounding, so different bits)."""
+    case = S.make_case(1, B=2, L=512)
+    base = S.make_weights(case.dims, torch.bfloat16, seed=206, x_proj_std=0.8, D_value=0.0)
+    A = base["A_log"].clone()
+    A[1234, 5] = torch.nextafter(A[1234, 5], torch.tensor(float("inf")))
+    mod = dict(base, A_log=A)
+
+    def run(w, flags=0):
+        case.weights = [w]
+        _, dbg, fl = G.run_gpu(case, debug=True, flags=flags, keys=("y",))
+        assert fl == 0
+        return dbg["y"]
+
+    y_mod = run(mod)
+    y_mod_general = run(mod, bd.R2L_FLAG_GENERAL_A)
+    assert torch.equal(y_mod.view(torch.int16), y_mod_general.view(torch.int16))
+    y_pow = run(base)
+    y_pow_general = run(base, bd.R2L_FLAG_GENERAL_A)
+    assert not torch.equal(y_pow.view(torch.int16), y_pow_general.view(torch.int16))
+    # both paths stay within tolerance of the oracle
+    case.weights = [mod]
+    want, inter = G.run_oracle(case, [0], intermediates=True)
+    assert G.err_norm(S.to_f64(y_mod[:512]), inter[0]["y"]) <= G.TOL_BF16
