@@ -25,7 +25,7 @@
 // dt_raw values with one tcgen05.ld.  dt_raw never touches HBM.  The layer
 // itself runs the DTMMA scan as the two-threads-per-channel kernel of
 // scan_pair.cuh; this one-thread DTMMA form is kept as its compile-time
-// alternative (R2L_SCAN_PAIR=0), and the form without DTMMA serves dt_rank ≠ 128.
+// alternative (R2L_SCAN_IMPL=0), and the form without DTMMA serves dt_rank ≠ 128.
 //
 // When a sequence is split into several chunks (to give the GPU enough
 // independent work), three launches cooperate through a small carry buffer:

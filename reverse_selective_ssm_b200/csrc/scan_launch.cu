@@ -5,6 +5,7 @@
 #include "scan_fast.cuh"
 #include "scan_fast.h"
 #include "scan_pair.cuh"
+#include "scan_split.cuh"
 #include "tmap.h"
 
 namespace r2l {
@@ -55,11 +56,46 @@ size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens, bool pair) {
 
 namespace {
 
-// Two threads per channel, B|C broadcast through tensor memory, for scans with
-// dt_proj fused (0: one thread per channel, B|C read from shared memory).
-#ifndef R2L_SCAN_PAIR
-#define R2L_SCAN_PAIR 1
+// The kernel behind scans with dt_proj fused: 2 = the recurrence on warps of
+// its own (scan_split.cuh), 1 = two threads per channel (scan_pair.cuh),
+// 0 = one thread per channel with B|C read from shared memory.
+#ifndef R2L_SCAN_IMPL
+#define R2L_SCAN_IMPL 1
 #endif
+
+template <bool FWD>
+cudaError_t launch_split(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
+  using namespace rscan;
+  namespace sp = rscan::split;
+  constexpr int CHS = sp::CHS;
+  const long long M = (long long)a.B * a.L;
+  CUtensorMap tu, tz, tdr, tbc, ty, tw;
+  if (!make_tmap_2d(&tu, a.u, 2, a.E, M, a.ldu * 2, CHS, TS, 0) ||
+      !make_tmap_2d(&tz, a.z, 2, a.E, M, a.ldz * 2, CHS, TS, 0) ||
+      !make_tmap_2d(&tbc, a.bc, 4, 32, M, a.ldbc * 4, 32, TS, 0) ||
+      !make_tmap_2d(&ty, a.y, 2, a.E, M, a.ldy * 2, CHS, TS, 0) ||
+      !make_tmap_2d(&tdr, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, 128) ||
+      !make_tmap_rows_by_parity(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CHS / 2, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(sp::scan_split_kernel<true, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sp::Smem::BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((a.E + CHS - 1) / CHS, nc, a.B);
+  if (nc > 1) {
+    if ((e = cudaFuncSetAttribute(sp::scan_split_kernel<false, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sp::Smem::BYTES)) != cudaSuccess)
+      return e;
+    sp::scan_split_kernel<false, FWD><<<grid, sp::THREADS, sp::Smem::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (launches) *launches += 2;
+  }
+  sp::scan_split_kernel<true, FWD><<<grid, sp::THREADS, sp::Smem::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaSuccess;
+}
 
 template <bool FWD>
 cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream_t st, int* launches) {
@@ -122,7 +158,8 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
   }
   cudaError_t e;
   const dim3 grid((a.E + CH - 1) / CH, nc, a.B);
-  if (DTMMA && R2L_SCAN_PAIR) return launch_pair<FWD>(a, p, nc, st, launches);
+  if (DTMMA && R2L_SCAN_IMPL == 2) return launch_split<FWD>(a, p, nc, st, launches);
+  if (DTMMA && R2L_SCAN_IMPL == 1) return launch_pair<FWD>(a, p, nc, st, launches);
   if ((e = prep_kernel<true, DTMMA, FWD>()) != cudaSuccess) return e;
   if (nc > 1) {
     if ((e = prep_kernel<false, DTMMA, FWD>()) != cudaSuccess) return e;

@@ -188,11 +188,38 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float&
                                           uint32_t t_bc, unsigned* err, bool& ok) {
   const int lane = threadIdx.x & 31;
   const int h = lane >> 4;
+  // With FINAL, u and z of this thread's tokens are read one sub-tile ahead:
+  // the y of a sub-tile is stored over its z rows, and a read placed after
+  // those stores could not be moved above them (the compiler cannot tell the
+  // rows apart).  The state-only pass stores nothing and reads in place.
+  bf16 u_nx[GT / 2], z_nx[GT / 2];
+  if (FINAL) {
+#pragma unroll
+    for (int i = 0; i < GT / 2; ++i) {
+      const int j = (FWD ? 0 : TS - GT) + 2 * i + h;
+      u_nx[i] = su[j * CHP];
+      z_nx[i] = sz[j * CHP];
+    }
+  }
 #pragma unroll
   for (int sb = 0; sb < TS / GT; ++sb) {
     const int g = sb / (GB / GT);                  // B|C group of this sub-tile
     const int gs = sb % (GB / GT);                 // sub-tile within the group
     const int j0 = FWD ? sb * GT : TS - GT - sb * GT;
+    bf16 u_cur[GT / 2], z_cur[GT / 2];
+#pragma unroll
+    for (int i = 0; i < GT / 2; ++i) {
+      u_cur[i] = FINAL ? u_nx[i] : su[(j0 + 2 * i + h) * CHP];
+      if (FINAL) z_cur[i] = z_nx[i];
+    }
+    if (FINAL && sb + 1 < TS / GT) {
+      const int jn = FWD ? (sb + 1) * GT : TS - GT - (sb + 1) * GT;
+#pragma unroll
+      for (int i = 0; i < GT / 2; ++i) {
+        u_nx[i] = su[(jn + 2 * i + h) * CHP];
+        z_nx[i] = sz[(jn + 2 * i + h) * CHP];
+      }
+    }
     // phase A for this thread's tokens t = 2i + h of the sub-tile
     float dec_o[GT / 2], du_o[GT / 2], Du_o[GT / 2], gz_o[GT / 2];
 #pragma unroll
@@ -200,13 +227,13 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float&
       const int j = j0 + 2 * i + h;
       float delta, r;
       softplus_and_decay(dto[j0 / 2 + i] + cx.dtb, delta, r);
-      const float uu = __bfloat162float(su[j * CHP]);
+      const float uu = __bfloat162float(u_cur[i]);
       const bool valid = FULL || (j >= jlo && j < jhi);
       dec_o[i] = valid ? (POW ? r : delta) : (POW ? 1.0f : 0.0f);
       du_o[i] = valid ? delta * uu : 0.0f;
       if (FINAL) {
         Du_o[i] = cx.Dc * uu;
-        gz_o[i] = silu_fast(__bfloat162float(sz[j * CHP]));
+        gz_o[i] = silu_fast(__bfloat162float(z_cur[i]));
       } else {
         sumd += valid ? delta : 0.0f;
       }

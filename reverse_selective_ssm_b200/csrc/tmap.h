@@ -16,4 +16,10 @@ namespace r2l {
 bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, long long inner, long long rows,
                   long long ld_bytes, int box_inner, int box_rows, int swizzle_bytes);
 
+// The same matrix (rows even) seen as {inner, parity, rows / 2}: a box
+// {box_inner, 1, box_rows} at coordinates (x, p, i0) holds rows 2·(i0 + i) + p
+// for i = 0 .. box_rows − 1, i.e. every second row starting at 2·i0 + p.
+bool make_tmap_rows_by_parity(CUtensorMap* m, const void* base, int elem_bytes, long long inner, long long rows,
+                              long long ld_bytes, int box_inner, int box_rows, int swizzle_bytes);
+
 }  // namespace r2l
