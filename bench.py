@@ -78,7 +78,7 @@ STAGE_SOURCES = {
     "conv": ["conv_fast.cuh", "gemm_convx.cuh"] + _COMMON,
     "dt_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "out_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
-    "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh"] + _COMMON,
+    "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh", "scan_split.cuh"] + _COMMON,
     "ln_residual": ["simt_kernels.cuh"] + _COMMON,
     "scan_bwd": ["scan_bwd.cu", "scan_bwd.h"] + _COMMON,
 }
@@ -111,6 +111,63 @@ def read_traffic(stage, workload_tag):
             except ValueError:
                 return None
     return None
+
+
+def read_profile_value(stage, workload_tag, key):
+    """A numeric field of the committed ncu summary of one stage, if it was
+    taken on the current kernel sources (else None)."""
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
+        kv = {}
+        for line in open(f):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("stage") == stage and kv.get("workload") == workload_tag and \
+                kv.get("source_sha") == source_sha(stage) and key in kv:
+            try:
+                return float(kv[key].split()[0])
+            except ValueError:
+                return None
+    return None
+
+
+# FP32 operations per (token, channel) that the scan's arithmetic needs, on the
+# FMA pipe: the 16 decays r, r², …, r¹⁶ (15 products), Δu·B (16), the state
+# update (16 FMAs) and ⟨C, H⟩ (16 FMAs and a final add) for the 16 states, plus
+# softplus (4), Δu and D·u (2), SiLU(z) (3) and the gate (2).
+SCAN_FP32_OPS_PER_TOKEN_CHANNEL = 15 + 16 + 16 + 17 + 4 + 2 + 3 + 2
+B200_SMS = 148
+
+
+def scan_ceilings(case, ms, clocks, workload_tag):
+    """The scan against the two ceilings that bind before HBM does: the FP32
+    pipe (128 lane-operations per clock per SM, all 148 SMs) on the
+    arithmetic the recurrence needs, and instruction issue (one warp
+    instruction per clock per scheduler) on the instructions the kernel
+    executes (ncu, committed summary).  Both at the median SM clock sampled
+    during the timed region (the maximum if none was sampled)."""
+    T, E = case.valid_tokens, case.dims.d_inner
+    mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz") or 1965.0
+    f = mhz * 1e6
+    sec = ms * 1e-3
+    ops = SCAN_FP32_OPS_PER_TOKEN_CHANNEL * float(T) * E
+    fp32_peak = B200_SMS * 128 * f
+    out = {"clock_mhz": mhz,
+           "fp32_pipe": {"ops_per_token_channel": SCAN_FP32_OPS_PER_TOKEN_CHANNEL,
+                         "achieved_tops": round(ops / sec / 1e12, 3), "peak_tops": round(fp32_peak / 1e12, 3),
+                         "frac": round(ops / sec / fp32_peak, 4),
+                         "ceiling_ms": round(ops / fp32_peak * 1e3, 4)}}
+    inst = read_profile_value("scan", workload_tag, "inst_per_token_channel")
+    if inst is not None:
+        warp_inst = inst * T * E / 32.0
+        ceiling = warp_inst / (B200_SMS * 4 * f)
+        out["issue"] = {"inst_per_token_channel": inst, "ceiling_ms": round(ceiling * 1e3, 4),
+                        "frac": round(ceiling / sec, 4),
+                        "source": "smsp__inst_executed of the committed ncu summary (profiles/)"}
+    fma = read_profile_value("scan", workload_tag, "fma_pipe_active_frac")
+    if fma is not None:
+        out["fp32_pipe"]["ncu_fma_pipe_active_frac"] = fma
+    return out
 
 
 class ClockSampler:
@@ -418,6 +475,31 @@ def run_ours(args, rank, world, local_rank):
 
     ms_total = max_over_ranks(ms_total, world, dev)
 
+    # ---- the general-A path: the same step with R2L_FLAG_GENERAL_A, timed on
+    # its own (A_log of a trained model is not the S4D-real initialisation)
+    general = None
+    if not args.general_a:
+        gdims = bd.dims_of(case.dims, case.dtype, bd.R2L_FLAG_GENERAL_A)
+        gev = [[[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(hooks)]
+               for _ in range(K)]
+        for k in range(max(2, args.warmup // 2)):
+            for hk in range(hooks):
+                bd.sidecar_forward(h, wdev[hk], gdims, case.s[hk], lengths, ws, stream)
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for k in range(K):
+            for hk in range(hooks):
+                bd.sidecar_forward_profiled(h, wdev[hk], gdims, case.s[hk], gev[k][hk], lengths, ws, stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        g_total = max_over_ranks(g0.elapsed_time(g1), world, dev)
+        si = bd.STAGES.index("scan")
+        g_scan = sum(gev[k][hk][si].elapsed_time(gev[k][hk][si + 1]) for k in range(K) for hk in range(hooks))
+        general = {"ms_per_step": g_total / K, "scan_ms_per_launch": g_scan / (K * hooks)}
+
     # ---- end to end through host buffers
     e2e = None
     if not args.no_e2e:
@@ -453,8 +535,15 @@ def run_ours(args, rank, world, local_rank):
                    "scan_path": "general-A" if args.general_a else "auto (power fast path when A=-(1..16))"},
         "roofline": roofline_kernel(case, dom, per_launch, peaks, peak_kind, workload_tag,
                                     tensor_peak(peaks, peak_kind, clk, ms_total)),
-        "roofline_scan": roofline_obj(case, "scan", per_launch["scan"], peaks, peak_kind, workload_tag),
+        "roofline_scan": dict(roofline_obj(case, "scan", per_launch["scan"], peaks, peak_kind, workload_tag),
+                              path="general-A" if args.general_a else "power (A = -(1..16), exact per-call check)",
+                              ceilings=scan_ceilings(case, per_launch["scan"], clk, workload_tag)),
         "stage_ms": {s: round(v, 5) for s, v in per_launch.items()},
+        "roofline_scan_general": None if general is None else dict(
+            roofline_obj(case, "scan", general["scan_ms_per_launch"], peaks, peak_kind, workload_tag),
+            path="general-A (R2L_FLAG_GENERAL_A: one exponential per state)",
+            ms_per_step=round(general["ms_per_step"], 4), traffic=None,
+            tokens_per_s=round(whole_job_rate(case.valid_tokens, world, 1, general["ms_per_step"]), 1)),
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,

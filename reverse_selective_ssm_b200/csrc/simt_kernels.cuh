@@ -44,15 +44,23 @@ __global__ void __launch_bounds__(1024)
 a_log_check_kernel(const float* __restrict__ A_log, int E, const __grid_constant__ LnTable tab,
                    unsigned* __restrict__ general) {
   // A_log is [E, 16] and 16-byte aligned: thread t reads uint4 number t +
-  // 1024·k, whose four entries are states 4·(t mod 4) … 4·(t mod 4) + 3
+  // 1024·k, whose four entries are states 4·(t mod 4) … 4·(t mod 4) + 3;
+  // eight independent loads per thread are in flight at a time
   const uint4* a4 = reinterpret_cast<const uint4*>(A_log);
   const int m0 = (threadIdx.x & 3) * 4;
   const uint32_t t0 = tab.bits[m0], t1 = tab.bits[m0 + 1], t2 = tab.bits[m0 + 2], t3 = tab.bits[m0 + 3];
   const int n4 = E * 4;
+  constexpr int U = 8;                 // loads in flight per thread
   int bad = 0;
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-    const uint4 v = a4[i];
-    bad |= (v.x != t0) | (v.y != t1) | (v.z != t2) | (v.w != t3);
+  for (int base = threadIdx.x; base < n4; base += U * blockDim.x) {
+    uint4 v[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int i = base + k * blockDim.x;
+      v[k] = i < n4 ? a4[i] : make_uint4(t0, t1, t2, t3);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) bad |= (v[k].x != t0) | (v[k].y != t1) | (v[k].z != t2) | (v[k].w != t3);
   }
   bad = __syncthreads_or(bad);
   if (threadIdx.x == 0) *general = bad ? 1u : 0u;

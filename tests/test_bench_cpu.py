@@ -6,6 +6,7 @@ import io
 import json
 
 import bench
+import pytest
 
 
 def _run(argv, env=None, monkeypatch=None):
@@ -78,3 +79,17 @@ def test_tensor_peak_follows_the_clock_record():
     assert p == 1370.0
     p, _ = bench.tensor_peak(peaks, "measured", None, 40.0)
     assert p == 1370.0
+
+
+def test_scan_ceilings_arithmetic():
+    """The FP32-pipe ceiling of the scan: 75 operations per (token,
+    channel) on 148 SMs x 128 lanes per clock; at 1965 MHz and the serving
+    shape (32768 tokens x 4096 channels) that is 0.2704 ms."""
+    from reverse_selective_ssm_b200 import synthetic as S
+    case = S.make_case(2, weights=False, B=8, L=8)      # only the dims and the token count are read
+    case.B, case.L, case.lengths = 8, 4096, None
+    out = bench.scan_ceilings(case, 0.6436, {"sm_mhz": 1965.0}, "none")
+    assert bench.SCAN_FP32_OPS_PER_TOKEN_CHANNEL == 75
+    assert out["fp32_pipe"]["ceiling_ms"] == pytest.approx(75 * 32768 * 4096 / (148 * 128 * 1965e6) * 1e3, rel=1e-3)
+    assert out["fp32_pipe"]["frac"] == pytest.approx(out["fp32_pipe"]["ceiling_ms"] / 0.6436, rel=1e-3)
+    assert "issue" not in out                             # no committed summary for this workload tag
