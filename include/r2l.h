@@ -284,8 +284,8 @@ R2L_API size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims *dims, in
  * plus dy [B·L, E].  Every reduction runs in a fixed order: the results are
  * bitwise reproducible for a given chunk_tokens.
  *
- * Supported: dims->dtype == R2L_FP32 (every activation array is fp32),
- * d_state == 16, d_inner a multiple of 64, B and L up to 65535 with
+ * Supported: dims->dtype R2L_FP32 (every array fp32) or R2L_BF16 (u and z
+ * bf16 as the bf16 forward stores them, every other array fp32), d_state == 16, d_inner a multiple of 64, B and L up to 65535 with
  * B·⌈L / chunk⌉ ≤ 2,097,120 (grid limits), the right-to-left block (the
  * R2L_FLAG_FORWARD_SCAN flag returns R2L_ERR_UNSUPPORTED); ldz, ld_dz and
  * ldbc multiples of 4.  chunk_tokens: positions per chunk (1 … 32; larger values are
@@ -300,6 +300,50 @@ R2L_API r2l_status r2l_reverse_scan_backward(const void *u, const void *z, int l
                                              float *ddt_b, const r2l_dims *dims, int B, int L,
                                              const int32_t *lengths, int chunk_tokens, void *workspace,
                                              size_t workspace_bytes, void *stream);
+
+/* Gradients of one hook's parameters: fp32 device arrays, 16-byte aligned,
+ * caller-owned, each shaped like the matching field of r2l_weights (in_proj_w
+ * [2E, d], conv_w [E, W], conv_b [E], x_proj_w [R+2N, E], dt_proj_w [E, R],
+ * dt_proj_b [E], A_log [E, N], D [E], out_proj_w [d, E], ln_w and ln_b [d]).
+ * ln_w / ln_b may be NULL when the hook has no LayerNorm.  Every array is
+ * written in full (not accumulated into).                                    */
+typedef struct {
+  float *in_proj_w, *conv_w, *conv_b, *x_proj_w, *dt_proj_w, *dt_proj_b, *A_log, *D, *out_proj_w, *ln_w, *ln_b;
+} r2l_grads;
+
+/* Bytes of device workspace r2l_sidecar_backward needs for a [B, L] batch;
+ * 0 for invalid or unsupported input.                                        */
+R2L_API size_t r2l_sidecar_backward_workspace_size(const r2l_dims *dims, int B, int L);
+
+/* The gradient of one hook (§3.4 steps ❶–❹), the step that training the
+ * sidecar alone (the paper's R2LM-PI setting, §3.4 and §4.1) back-propagates
+ * through.  For the hook's input hidden [B, L, d] (act dtype, as given to
+ * r2l_sidecar_forward) and dh_out = ∂L/∂h⁺ (fp32 [B, L, d]) it writes
+ *
+ *   dh    fp32 [B, L, d]  ∂L/∂h: dh_out on padding rows (the hook neither reads
+ *                          nor writes them), dh_out + ∂L/∂h through the sidecar
+ *                          on valid rows
+ *   *ds   fp32 scalar     ∂L/∂s = (1 − tanh²(s)) Σ dh_out ⊙ ĥ (device pointer)
+ *   grads                 ∂L/∂(every parameter), summed over the batch
+ *
+ * The forward is recomputed into the workspace, then the chain rule runs in
+ * reverse: gate, LayerNorm, out_proj, the scan (bf16 u and z, fp32 state),
+ * dt_proj, x_proj, conv + SiLU, in_proj.  GEMM operands are bf16 (gradients
+ * rounded once to bf16 where they feed a GEMM), accumulation fp32; every
+ * reduction over positions runs in a fixed order, so results are bitwise
+ * reproducible.
+ *
+ * Supported: dims->dtype R2L_BF16, d_state 16, d_conv 4, d_model and dt_rank
+ * multiples of 8, d_inner a multiple of 64, the right-to-left block
+ * (R2L_FLAG_FORWARD_SCAN returns R2L_ERR_UNSUPPORTED).  workspace ≥
+ * r2l_sidecar_backward_workspace_size(dims, B, L) bytes, 16-byte aligned; its
+ * first 16 bytes are the status word r2l_get_device_status reads.  Other
+ * arguments, conventions and errors as r2l_sidecar_forward; hidden is not
+ * written.                                                                     */
+R2L_API r2l_status r2l_sidecar_backward(const void *hidden, const r2l_weights *weights, const r2l_dims *dims,
+                                        float s, int B, int L, const int32_t *lengths, const float *dh_out,
+                                        float *dh, float *ds, const r2l_grads *grads, void *workspace,
+                                        size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream`, then reads the device status word that the last
  * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*

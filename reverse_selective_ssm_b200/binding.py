@@ -28,7 +28,7 @@ EXPORTS = ("r2l_abi_version", "r2l_status_string", "r2l_workspace_size", "r2l_si
            "r2l_sidecar_forward_debug", "r2l_sidecar_forward_profiled", "r2l_sidecar_stack",
            "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan",
            "r2l_reverse_scan_noalloc", "r2l_reverse_scan_backward_workspace_size",
-           "r2l_reverse_scan_backward")
+           "r2l_reverse_scan_backward", "r2l_sidecar_backward_workspace_size", "r2l_sidecar_backward")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -49,6 +49,13 @@ class Dims(ctypes.Structure):
 
 
 class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "in_proj_w", "conv_w", "conv_b", "x_proj_w", "dt_proj_w", "dt_proj_b", "A_log", "D",
+        "out_proj_w", "ln_w", "ln_b")]
+
+
+class Grads(ctypes.Structure):
+    """r2l_grads: fp32 device arrays shaped like the weights."""
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "in_proj_w", "conv_w", "conv_b", "x_proj_w", "dt_proj_w", "dt_proj_b", "A_log", "D",
         "out_proj_w", "ln_w", "ln_b")]
@@ -105,6 +112,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.r2l_reverse_scan_backward.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, vp, vp, vp, vp, ci, vp, vp, ci,
                                               vp, vp, vp, ctypes.POINTER(Dims), ci, ci, vp, ci, vp,
                                               ctypes.c_size_t, vp]
+    lib.r2l_sidecar_backward_workspace_size.restype = ctypes.c_size_t
+    lib.r2l_sidecar_backward_workspace_size.argtypes = [ctypes.POINTER(Dims), ci, ci]
+    lib.r2l_sidecar_backward.restype = ci
+    lib.r2l_sidecar_backward.argtypes = [vp, ctypes.POINTER(Weights), ctypes.POINTER(Dims), cf, ci, ci, vp, vp, vp,
+                                         vp, ctypes.POINTER(Grads), vp, ctypes.c_size_t, vp]
     lib.r2l_get_device_status.restype = ci
     lib.r2l_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -306,3 +318,43 @@ def get_device_status(workspace: torch.Tensor, stream=None):
 
 def weights_to_device(w: Dict[str, Optional[torch.Tensor]], device="cuda"):
     return {k: (None if v is None else v.to(device).contiguous()) for k, v in w.items()}
+
+
+# weight-dict key -> r2l_grads field, as for the weights
+GRAD_KEYS = tuple(k for k, _ in _WMAP)
+
+
+def sidecar_backward_workspace_size(dims: Dims, B: int, L: int) -> int:
+    return int(load().r2l_sidecar_backward_workspace_size(ctypes.byref(dims), B, L))
+
+
+def alloc_grads(weights: Dict[str, Optional[torch.Tensor]], device="cuda") -> Dict[str, Optional[torch.Tensor]]:
+    """fp32 gradient buffers shaped like a hook's weights (None where the
+    weight is None)."""
+    return {k: None if v is None else torch.empty(v.shape, dtype=torch.float32, device=device)
+            for k, v in weights.items()}
+
+
+def sidecar_backward(hidden: torch.Tensor, weights, dims: Dims, s: float, dh_out: torch.Tensor,
+                     grads: Dict[str, Optional[torch.Tensor]], lengths=None, workspace: Optional[torch.Tensor] = None,
+                     stream=None, check: bool = True):
+    """r2l_sidecar_backward: returns (dh [B, L, d] fp32, ds (a 1-element fp32
+    device tensor)); grads (from alloc_grads) receives every parameter's
+    gradient."""
+    lib = load()
+    B, L = hidden.shape[0], hidden.shape[1]
+    if workspace is None:
+        workspace = torch.empty(max(sidecar_backward_workspace_size(dims, B, L), 16), dtype=torch.uint8,
+                                device=hidden.device)
+    w = weights if isinstance(weights, Weights) else weights_struct(weights)
+    g = Grads()
+    for key, field in _WMAP:
+        setattr(g, field, _ptr(grads.get(key)))
+    dh = torch.empty(dh_out.shape, dtype=torch.float32, device=hidden.device)
+    ds = torch.zeros(4, dtype=torch.float32, device=hidden.device)
+    st = lib.r2l_sidecar_backward(_ptr(hidden), ctypes.byref(w), ctypes.byref(dims), float(s), B, L, _ptr(lengths),
+                                  _ptr(dh_out), _ptr(dh), _ptr(ds), ctypes.byref(g), _ptr(workspace),
+                                  workspace.numel(), _stream_ptr(stream))
+    if check and st != 0:
+        raise R2LError(st, "r2l_sidecar_backward")
+    return dh, ds[:1]

@@ -18,12 +18,14 @@
 #include "scan_fast.h"
 #include "scan_bwd.h"
 #include "conv_fast.cuh"
+#include "bwd_kernels.cuh"
 
 // conv + SiLU fused into the x_proj GEMM on the bf16 path (0: separate kernels).
 #ifndef R2L_CONVX
 #define R2L_CONVX 1
 #endif
 
+#include <algorithm>
 #include <type_traits>
 
 using r2l::bf16;
@@ -227,7 +229,7 @@ r2l_status launch_ln_bf16(int nv, bool has_ln, unsigned blocks, cudaStream_t st,
 
 template <typename T>
 r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, int B, int L,
-                     char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof) {
+                     char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof, bool residual = true) {
   Prof dummy;
   if (!prof) prof = &dummy;
   const long long M = p.M;
@@ -343,6 +345,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     if (dbg->y && cudaMemcpyAsync(dbg->y, y, rowsE * E * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
     if (dbg->o && cudaMemcpyAsync(dbg->o, o, rowsE * d * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
   }
+  // stop here when only the intermediates are wanted (the hook's gradient)
+  if (!residual) return R2L_OK;
   // a7 + a8: LayerNorm (optional) and h += g · ĥ on valid rows
   float* hhat = dbg ? dbg->hhat : nullptr;
   R2L_TRY(prof->mark(R2L_STAGE_LN_RESIDUAL, st));
@@ -530,7 +534,7 @@ r2l_status r2l_reverse_scan(const void* u, const void* z, int ldz, const void* d
 
 size_t r2l_reverse_scan_backward_workspace_size(const r2l_dims* dims, int B, int L, int chunk_tokens) {
   if (!dims || B <= 0 || L <= 0 || dims->d_inner <= 0 || chunk_tokens < 0) return 0;
-  if (dims->dtype != R2L_FP32 || dims->d_state != 16 || dims->d_inner % 64) return 0;
+  if ((dims->dtype != R2L_FP32 && dims->dtype != R2L_BF16) || dims->d_state != 16 || dims->d_inner % 64) return 0;
   if (!r2l::scan_bwd_supported(B, L, dims->d_inner, chunk_tokens)) return 0;
   return align_up(16, kAlign) + align_up(r2l::scan_bwd_scratch_bytes(B, L, dims->d_inner, chunk_tokens), kAlign);
 }
@@ -546,8 +550,8 @@ r2l_status r2l_reverse_scan_backward(const void* u, const void* z, int ldz, cons
     return R2L_ERR_INVALID_ARG;
   if (B <= 0 || L <= 0 || dims->d_inner <= 0 || chunk_tokens < 0) return R2L_ERR_INVALID_ARG;
   if (dims->dtype != R2L_BF16 && dims->dtype != R2L_FP32) return R2L_ERR_INVALID_ARG;
-  if (dims->dtype != R2L_FP32 || dims->d_state != 16 || (dims->flags & R2L_FLAG_FORWARD_SCAN))
-    return R2L_ERR_UNSUPPORTED;
+  if (dims->d_state != 16 || (dims->flags & R2L_FLAG_FORWARD_SCAN)) return R2L_ERR_UNSUPPORTED;
+  const bool act16 = dims->dtype == R2L_BF16;   // u and z in bf16, everything else fp32
   const int E = dims->d_inner;
   if (E % 64) return R2L_ERR_UNSUPPORTED;
   if (ldz < E || ld_dz < E || ldbc < 32 || ld_dbc < 32) return R2L_ERR_INVALID_ARG;
@@ -565,7 +569,9 @@ r2l_status r2l_reverse_scan_backward(const void* u, const void* z, int ldz, cons
   char* ws = (char*)workspace;
   if (cudaMemsetAsync(ws, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
   r2l::ScanBwdArgs a{};
-  a.u = (const float*)u; a.z = (const float*)z; a.ldz = ldz; a.dt_raw = (const float*)dt_raw;
+  a.u = act16 ? nullptr : (const float*)u; a.z = act16 ? nullptr : (const float*)z;
+  a.u16 = act16 ? (const bf16*)u : nullptr; a.z16 = act16 ? (const bf16*)z : nullptr;
+  a.ldz = ldz; a.dt_raw = (const float*)dt_raw;
   a.bc = bc; a.ldbc = ldbc; a.A_log = A_log; a.D = D; a.dt_b = dt_b; a.dy = (const float*)dy;
   a.du = (float*)du; a.dz = (float*)dz; a.ld_dz = ld_dz; a.ddt_raw = (float*)ddt_raw;
   a.dbc = dbc; a.ld_dbc = ld_dbc; a.dA_log = dA_log; a.dD = dD; a.ddt_b = ddt_b;
@@ -584,6 +590,311 @@ r2l_status r2l_get_device_status(const void* workspace, void* stream, uint32_t* 
   if (cudaMemcpy(&f, workspace, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess) return R2L_ERR_CUDA;
   *flags_out = f;
   return f ? R2L_ERR_DEVICE_CHECK : R2L_OK;
+}
+
+}  // extern "C"
+
+// ============================================================================
+// The gradient of one hook (r2l_sidecar_backward).  The forward is recomputed
+// into the workspace (as r2l_sidecar_forward computes it, without the final
+// residual), then the chain rule runs in reverse: gate and LayerNorm, out_proj,
+// the scan, dt_proj, x_proj, conv + SiLU, in_proj.  Input gradients are
+// tcgen05 GEMMs against transposed weights; weight gradients are tcgen05 GEMMs
+// of transposed (position-major) activations, with padding positions zeroed so
+// that they contribute nothing.
+// ============================================================================
+namespace {
+
+struct BwdPlan {
+  Plan f;                                        // the forward's regions
+  long long Mp;                                  // positions rounded up to 8 (K of the weight gradients)
+  size_t dt32, winT, woutT, wxT, wdtT, stats, dsrow, do16, lnpart, dy, doT, yT, dus, dz, ddt, dbcs, sbwd, sbwd_bytes,
+      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, dpre, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, total;
+};
+
+long long row_chunks(long long M) { return (M + r2l::bwd::ROW_CHUNK - 1) / r2l::bwd::ROW_CHUNK; }
+
+bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
+  if (!make_plan(dm, B, L, &q->f)) return false;
+  const Plan& p = q->f;
+  const size_t M = (size_t)p.M, E = p.E, d = p.d, R = p.R, N2 = 2 * p.N, ldd = p.ldd;
+  q->Mp = (p.M + 7) / 8 * 8;
+  const size_t Mp = (size_t)q->Mp;
+  size_t off = p.total;
+  auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, kAlign); return at; };
+  q->dt32 = take(M * E * 4);
+  q->winT = take(d * 2 * E * 2);
+  q->woutT = take(E * d * 2);
+  q->wxT = take(E * ldd * 2);
+  q->wdtT = take(R * E * 2);
+  q->stats = take(M * 8);
+  q->dsrow = take(M * 4);
+  q->do16 = take(M * d * 2);
+  q->lnpart = take((size_t)row_chunks(p.M) * 2 * d * 4);
+  q->dy = take(M * E * 4);
+  q->doT = take(d * Mp * 2);
+  q->yT = take(E * Mp * 2);
+  q->dus = take(M * E * 4);
+  q->dz = take(M * E * 4);
+  q->ddt = take(M * E * 4);
+  q->dbcs = take(M * N2 * 4);
+  r2l_dims sd = *dm;
+  sd.dtype = R2L_BF16;
+  q->sbwd_bytes = r2l_reverse_scan_backward_workspace_size(&sd, B, L, 0);
+  if (q->sbwd_bytes == 0) return false;
+  q->sbwd = take(q->sbwd_bytes);
+  q->ddt16 = take(M * E * 2);
+  q->ddtT = take(E * Mp * 2);
+  q->drT = take(R * Mp * 2);
+  q->ddr = take(M * R * 4);
+  q->ddbc16 = take(M * ldd * 2);
+  q->ddbcT = take(ldd * Mp * 2);
+  q->uT = take(E * Mp * 2);
+  q->dux = take(M * E * 4);
+  q->dpre = take(M * E * 4);
+  q->cpart = take((size_t)row_chunks(p.M) * 5 * E * 4);
+  q->dxz16 = take(M * 2 * E * 2);
+  q->dxzT = take(2 * E * Mp * 2);
+  q->hT = take(d * Mp * 2);
+  q->dhtmp = take(M * d * 4);
+  // split-K scratch: the largest any fp32-output GEMM below asks for
+  size_t gp = 0;
+  auto need = [&](long long m, int n, int k) { gp = std::max(gp, r2l::tc_gemm_partial_bytes(m, n, k)); };
+  need(p.M, p.E, p.R);                 // dt_raw
+  need(p.M, p.E, p.d);                 // dy
+  need(p.d, p.E, (int)q->Mp);          // dW_out
+  need(p.M, p.R, p.E);                 // dΔr
+  need(p.E, p.R, (int)q->Mp);          // dW_dt
+  need(p.M, p.E, p.ldd);               // du_x
+  need(p.ldd, p.E, (int)q->Mp);        // dW_x
+  need(p.M, p.d, 2 * p.E);             // dh
+  need(2LL * p.E, p.d, (int)q->Mp);    // dW_in
+  q->gpart_bytes = gp;
+  q->gpart = take(gp);
+  q->total = off;
+  return true;
+}
+
+int grid_for(long long n, int threads) {
+  long long b = (n + threads - 1) / threads;
+  return (int)(b < 148 * 16 ? (b > 0 ? b : 1) : 148 * 16);
+}
+
+// out[c, m] = bf16(in[m, c]) over M rows (ld_out = Mp), padding rows zeroed.
+template <typename TIn>
+r2l_status transpose(const TIn* in, long long ld_in, long long M, int C, bf16* out, long long ld_out, const int* len,
+                     int L, cudaStream_t st) {
+  if (M <= 0 || C <= 0) return R2L_OK;
+  const dim3 grid((unsigned)((C + 31) / 32), (unsigned)((ld_out + 31) / 32));
+  r2l::bwd::transpose_bf16_kernel<TIn><<<grid, 256, 0, st>>>(in, ld_in, (int)M, C, out, ld_out, len, L);
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+// C[m, n] = Σ_k A[m, k]·B[n, k], bf16 operands, fp32 result.
+r2l_status gemm_f32(const bf16* A, int lda, const bf16* Bm, int ldb, float* C, int ldc, long long M, int N, int K,
+                    const int* len, int L, unsigned* err, float* partial, size_t partial_bytes, cudaStream_t st) {
+  r2l::TcGemm g{};
+  g.A = A; g.lda = lda; g.B = Bm; g.ldb = ldb; g.C = C; g.ldc = ldc; g.c_fp32 = true;
+  g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
+  g.partial = partial; g.partial_bytes = partial_bytes;
+  return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
+}
+
+r2l_status check_grads(const r2l_grads* gr, const r2l_weights* w) {
+  if (!gr) return R2L_ERR_INVALID_ARG;
+  const void* ptrs[] = {gr->in_proj_w, gr->conv_w, gr->conv_b, gr->x_proj_w, gr->dt_proj_w,
+                        gr->dt_proj_b, gr->A_log, gr->D, gr->out_proj_w};
+  for (const void* q : ptrs) {
+    if (!q) return R2L_ERR_INVALID_ARG;
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  }
+  if (w->ln_w && (!gr->ln_w || !gr->ln_b)) return R2L_ERR_INVALID_ARG;
+  if (gr->ln_w && (!aligned16(gr->ln_w) || !aligned16(gr->ln_b))) return R2L_ERR_ALIGNMENT;
+  return R2L_OK;
+}
+
+r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dims* dims, float s, int B, int L,
+                         const int32_t* lengths, const float* dh_out, float* dh, float* ds, const r2l_grads* gr,
+                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  namespace K = r2l::bwd;
+  BwdPlan q;
+  if (!make_bwd_plan(dims, B, L, &q)) return R2L_ERR_INVALID_ARG;
+  const Plan& p = q.f;
+  char* ws = (char*)workspace;
+  const long long M = p.M, Mp = q.Mp;
+  const int E = p.E, d = p.d, R = p.R, ldd = p.ldd;
+  const int* len = (const int*)(ws + p.len);
+  unsigned* err = (unsigned*)(ws + p.status);
+  float* gpart = (float*)(ws + q.gpart);
+  const size_t gpb = q.gpart_bytes;
+  const double gd = std::tanh((double)s);
+  const float g = (float)gd;
+  const float dgate = (float)(1.0 - gd * gd);   // d tanh(s) / ds
+
+  // ---- the forward's intermediates: xz, u, Δr|B|C, Δr (bf16), y, o; dt_raw in fp32
+  R2L_TRY(prep(p, ws, lengths, B, L, st));
+  // run_layer with residual = false reads hidden and writes nothing to it
+  R2L_TRY(run_layer<bf16>((bf16*)const_cast<void*>(hidden), w, p, g, B, L, ws, st, nullptr, nullptr, false));
+  const bf16* xz = (const bf16*)(ws + p.xz);
+  const bf16* u = (const bf16*)(ws + p.u);
+  const float* dbc = (const float*)(ws + p.dbc);
+  const bf16* dr = (const bf16*)(ws + p.dr);
+  const bf16* y = (const bf16*)(ws + p.y);
+  const bf16* o = (const bf16*)(ws + p.o);
+  float* dt32 = (float*)(ws + q.dt32);
+  R2L_TRY(gemm_f32(dr, R, (const bf16*)w->dt_proj_w, R, dt32, E, M, E, R, len, L, err, gpart, gpb, st));
+
+  // ---- weights transposed once: W_outᵀ [E, d], W_dtᵀ [R, E], W_xᵀ [E, R+2N], W_inᵀ [d, 2E]
+  bf16* woutT = (bf16*)(ws + q.woutT);
+  bf16* wdtT = (bf16*)(ws + q.wdtT);
+  bf16* wxT = (bf16*)(ws + q.wxT);
+  bf16* winT = (bf16*)(ws + q.winT);
+  R2L_TRY(transpose((const bf16*)w->out_proj_w, E, d, E, woutT, d, nullptr, d, st));
+  R2L_TRY(transpose((const bf16*)w->dt_proj_w, R, E, R, wdtT, E, nullptr, E, st));
+  R2L_TRY(transpose((const bf16*)w->x_proj_w, E, ldd, E, wxT, ldd, nullptr, ldd, st));
+  R2L_TRY(transpose((const bf16*)w->in_proj_w, d, 2LL * E, d, winT, 2LL * E, nullptr, 2 * E, st));
+
+  // ---- ❹ gate and ❸ LayerNorm
+  float2* stats = (float2*)(ws + q.stats);
+  float* dsrow = (float*)(ws + q.dsrow);
+  bf16* do16 = (bf16*)(ws + q.do16);
+  const bool has_ln = w->ln_w != nullptr;
+  const unsigned rblocks = (unsigned)((M + 7) / 8);
+  if (has_ln)
+    K::ln_gate_bwd_rows_kernel<true><<<rblocks, 256, 0, st>>>(o, dh_out, w->ln_w, w->ln_b, g, d, len, L, M, stats,
+                                                              dsrow, do16);
+  else
+    K::ln_gate_bwd_rows_kernel<false><<<rblocks, 256, 0, st>>>(o, dh_out, nullptr, nullptr, g, d, len, L, M, stats,
+                                                               dsrow, do16);
+  R2L_LAUNCH_CHECK();
+  K::sum_kernel<<<1, 1024, 0, st>>>(dsrow, M, dgate, ds);
+  R2L_LAUNCH_CHECK();
+  const long long nrc = row_chunks(M);
+  if (has_ln) {
+    float* lnpart = (float*)(ws + q.lnpart);
+    K::ln_bwd_cols_kernel<<<dim3((unsigned)((d + 127) / 128), (unsigned)nrc), 128, 0, st>>>(o, dh_out, g, d, len, L,
+                                                                                            M, stats, lnpart);
+    R2L_LAUNCH_CHECK();
+    K::colsum_kernel<<<(d + 255) / 256, 256, 0, st>>>(lnpart, (int)nrc, 2LL * d, d, 1.0f, gr->ln_w);
+    K::colsum_kernel<<<(d + 255) / 256, 256, 0, st>>>(lnpart + d, (int)nrc, 2LL * d, d, 1.0f, gr->ln_b);
+    R2L_LAUNCH_CHECK();
+  }
+
+  // ---- out_proj: dy = do·W_out, dW_out = doᵀ·y
+  float* dy = (float*)(ws + q.dy);
+  R2L_TRY(gemm_f32(do16, d, woutT, d, dy, E, M, E, d, len, L, err, gpart, gpb, st));
+  bf16* doT = (bf16*)(ws + q.doT);
+  bf16* yT = (bf16*)(ws + q.yT);
+  R2L_TRY(transpose(do16, d, M, d, doT, Mp, len, L, st));
+  R2L_TRY(transpose(y, E, M, E, yT, Mp, len, L, st));
+  R2L_TRY(gemm_f32(doT, (int)Mp, yT, (int)Mp, gr->out_proj_w, E, d, E, (int)Mp, nullptr, d, err, gpart, gpb, st));
+
+  // ---- ❷ the scan (bf16 u and z, fp32 dt_raw, B|C and dy)
+  float* dus = (float*)(ws + q.dus);
+  float* dz = (float*)(ws + q.dz);
+  float* ddt = (float*)(ws + q.ddt);
+  float* dbcs = (float*)(ws + q.dbcs);
+  {
+    r2l::ScanBwdArgs a{};
+    a.u16 = u; a.z16 = xz + E; a.ldz = 2 * E; a.dt_raw = dt32; a.bc = dbc + R; a.ldbc = ldd;
+    a.A_log = w->A_log; a.D = w->D; a.dt_b = w->dt_proj_b; a.dy = dy;
+    a.du = dus; a.dz = dz; a.ld_dz = E; a.ddt_raw = ddt; a.dbc = dbcs; a.ld_dbc = 2 * p.N;
+    a.dA_log = gr->A_log; a.dD = gr->D; a.ddt_b = gr->dt_proj_b;
+    a.B = B; a.L = L; a.E = E; a.chunk_tokens = 0; a.lengths = len;
+    a.status = err;
+    char* sw = ws + q.sbwd;
+    if (cudaMemsetAsync(sw, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (r2l::scan_bwd_f32(a, sw + align_up(16, kAlign), st) != cudaSuccess) return R2L_ERR_CUDA;
+  }
+
+  // ---- dt_proj: dΔr = ddt_raw·W_dt, dW_dt = ddt_rawᵀ·Δr
+  bf16* ddt16 = (bf16*)(ws + q.ddt16);
+  K::to_bf16_rows_kernel<float><<<grid_for(M * E, 256), 256, 0, st>>>(ddt, E, (int)M, E, ddt16, E, len, L);
+  R2L_LAUNCH_CHECK();
+  float* ddr = (float*)(ws + q.ddr);
+  R2L_TRY(gemm_f32(ddt16, E, wdtT, E, ddr, R, M, R, E, len, L, err, gpart, gpb, st));
+  bf16* ddtT = (bf16*)(ws + q.ddtT);
+  bf16* drT = (bf16*)(ws + q.drT);
+  R2L_TRY(transpose(ddt16, E, M, E, ddtT, Mp, len, L, st));
+  R2L_TRY(transpose(dr, R, M, R, drT, Mp, len, L, st));
+  R2L_TRY(gemm_f32(ddtT, (int)Mp, drT, (int)Mp, gr->dt_proj_w, R, E, R, (int)Mp, nullptr, E, err, gpart, gpb, st));
+
+  // ---- x_proj: d[Δr|B|C] → du_x = d[Δr|B|C]·W_x, dW_x = d[Δr|B|C]ᵀ·u
+  bf16* ddbc16 = (bf16*)(ws + q.ddbc16);
+  K::to_bf16_rows_kernel<float><<<grid_for(M * R, 256), 256, 0, st>>>(ddr, R, (int)M, R, ddbc16, ldd, len, L);
+  K::to_bf16_rows_kernel<float><<<grid_for(M * 2 * p.N, 256), 256, 0, st>>>(dbcs, 2 * p.N, (int)M, 2 * p.N,
+                                                                           ddbc16 + R, ldd, len, L);
+  R2L_LAUNCH_CHECK();
+  float* dux = (float*)(ws + q.dux);
+  R2L_TRY(gemm_f32(ddbc16, ldd, wxT, ldd, dux, E, M, E, ldd, len, L, err, gpart, gpb, st));
+  bf16* ddbcT = (bf16*)(ws + q.ddbcT);
+  bf16* uT = (bf16*)(ws + q.uT);
+  R2L_TRY(transpose(ddbc16, ldd, M, ldd, ddbcT, Mp, len, L, st));
+  R2L_TRY(transpose(u, E, M, E, uT, Mp, len, L, st));
+  R2L_TRY(gemm_f32(ddbcT, (int)Mp, uT, (int)Mp, gr->x_proj_w, E, ldd, E, (int)Mp, nullptr, ldd, err, gpart, gpb,
+                   st));
+
+  // ---- conv + SiLU: dpre, dx (into dxz), dconv_w, dconv_b; dz into dxz
+  float* dpre = (float*)(ws + q.dpre);
+  bf16* dxz16 = (bf16*)(ws + q.dxz16);
+  K::conv_silu_bwd_pre_kernel<<<grid_for(M * E, 256), 256, 0, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E,
+                                                                   len, L, M, dpre);
+  R2L_LAUNCH_CHECK();
+  K::conv_bwd_dx_kernel<<<grid_for(M * E, 256), 256, 0, st>>>(dpre, w->conv_w, E, len, L, M, dxz16, 2LL * E);
+  K::to_bf16_rows_kernel<float><<<grid_for(M * E, 256), 256, 0, st>>>(dz, E, (int)M, E, dxz16 + E, 2LL * E, len, L);
+  float* cpart = (float*)(ws + q.cpart);
+  K::conv_bwd_params_kernel<<<dim3((unsigned)((E + 127) / 128), (unsigned)nrc), 128, 0, st>>>(dpre, xz, 2LL * E, E,
+                                                                                             len, L, M, cpart);
+  K::conv_bwd_reduce_kernel<<<(E + 127) / 128, 128, 0, st>>>(cpart, (int)nrc, E, gr->conv_w, gr->conv_b);
+  R2L_LAUNCH_CHECK();
+
+  // ---- in_proj: dh = dh⁺ + [dx | dz]·W_in, dW_in = [dx | dz]ᵀ·h
+  float* dhtmp = (float*)(ws + q.dhtmp);
+  R2L_TRY(gemm_f32(dxz16, 2 * E, winT, 2 * E, dhtmp, d, M, d, 2 * E, len, L, err, gpart, gpb, st));
+  K::add_rows_kernel<<<grid_for(M * d, 256), 256, 0, st>>>(dh_out, dhtmp, d, len, L, M, dh);
+  R2L_LAUNCH_CHECK();
+  bf16* dxzT = (bf16*)(ws + q.dxzT);
+  bf16* hT = (bf16*)(ws + q.hT);
+  R2L_TRY(transpose(dxz16, 2LL * E, M, 2 * E, dxzT, Mp, len, L, st));
+  R2L_TRY(transpose((const bf16*)hidden, d, M, d, hT, Mp, len, L, st));
+  R2L_TRY(gemm_f32(dxzT, (int)Mp, hT, (int)Mp, gr->in_proj_w, d, 2LL * E, d, (int)Mp, nullptr, 2 * E, err, gpart,
+                   gpb, st));
+  return R2L_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t r2l_sidecar_backward_workspace_size(const r2l_dims* dims, int B, int L) {
+  if (!dims || dims->dtype != R2L_BF16) return 0;
+  BwdPlan q;
+  if (!make_bwd_plan(dims, B, L, &q)) return 0;
+  return q.total;
+}
+
+r2l_status r2l_sidecar_backward(const void* hidden, const r2l_weights* weights, const r2l_dims* dims, float s, int B,
+                                int L, const int32_t* lengths, const float* dh_out, float* dh, float* ds,
+                                const r2l_grads* grads, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!hidden || !dims || !dh_out || !dh || !ds) return R2L_ERR_INVALID_ARG;
+  Plan p;
+  if (!make_plan(dims, B, L, &p)) return R2L_ERR_INVALID_ARG;
+  if (dims->d_state != 16 || dims->d_conv != 4) return R2L_ERR_UNSUPPORTED;
+  if (dims->dtype != R2L_BF16 || (dims->flags & R2L_FLAG_FORWARD_SCAN)) return R2L_ERR_UNSUPPORTED;
+  if ((dims->d_model % 8) || (dims->d_inner % 64) || (dims->dt_rank % 8)) return R2L_ERR_UNSUPPORTED;
+  if (L > 65535 || B > 65535 || (p.M + 63) / 64 > 65535) return R2L_ERR_UNSUPPORTED;
+  R2L_TRY(check_weights(weights));
+  R2L_TRY(check_grads(grads, weights));
+  for (const void* q : {hidden, (const void*)dh_out, (const void*)dh})
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  if (((uintptr_t)ds & 3u) || (lengths && ((uintptr_t)lengths & 3u))) return R2L_ERR_ALIGNMENT;
+  BwdPlan q;
+  if (!make_bwd_plan(dims, B, L, &q)) return R2L_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < q.total) return R2L_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return R2L_ERR_ALIGNMENT;
+  return backward_impl(hidden, weights, dims, s, B, L, lengths, dh_out, dh, ds, grads, workspace, workspace_bytes,
+                       (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -51,6 +51,8 @@ constexpr int WARPS = THREADS / 32;
 struct Args {
   const float* u;
   const float* z;
+  const bf16* u16;         // bf16 u and z instead (when not null)
+  const bf16* z16;
   int ldz;
   const float* dt;
   const float* bc;
@@ -107,6 +109,13 @@ __device__ __forceinline__ float exp2_mufu(float x) {
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+// four consecutive bf16 (8-byte aligned) widened to fp32
+__device__ __forceinline__ float4 ld4h(const bf16* p) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 __device__ __forceinline__ float get(const float4& v, int j) { return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w; }
 
@@ -206,9 +215,9 @@ __device__ __forceinline__ void stage_chunk(const Args& a, const Lane& l, const 
     const float4 dtb = ld4(a.dt_b + col);
     const float4 v4 = ld4(a.dt + row * a.E + col);
     float4 u4 = make_float4(0.f, 0.f, 0.f, 0.f), z4 = u4, dy4 = u4;
-    if (NEED_U) u4 = ld4(a.u + row * a.E + col);
+    if (NEED_U) u4 = a.u16 ? ld4h(a.u16 + row * a.E + col) : ld4(a.u + row * a.E + col);
     if (NEED_Z) {
-      z4 = ld4(a.z + row * a.ldz + col);
+      z4 = a.z16 ? ld4h(a.z16 + row * a.ldz + col) : ld4(a.z + row * a.ldz + col);
       dy4 = ld4(a.dy + row * a.E + col);
     }
     float o[NSTAGE][4];
@@ -615,7 +624,7 @@ size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens) {
 cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   using namespace sbwd;
   Args a{};
-  a.u = g.u; a.z = g.z; a.ldz = g.ldz; a.dt = g.dt_raw; a.bc = g.bc; a.ldbc = g.ldbc;
+  a.u = g.u; a.z = g.z; a.u16 = g.u16; a.z16 = g.z16; a.ldz = g.ldz; a.dt = g.dt_raw; a.bc = g.bc; a.ldbc = g.ldbc;
   a.A_log = g.A_log; a.D = g.D; a.dt_b = g.dt_b; a.dy = g.dy;
   a.du = g.du; a.dz = g.dz; a.ld_dz = g.ld_dz; a.ddt = g.ddt_raw; a.dbc = g.dbc; a.ld_dbc = g.ld_dbc;
   a.dA_log = g.dA_log; a.dD = g.dD; a.ddt_b = g.ddt_b;

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <cuda_bf16.h>
 
 namespace r2l {
 
@@ -10,6 +11,8 @@ constexpr int SCAN_BWD_MAX_CHUNK = 32;   // positions per chunk (shared memory: 
 
 struct ScanBwdArgs {
   const float *u, *z, *dt_raw, *bc, *A_log, *D, *dt_b, *dy;
+  // bf16 u and z (what the bf16 forward writes) in place of u and z when set
+  const __nv_bfloat16 *u16, *z16;
   int ldz, ldbc;
   float *du, *dz, *ddt_raw, *dbc, *dA_log, *dD, *ddt_b;
   int ld_dz, ld_dbc;

@@ -155,13 +155,12 @@ def test_scan_backward_argument_checks(lib):
     n = bd.reverse_scan_backward_workspace_size(f32, 2, 40, 0)
     assert n >= 3 * (2 * 3 * 128 * 16 * 4)              # three [B][chunks][E][16] fp32 arrays (T = 16: 3 chunks)
     assert bd.reverse_scan_backward_workspace_size(f32, 2, 40, 8) > n   # shorter chunks, more carries
-    assert bd.reverse_scan_backward_workspace_size(bd.make_dims(64, 128), 2, 40, 0) == 0      # bf16
+    assert bd.reverse_scan_backward_workspace_size(bd.make_dims(64, 128), 2, 40, 0) == n      # bf16 u, z: same scratch
     assert bd.reverse_scan_backward_workspace_size(bd.make_dims(64, 96, dtype=torch.float32), 2, 40, 0) == 0
     assert _bwd(lib, bad=(0, None)) == 1
     assert _bwd(lib, bad=(14, None)) == 1
     assert _bwd(lib, B=0) == 1
     assert _bwd(lib, chunk=-1) == 1
-    assert _bwd(lib, dims=bd.make_dims(64, 128)) == 2                                  # bf16: not yet
     assert _bwd(lib, dims=bd.make_dims(64, 96, dtype=torch.float32), ldz=96) == 2      # E % 64
     assert _bwd(lib, dims=bd.make_dims(64, 128, dtype=torch.float32, flags=bd.R2L_FLAG_FORWARD_SCAN)) == 2
     assert _bwd(lib, ldz=64) == 1
@@ -175,3 +174,45 @@ def test_scan_backward_argument_checks(lib):
     big = bd.make_dims(64, 128, dtype=torch.float32)
     assert bd.reverse_scan_backward_workspace_size(big, 65535, 65535, 1) == 0     # beyond the launch grid
     assert _bwd(lib, B=65535, L=65535, chunk=1, ws_bytes=1 << 40) == 2
+
+
+def _hook_bwd(lib, dims=None, B=2, L=40, ws=FAKE, ws_bytes=None, w=None, g=None, dh_out=FAKE, ds=FAKE + 16,
+              lengths=None):
+    dims = dims or bd.make_dims(64, 128, dt_rank=8)
+    w = w or _weights()
+    if g is None:
+        g = bd.Grads()
+        for f, _ in bd.Grads._fields_:
+            setattr(g, f, FAKE)
+    if ws_bytes is None:
+        ws_bytes = bd.sidecar_backward_workspace_size(dims, B, L) or 1
+    return lib.r2l_sidecar_backward(FAKE, ctypes.byref(w), ctypes.byref(dims), 0.5, B, L, lengths, dh_out, FAKE, ds,
+                                    ctypes.byref(g), ws, ws_bytes, None)
+
+
+def test_hook_backward_argument_checks(lib):
+    """r2l_sidecar_backward rejects bad arguments on the host (no GPU needed)."""
+    bf = bd.make_dims(64, 128, dt_rank=8)
+    n = bd.sidecar_backward_workspace_size(bf, 2, 40)
+    assert n > bd.workspace_size(bf, 2, 40)                  # the forward's regions and the gradient's
+    assert bd.sidecar_backward_workspace_size(bf, 4, 40) > n
+    assert bd.sidecar_backward_workspace_size(bd.make_dims(64, 128, dt_rank=8, dtype=torch.float32), 2, 40) == 0
+    assert _hook_bwd(lib, dh_out=None) == 1
+    assert _hook_bwd(lib, B=0) == 1
+    assert _hook_bwd(lib, dims=bd.make_dims(64, 128, dt_rank=8, dtype=torch.float32)) == 2
+    assert _hook_bwd(lib, dims=bd.make_dims(64, 128, dt_rank=8, flags=bd.R2L_FLAG_FORWARD_SCAN)) == 2
+    assert _hook_bwd(lib, dims=bd.make_dims(64, 96, dt_rank=8)) == 2                     # d_inner % 64
+    g = bd.Grads()
+    for f, _ in bd.Grads._fields_:
+        setattr(g, f, FAKE)
+    g.A_log = None
+    assert _hook_bwd(lib, g=g) == 1
+    g.A_log = FAKE + 4
+    assert _hook_bwd(lib, g=g) == 3
+    g.A_log = FAKE
+    g.ln_w = None                                                              # the hook has a LayerNorm
+    assert _hook_bwd(lib, g=g) == 1
+    assert _hook_bwd(lib, ds=FAKE + 2) == 3
+    assert _hook_bwd(lib, ws=None) == 4
+    assert _hook_bwd(lib, ws_bytes=16) == 4
+    assert _hook_bwd(lib, ws=FAKE + 8) == 3

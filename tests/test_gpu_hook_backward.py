@@ -1,0 +1,140 @@
+"""The gradient of one whole hook (r2l_sidecar_backward) against the oracle of
+oracle/sidecar_backward.py: the chain rule through §3.4 steps ❶–❹ of "Bifocal
+Diffusion Language Models" (arXiv 2606.27732v1), the step that training the
+sidecar alone (R2LM-PI, §3.4 and §4.1) back-propagates through.
+
+Every output is checked: dh (and, bit for bit, that padding rows pass dh⁺
+through), ds, and the gradient of every parameter.  Widths are those of
+workload 1 (d_model 2048, d_inner 4096, dt_rank 128).  Tolerance: the bf16
+path's max |a − b| / max |b| ≤ 2e-2, per output; the GPU's forward
+intermediates are stored in bf16 and the gradients that feed a GEMM are
+rounded once to bf16, where the oracle keeps float64 throughout.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from reverse_selective_ssm_b200 import binding as bd
+from reverse_selective_ssm_b200 import synthetic as S
+
+from . import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+PARAMS = ("W_in", "conv_w", "conv_b", "W_x", "W_dt", "b_dt", "A_log", "D", "W_out", "ln_w", "ln_b")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    bd.load()
+
+
+def make(B, L, seed, lengths=None, ln="seeded", x_proj_std=0.8, D_value=0.5):
+    dims = S.BIG
+    h = S.make_hidden(B, L, dims.d_model, torch.bfloat16, seed=seed)
+    if lengths is not None:
+        h = S.poison_padding(h, lengths)
+    w = S.make_weights(dims, torch.bfloat16, seed=seed + 1000, x_proj_std=x_proj_std, D_value=D_value, ln=ln)
+    g = torch.Generator().manual_seed(seed + 2000)
+    dh_out = torch.randn((B, L, dims.d_model), generator=g, dtype=torch.float32)
+    return dims, h, w, dh_out
+
+
+def run_gpu(dims, h, w, s, dh_out, lengths=None):
+    dev = "cuda"
+    B, L = h.shape[0], h.shape[1]
+    bdims = bd.dims_of(dims, torch.bfloat16)
+    wdev = bd.weights_to_device(w, dev)
+    grads = bd.alloc_grads(wdev, dev)
+    for v in grads.values():
+        if v is not None:
+            v.fill_(float("nan"))                # every gradient must be written
+    ws = torch.empty(bd.sidecar_backward_workspace_size(bdims, B, L), dtype=torch.uint8, device=dev)
+    ln = None if lengths is None else lengths.to(dev)
+    dh, ds = bd.sidecar_backward(h.to(dev), wdev, bdims, s, dh_out.to(dev), grads, ln, workspace=ws)
+    torch.cuda.synchronize()
+    st, flags = bd.get_device_status(ws)
+    assert st == 0 and flags == 0, (st, flags)
+    return dh.cpu(), float(ds.cpu()[0]), {k: None if v is None else v.cpu() for k, v in grads.items()}
+
+
+def run_oracle(h, w, s, dh_out, lengths=None):
+    return O.sidecar_backward_batch(S.to_f64(h), S.weights_f64(w), s, S.to_f64(dh_out),
+                                    None if lengths is None else lengths.tolist())
+
+
+def compare(got, want, h, dh_out, lengths, tol=TOL):
+    dh, ds, grads = got
+    B, L = h.shape[0], h.shape[1]
+    lens = [L] * B if lengths is None else lengths.tolist()
+    errs = {}
+    valid = np.concatenate([S.to_f64(dh[b, :n]).ravel() for b, n in enumerate(lens)])
+    ref = np.concatenate([want["dh"][b, :n].ravel() for b, n in enumerate(lens)])
+    errs["dh"] = G.err_norm(valid, ref)
+    for b, n in enumerate(lens):              # padding rows: dh⁺ passed through, bit for bit
+        assert torch.equal(dh[b, n:].view(torch.int32), dh_out[b, n:].view(torch.int32)), f"padding of {b}"
+    errs["ds"] = abs(ds - want["ds"]) / max(abs(want["ds"]), 1e-30)
+    for k in PARAMS:
+        wk = want.get("d" + k)
+        if wk is None:
+            assert grads.get(k) is None
+            continue
+        gk = grads[k]
+        assert torch.isfinite(gk).all(), f"d{k} not written"
+        errs["d" + k] = G.err_norm(S.to_f64(gk), wk)
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"errors above {tol}: {bad} (all: {errs})"
+    return errs
+
+
+def test_hook_backward_ragged_against_oracle():
+    """B = 2 × L = 160, one sequence ragged (97), NaN padding, seeded LayerNorm,
+    a visible scan (x_proj std 0.8), s = 0.7."""
+    lengths = torch.tensor([160, 97], dtype=torch.int32)
+    dims, h, w, dh_out = make(2, 160, seed=81, lengths=lengths)
+    got = run_gpu(dims, h, w, 0.7, dh_out, lengths)
+    compare(got, run_oracle(h, w, 0.7, dh_out, lengths), h, dh_out, lengths)
+
+
+def test_hook_backward_without_layernorm():
+    """No LayerNorm (ĥ = o), s = −1.2, one sequence of 128."""
+    dims, h, w, dh_out = make(1, 128, seed=82, ln="none")
+    got = run_gpu(dims, h, w, -1.2, dh_out)
+    compare(got, run_oracle(h, w, -1.2, dh_out), h, dh_out, None)
+
+
+def test_hook_backward_workload_1():
+    """Workload 1 as it stands (B = 1, L = 2048, the configs' N(0, 0.02)
+    weights and D = 1, s = 1.0)."""
+    case = S.make_case(1)
+    g = torch.Generator().manual_seed(83)
+    dh_out = torch.randn(case.h.shape, generator=g, dtype=torch.float32)
+    got = run_gpu(case.dims, case.h, case.weights[0], case.s[0], dh_out)
+    compare(got, run_oracle(case.h, case.weights[0], case.s[0], dh_out), case.h, dh_out, None)
+
+
+def test_hook_backward_reproducible():
+    lengths = torch.tensor([96, 45], dtype=torch.int32)
+    dims, h, w, dh_out = make(2, 96, seed=84, lengths=lengths)
+    a = run_gpu(dims, h, w, 0.4, dh_out, lengths)
+    b = run_gpu(dims, h, w, 0.4, dh_out, lengths)
+    assert torch.equal(a[0].view(torch.int32), b[0].view(torch.int32))
+    assert a[1] == b[1]
+    for k in PARAMS:
+        assert torch.equal(a[2][k].view(torch.int32), b[2][k].view(torch.int32)), k
+
+
+def test_hook_backward_zero_gate():
+    """s = 0: the hook is the identity, so dh = dh⁺ bit for bit and every
+    parameter's gradient is zero; only ds = Σ dh⁺ ⊙ ĥ is not."""
+    dims, h, w, dh_out = make(1, 64, seed=85)
+    dh, ds, grads = run_gpu(dims, h, w, 0.0, dh_out)
+    assert torch.equal(dh.view(torch.int32), dh_out.view(torch.int32))
+    for k in PARAMS:
+        assert torch.count_nonzero(grads[k]) == 0, k
+    want = run_oracle(h, w, 0.0, dh_out)
+    assert abs(ds - want["ds"]) <= TOL * abs(want["ds"])

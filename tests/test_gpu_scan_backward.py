@@ -31,16 +31,21 @@ def _lib():
     bd.load()
 
 
-def run_gpu(c, B, L, E, lengths=None, chunk=0):
+def run_gpu(c, B, L, E, lengths=None, chunk=0, act=torch.float32):
+    """act = torch.bfloat16: u and z are passed in bf16 (what the bf16 forward
+    stores), every other array in fp32."""
     dev = "cuda"
     d = {k: v.to(dev).contiguous() for k, v in c.items()}
+    if act == torch.bfloat16:
+        d["u"] = d["u"].to(torch.bfloat16)
+        d["z"] = d["z"].to(torch.bfloat16)
     M = B * L
     o = {k: torch.full((M, E), 7.0, device=dev) for k in ("du", "ddt_raw", "dz")}
     o["dbc"] = torch.full((M, 32), 7.0, device=dev)
     o["dA_log"] = torch.empty((E, 16), device=dev)
     o["dD"] = torch.empty(E, device=dev)
     o["ddt_b"] = torch.empty(E, device=dev)
-    dims = bd.make_dims(64, E, dtype=torch.float32)
+    dims = bd.make_dims(64, E, dtype=act)
     ln = None if lengths is None else lengths.to(dev)
     n = bd.reverse_scan_backward_workspace_size(dims, B, L, chunk)
     ws = torch.empty(n, dtype=torch.uint8, device=dev)
@@ -125,3 +130,18 @@ def test_scan_backward_serving_size_sampled_channels():
     want = oracle(c, B, L, E, None, channels=ch)
     compare(got, want, B, L, E, None, names=("du", "ddt_raw", "dz", "dA_log", "dD", "ddt_b"), channels=ch)
     assert torch.isfinite(got["dbc"]).all()
+
+
+@pytest.mark.parametrize("chunk", [0, 7])
+def test_scan_backward_bf16_inputs(chunk):
+    """u and z in bf16, as the bf16 forward writes them (dims dtype R2L_BF16),
+    against the oracle on those same bf16 values widened exactly: the only
+    differences left are the kernel's fp32 arithmetic, so the fp32 tolerance
+    holds.  Ragged lengths, an empty sequence, NaN padding."""
+    B, L, E = 3, 70, 128
+    lengths = torch.tensor([70, 33, 0], dtype=torch.int32)
+    c = S.make_scan_bwd_case(B, L, E, seed=65, lengths=lengths)
+    c["u"] = c["u"].to(torch.bfloat16).float()
+    c["z"] = c["z"].to(torch.bfloat16).float()
+    got = run_gpu(c, B, L, E, lengths, chunk, act=torch.bfloat16)
+    compare(got, oracle(c, B, L, E, lengths), B, L, E, lengths)
