@@ -38,7 +38,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Byte offsets of the workspace regions for a [B, L] batch.
 struct Plan {
-  size_t status, len, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, total;
+  size_t status, len, aflags, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, total;
   int chunk_tokens;  // scan chunk length (bf16 path)
   long long M;
   int E, d, R, N, ldd;
@@ -62,6 +62,7 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   size_t off = 0;
   p->status = off; off = align_up(off + 16, kAlign);
   p->len = off;    off = align_up(off + sizeof(int) * (size_t)B, kAlign);
+  p->aflags = off; off = align_up(off + sizeof(unsigned) * r2l::kMaxCheckedHooks, kAlign);   // per-hook power-path flags
   p->xz = off;     off = align_up(off + M * 2 * p->E * p->act, kAlign);
   p->u = off;      off = align_up(off + M * p->E * p->act, kAlign);
   p->dbc = off;    off = align_up(off + M * p->ldd * sizeof(float), kAlign);
@@ -170,7 +171,19 @@ r2l_status check_a_log(const float* A_log, int E, unsigned* status, bool force_g
                        Prof* prof) {
   if (force_general) return R2L_OK;
   if (prof) prof->launches++;
-  r2l::a_log_check_kernel<<<1, 1024, 0, st>>>(A_log, E, ln_table(), status + 1);
+  r2l::ALogSet set{};
+  set.a[0] = A_log;
+  r2l::a_log_check_kernel<<<1, 1024, 0, st>>>(set, E, ln_table(), status + 1);
+  R2L_LAUNCH_CHECK();
+  return R2L_OK;
+}
+
+// The same decision for the n hooks of a stack (n ≤ kMaxCheckedHooks), in one
+// launch: flags[k] for hook k.
+r2l_status check_a_log_hooks(const r2l_weights* w, int n, int E, unsigned* flags, cudaStream_t st) {
+  r2l::ALogSet set{};
+  for (int k = 0; k < n; ++k) set.a[k] = w[k].A_log;
+  r2l::a_log_check_kernel<<<n, 1024, 0, st>>>(set, E, ln_table(), flags);
   R2L_LAUNCH_CHECK();
   return R2L_OK;
 }
@@ -229,7 +242,8 @@ r2l_status launch_ln_bf16(int nv, bool has_ln, unsigned blocks, cudaStream_t st,
 
 template <typename T>
 r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, int B, int L,
-                     char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof, bool residual = true) {
+                     char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof, bool residual = true,
+                     const unsigned* a_flag = nullptr) {
   Prof dummy;
   if (!prof) prof = &dummy;
   const long long M = p.M;
@@ -304,7 +318,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   R2L_TRY(prof->mark(R2L_STAGE_SCAN, st));
   prof->launches++;
   if constexpr (kTC) {
-    R2L_TRY(check_a_log(w->A_log, E, err, (p.flags & R2L_FLAG_GENERAL_A) != 0, st, prof));
+    // the power-path decision: this hook's flag from the stack's one check, or its own
+    if (!a_flag) R2L_TRY(check_a_log(w->A_log, E, err, (p.flags & R2L_FLAG_GENERAL_A) != 0, st, prof));
     r2l::ScanArgs sa{};
     sa.u = u; sa.ldu = E;
     sa.z = xz + E; sa.ldz = 2 * E;
@@ -317,7 +332,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.carry = (float*)(ws + p.carry);
     sa.err = err;
     sa.force_general = (int)(p.flags & R2L_FLAG_GENERAL_A);
-    sa.a_general = err + 1;
+    sa.a_general = a_flag ? a_flag : err + 1;
     sa.dt_mma = dt_fused ? 1 : 0;
     sa.forward = fwd ? 1 : 0;
     sa.dr = dr; sa.lddr = R;
@@ -453,15 +468,21 @@ r2l_status r2l_sidecar_stack(void* hidden, const r2l_weights* weights, const flo
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)workspace;
   bool prepared = false;
+  // one launch decides the scan's power path for every hook (bf16 path)
+  const bool one_check = dims->dtype == R2L_BF16 && !(dims->flags & R2L_FLAG_GENERAL_A) &&
+                         n_hooks <= r2l::kMaxCheckedHooks;
+  unsigned* aflags = (unsigned*)(ws + p.aflags);
   for (int k = 0; k < n_hooks; ++k) {
     const float g = (float)std::tanh((double)s[k]);
     if (g == 0.0f) continue;
     if (!prepared) {
       R2L_TRY(prep(p, ws, lengths, B, L, st));
+      if (one_check) R2L_TRY(check_a_log_hooks(weights, n_hooks, p.E, aflags, st));
       prepared = true;
     }
     if (dims->dtype == R2L_BF16)
-      R2L_TRY(run_layer<bf16>((bf16*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
+      R2L_TRY(run_layer<bf16>((bf16*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr, true,
+                              one_check ? aflags + k : nullptr));
     else
       R2L_TRY(run_layer<float>((float*)hidden, &weights[k], p, g, B, L, ws, st, nullptr, nullptr));
   }

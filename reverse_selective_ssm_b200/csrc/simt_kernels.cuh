@@ -40,13 +40,20 @@ struct LnTable {
   uint32_t bits[16];
 };
 
+// The A_log arrays of up to kMaxCheckedHooks hooks, checked by one launch
+// (block k checks hook k and writes general[k]).
+constexpr int kMaxCheckedHooks = 64;
+struct ALogSet {
+  const float* a[kMaxCheckedHooks];
+};
+
 __global__ void __launch_bounds__(1024)
-a_log_check_kernel(const float* __restrict__ A_log, int E, const __grid_constant__ LnTable tab,
+a_log_check_kernel(const __grid_constant__ ALogSet set, int E, const __grid_constant__ LnTable tab,
                    unsigned* __restrict__ general) {
   // A_log is [E, 16] and 16-byte aligned: thread t reads uint4 number t +
   // 1024·k, whose four entries are states 4·(t mod 4) … 4·(t mod 4) + 3;
   // eight independent loads per thread are in flight at a time
-  const uint4* a4 = reinterpret_cast<const uint4*>(A_log);
+  const uint4* a4 = reinterpret_cast<const uint4*>(set.a[blockIdx.x]);
   const int m0 = (threadIdx.x & 3) * 4;
   const uint32_t t0 = tab.bits[m0], t1 = tab.bits[m0 + 1], t2 = tab.bits[m0 + 2], t3 = tab.bits[m0 + 3];
   const int n4 = E * 4;
@@ -63,7 +70,7 @@ a_log_check_kernel(const float* __restrict__ A_log, int E, const __grid_constant
     for (int k = 0; k < U; ++k) bad |= (v[k].x != t0) | (v[k].y != t1) | (v[k].z != t2) | (v[k].w != t3);
   }
   bad = __syncthreads_or(bad);
-  if (threadIdx.x == 0) *general = bad ? 1u : 0u;
+  if (threadIdx.x == 0) general[blockIdx.x] = bad ? 1u : 0u;
 }
 
 // ---------------------------------------------------------------------------

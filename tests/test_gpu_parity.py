@@ -283,3 +283,26 @@ def test_power_path_is_decided_once_per_call_exactly():
     case.weights = [mod]
     want, inter = G.run_oracle(case, [0], intermediates=True)
     assert G.err_norm(S.to_f64(y_mod[:512]), inter[0]["y"]) <= G.TOL_BF16
+
+
+def test_stack_decides_the_power_path_per_hook():
+    """r2l_sidecar_stack decides the path of all its hooks in one launch: a
+    stack whose second hook's A_log is one ulp off ln(m+1) in one entry gives,
+    bit for bit, what two r2l_sidecar_forward calls give (the first on the
+    power path, the second on the general path)."""
+    case = S.make_case(1, B=2, L=384)
+    w0 = S.make_weights(case.dims, torch.bfloat16, seed=207, x_proj_std=0.8, D_value=0.0)
+    w1 = S.make_weights(case.dims, torch.bfloat16, seed=208, x_proj_std=0.8, D_value=0.0)
+    A = w1["A_log"].clone()
+    A[77, 13] = torch.nextafter(A[77, 13], torch.tensor(float("inf")))
+    w1["A_log"] = A
+    case.weights = [w0, w1]
+    case.s = [0.8, -0.6]
+    stacked, _, fl = G.run_gpu(case)
+    assert fl == 0
+    one = S.make_case(1, B=2, L=384, weights=False)
+    one.weights, one.s = [w0], [0.8]
+    mid, _, _ = G.run_gpu(one)
+    one.h, one.weights, one.s = mid, [w1], [-0.6]
+    two, _, _ = G.run_gpu(one)
+    assert torch.equal(stacked.view(torch.int16), two.view(torch.int16))
