@@ -55,6 +55,9 @@ def parse_args(argv=None):
     ap.add_argument("--scan-backward", action="store_true",
                     help="time the fp32 reverse-scan gradient (r2l_reverse_scan_backward) at B=8, L=4096, "
                          "d_inner=4096 instead of the forward")
+    ap.add_argument("--hook-backward", action="store_true",
+                    help="time the whole hook's gradient (r2l_sidecar_backward: dh, ds and every parameter) on "
+                         "the workload instead of the forward")
     return ap.parse_args(argv)
 
 
@@ -885,6 +888,155 @@ def run_reference_backward(args, rank, world):
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------- whole-hook gradient
+
+HOOK_BWD_METRIC = "R2L sidecar hook backward tokens/sec at B=8,L=4096,d=2048 (dh, ds and every parameter gradient)"
+
+
+def hook_bwd_gemm_flops(case):
+    """Tensor-core work of one r2l_sidecar_backward call: the recomputed
+    forward's projections, then for out_proj, dt_proj, x_proj and in_proj an
+    input-gradient and a weight-gradient GEMM of the same size each."""
+    d, E, R, N = case.dims.d_model, case.dims.d_inner, case.dims.dt_rank, case.dims.d_state
+    T = float(case.valid_tokens)
+    fwd = 2.0 * T * (d * 2 * E + E * (R + 2 * N) + R * E + E * d)
+    return fwd + 2.0 * fwd
+
+
+def run_hook_backward(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from reverse_selective_ssm_b200 import binding as bd
+    from reverse_selective_ssm_b200 import synthetic as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bd.load()
+    case = S.make_case(args.config, B=args.batch, L=args.seq, shard=(rank, world))
+    dims = bd.dims_of(case.dims, case.dtype)
+    h = case.h.to(dev)
+    w = bd.weights_to_device(case.weights[0], dev)
+    grads = bd.alloc_grads(w, dev)
+    lengths = None if case.lengths is None else case.lengths.to(dev)
+    g = torch.Generator().manual_seed(90 + case.meta["first_sequence"])
+    dh_host = torch.randn(case.h.shape, generator=g, dtype=torch.float32)
+    dh_out = dh_host.to(dev)
+    ws = torch.empty(bd.sidecar_backward_workspace_size(dims, case.B, case.L), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(x=h, gout=dh_out):
+        return bd.sidecar_backward(x, w, dims, case.s[0], gout, grads, lengths, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    st, fl = bd.get_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} flags {fl}")
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for _ in range(K):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        # the hidden states and dh⁺ come from pinned host memory and dh, ds and every
+        # parameter gradient go back, every step
+        h_pin, g_pin = case.h.pin_memory(), dh_host.pin_memory()
+        outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items() if v is not None}
+        dh_pin = torch.empty(case.h.shape, dtype=torch.float32).pin_memory()
+        ds_pin = torch.empty(1, dtype=torch.float32).pin_memory()
+        h2d = h_pin.numel() * h_pin.element_size() + g_pin.numel() * g_pin.element_size()
+        d2h = sum(v.numel() * v.element_size() for v in outs.values()) + dh_pin.numel() * 4 + 4
+
+        def e2e_step():
+            h.copy_(h_pin, non_blocking=True)
+            dh_out.copy_(g_pin, non_blocking=True)
+            dh, ds = call()
+            dh_pin.copy_(dh, non_blocking=True)
+            ds_pin.copy_(ds, non_blocking=True)
+            for k, v in outs.items():
+                v.copy_(grads[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(1, min(K, 5))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": round(whole_job_rate(case.valid_tokens, world, ke, ms_e), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
+               "api": "r2l_sidecar_backward via binding, pinned host hidden states, dh+ and gradients"}
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    per_call = ms / K
+    flops = hook_bwd_gemm_flops(case)
+    tpeak, tnote = tensor_peak(peaks, peak_kind, clk, ms)
+    achieved = flops / (per_call * 1e-3) / 1e12
+    line = {
+        "metric": HOOK_BWD_METRIC if args.config == 2 else f"R2L sidecar hook backward tokens/sec, {case.name}",
+        "value": round(whole_job_rate(case.valid_tokens, world, K, ms), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(per_call, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (the workload's seeded hidden states and weights; dh+ ~ N(0, 1))",
+        "config": {"workload": case.name, "B": case.B, "L": case.L, "global_batch": case.meta["global_batch"],
+                   "s": case.s[0], "l2": "inputs larger than L2 (~10 GB of workspace touched per step), no flush",
+                   "parallelism": f"dp{world}: rank r runs sequences [r*{case.B}, (r+1)*{case.B}) of the global "
+                                  f"batch; parameter gradients would then take one all-reduce (not part of this "
+                                  f"entry point)"},
+        "roofline": {"kernel": "r2l_sidecar_backward (its tcgen05 GEMMs: the recomputed forward, then an input- "
+                               "and a weight-gradient GEMM per projection) over the whole call",
+                     "bound": "tensor", "achieved": round(achieved, 2), "peak": tpeak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tpeak, 4), "peak_source": tnote, "algorithmic_per_launch": flops,
+                     "ms_per_launch": round(per_call, 4), "traffic": None},
+        "gpu_launches": None, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_hook_backward(case, dh_host)
+    return line
+
+
+def cpu_baseline_hook_backward(case, dh_host, n=128):
+    """The whole-hook gradient oracle, as it stands, timed on a bounded
+    sample: the last n positions of sequence 0 run as a sequence of their
+    own (a timing sample only: the gradient at a position also depends on
+    dh+ at the positions before it)."""
+    import oracle as O
+    from reverse_selective_ssm_b200 import synthetic as S
+    L = case.L
+    h = S.to_f64(case.h[0:1, L - n:])
+    t = time.perf_counter()
+    O.sidecar_backward_batch(h, S.weights_f64(case.weights[0]), case.s[0], S.to_f64(dh_host[0:1, L - n:]))
+    dt = time.perf_counter() - t
+    return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"the last {n} positions of sequence 0 as a sequence of their own, numpy float64 "
+                      f"whole-hook gradient oracle, {dt:.1f} s"}
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -930,13 +1082,43 @@ def run_reference(args, rank, world):
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_reference_hook_backward(args, rank, world):
+    """The whole-hook gradient oracle timed on the host cores, each step the
+    bounded sample of cpu_baseline_hook_backward."""
+    if rank != 0:
+        return None
+    import torch
+    from reverse_selective_ssm_b200 import synthetic as S
+    case = S.make_case(args.config, B=args.batch, L=args.seq)
+    g = torch.Generator().manual_seed(90)
+    dh_host = torch.randn(case.h.shape, generator=g, dtype=torch.float32)
+    n = min(128, case.L)
+    for _ in range(args.warmup):
+        cpu_baseline_hook_backward(case, dh_host, n)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline_hook_backward(case, dh_host, n)
+    dt = time.perf_counter() - t
+    v = round(n * args.steps / dt, 2)
+    cb = {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+          "sample": f"per step the last {n} positions of sequence 0 as a sequence of their own, numpy float64 "
+                    f"whole-hook gradient oracle"}
+    return {"metric": HOOK_BWD_METRIC if args.config == 2 else f"R2L sidecar hook backward tokens/sec, {case.name}",
+            "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": case.name, "B": case.B, "L": case.L}, "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        line = run_reference_backward(args, rank, world) if args.scan_backward else run_reference(args, rank, world)
+        line = run_reference_backward(args, rank, world) if args.scan_backward else \
+            run_reference_hook_backward(args, rank, world) if args.hook_backward else run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return 0
@@ -947,7 +1129,8 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = (run_scan_backward if args.scan_backward else run_ours)(args, rank, world, local_rank)
+        fn = run_scan_backward if args.scan_backward else run_hook_backward if args.hook_backward else run_ours
+        line = fn(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()

@@ -93,3 +93,22 @@ def test_scan_ceilings_arithmetic():
     assert out["fp32_pipe"]["ceiling_ms"] == pytest.approx(75 * 32768 * 4096 / (148 * 128 * 1965e6) * 1e3, rel=1e-3)
     assert out["fp32_pipe"]["frac"] == pytest.approx(out["fp32_pipe"]["ceiling_ms"] / 0.6436, rel=1e-3)
     assert "issue" not in out                             # no committed summary for this workload tag
+
+
+def test_reference_arm_hook_backward_line():
+    out = _run(["--impl", "reference", "--hook-backward", "--steps", "1", "--warmup", "0", "--config", "1",
+                "--seq", "32"])
+    assert len(out) == 1
+    _check(out[0], out[0]["metric"])
+    assert "hook backward" in out[0]["metric"]
+
+
+def test_hook_backward_gemm_flops():
+    """Three times the forward's projection flops: the recomputed forward and an
+    input- and a weight-gradient GEMM per projection (52.69 MFLOP per token
+    per layer at d_model 2048, d_inner 4096, dt_rank 128)."""
+    from reverse_selective_ssm_b200 import synthetic as S
+    case = S.make_case(1, weights=False, L=8)
+    per_token = 2 * (2048 * 8192 + 4096 * 160 + 128 * 4096 + 4096 * 2048)
+    assert per_token == 52690944
+    assert bench.hook_bwd_gemm_flops(case) == 3 * per_token * 8
