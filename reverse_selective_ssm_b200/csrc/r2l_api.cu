@@ -630,7 +630,7 @@ struct BwdPlan {
   Plan f;                                        // the forward's regions
   long long Mp;                                  // positions rounded up to 8 (K of the weight gradients)
   size_t dt32, winT, woutT, wxT, wdtT, stats, dsrow, do16, lnpart, dy, doT, yT, dus, dz, ddt, dbcs, sbwd, sbwd_bytes,
-      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, dpre, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, total;
+      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, total;
 };
 
 long long row_chunks(long long M) { return (M + r2l::bwd::ROW_CHUNK - 1) / r2l::bwd::ROW_CHUNK; }
@@ -672,7 +672,6 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   q->ddbcT = take(ldd * Mp * 2);
   q->uT = take(E * Mp * 2);
   q->dux = take(M * E * 4);
-  q->dpre = take(M * E * 4);
   q->cpart = take((size_t)row_chunks(p.M) * 5 * E * 4);
   q->dxz16 = take(M * 2 * E * 2);
   q->dxzT = take(2 * E * Mp * 2);
@@ -696,20 +695,24 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   return true;
 }
 
-int grid_for(long long n, int threads) {
-  long long b = (n + threads - 1) / threads;
-  return (int)(b < 148 * 16 ? (b > 0 ? b : 1) : 148 * 16);
-}
-
-// out[c, m] = bf16(in[m, c]) over M rows (ld_out = Mp), padding rows zeroed.
+// in[m, c] (M rows, C columns) rounded to bf16 into out[m, c] (when out is not
+// null, ld_out) and into its transpose outT[c, m] (when outT is not null, ldT ≥
+// M; columns M … ldT−1 zero).  Padding rows are zero in both.
 template <typename TIn>
-r2l_status transpose(const TIn* in, long long ld_in, long long M, int C, bf16* out, long long ld_out, const int* len,
-                     int L, cudaStream_t st) {
+r2l_status cvt_transpose(const TIn* in, long long ld_in, long long M, int C, bf16* out, long long ld_out, bf16* outT,
+                         long long ldT, const int* len, int L, cudaStream_t st) {
   if (M <= 0 || C <= 0) return R2L_OK;
-  const dim3 grid((unsigned)((C + 31) / 32), (unsigned)((ld_out + 31) / 32));
-  r2l::bwd::transpose_bf16_kernel<TIn><<<grid, 256, 0, st>>>(in, ld_in, (int)M, C, out, ld_out, len, L);
+  const long long rows = outT ? std::max(M, ldT) : M;
+  const dim3 grid((unsigned)((C + 63) / 64), (unsigned)((rows + 63) / 64));
+  r2l::bwd::cvt_transpose_kernel<TIn><<<grid, 256, 0, st>>>(in, ld_in, M, C, out, ld_out, outT, ldT, len, L);
   R2L_LAUNCH_CHECK();
   return R2L_OK;
+}
+
+template <typename TIn>
+r2l_status transpose(const TIn* in, long long ld_in, long long M, int C, bf16* outT, long long ldT, const int* len,
+                     int L, cudaStream_t st) {
+  return cvt_transpose<TIn>(in, ld_in, M, C, nullptr, 0, outT, ldT, len, L, st);
 }
 
 // C[m, n] = Σ_k A[m, k]·B[n, k], bf16 operands, fp32 result.
@@ -794,11 +797,10 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   const long long nrc = row_chunks(M);
   if (has_ln) {
     float* lnpart = (float*)(ws + q.lnpart);
-    K::ln_bwd_cols_kernel<<<dim3((unsigned)((d + 127) / 128), (unsigned)nrc), 128, 0, st>>>(o, dh_out, g, d, len, L,
+    K::ln_bwd_cols_kernel<<<dim3((unsigned)((d + 511) / 512), (unsigned)nrc), 128, 0, st>>>(o, dh_out, g, d, len, L,
                                                                                             M, stats, lnpart);
     R2L_LAUNCH_CHECK();
-    K::colsum_kernel<<<(d + 255) / 256, 256, 0, st>>>(lnpart, (int)nrc, 2LL * d, d, 1.0f, gr->ln_w);
-    K::colsum_kernel<<<(d + 255) / 256, 256, 0, st>>>(lnpart + d, (int)nrc, 2LL * d, d, 1.0f, gr->ln_b);
+    K::chunk_sum_kernel<0><<<(2 * d + 31) / 32, 256, 0, st>>>(lnpart, (int)nrc, 2 * d, d, gr->ln_w, gr->ln_b);
     R2L_LAUNCH_CHECK();
   }
 
@@ -831,53 +833,48 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
 
   // ---- dt_proj: dΔr = ddt_raw·W_dt, dW_dt = ddt_rawᵀ·Δr
   bf16* ddt16 = (bf16*)(ws + q.ddt16);
-  K::to_bf16_rows_kernel<float><<<grid_for(M * E, 256), 256, 0, st>>>(ddt, E, (int)M, E, ddt16, E, len, L);
-  R2L_LAUNCH_CHECK();
+  bf16* ddtT = (bf16*)(ws + q.ddtT);
+  R2L_TRY(cvt_transpose(ddt, E, M, E, ddt16, E, ddtT, Mp, len, L, st));
   float* ddr = (float*)(ws + q.ddr);
   R2L_TRY(gemm_f32(ddt16, E, wdtT, E, ddr, R, M, R, E, len, L, err, gpart, gpb, st));
-  bf16* ddtT = (bf16*)(ws + q.ddtT);
   bf16* drT = (bf16*)(ws + q.drT);
-  R2L_TRY(transpose(ddt16, E, M, E, ddtT, Mp, len, L, st));
   R2L_TRY(transpose(dr, R, M, R, drT, Mp, len, L, st));
   R2L_TRY(gemm_f32(ddtT, (int)Mp, drT, (int)Mp, gr->dt_proj_w, R, E, R, (int)Mp, nullptr, E, err, gpart, gpb, st));
 
   // ---- x_proj: d[Δr|B|C] → du_x = d[Δr|B|C]·W_x, dW_x = d[Δr|B|C]ᵀ·u
   bf16* ddbc16 = (bf16*)(ws + q.ddbc16);
-  K::to_bf16_rows_kernel<float><<<grid_for(M * R, 256), 256, 0, st>>>(ddr, R, (int)M, R, ddbc16, ldd, len, L);
-  K::to_bf16_rows_kernel<float><<<grid_for(M * 2 * p.N, 256), 256, 0, st>>>(dbcs, 2 * p.N, (int)M, 2 * p.N,
-                                                                           ddbc16 + R, ldd, len, L);
-  R2L_LAUNCH_CHECK();
+  bf16* ddbcT = (bf16*)(ws + q.ddbcT);
+  R2L_TRY(cvt_transpose(ddr, R, M, R, ddbc16, ldd, ddbcT, Mp, len, L, st));
+  R2L_TRY(cvt_transpose(dbcs, 2LL * p.N, M, 2 * p.N, ddbc16 + R, ldd, ddbcT + (size_t)R * Mp, Mp, len, L, st));
   float* dux = (float*)(ws + q.dux);
   R2L_TRY(gemm_f32(ddbc16, ldd, wxT, ldd, dux, E, M, E, ldd, len, L, err, gpart, gpb, st));
-  bf16* ddbcT = (bf16*)(ws + q.ddbcT);
   bf16* uT = (bf16*)(ws + q.uT);
-  R2L_TRY(transpose(ddbc16, ldd, M, ldd, ddbcT, Mp, len, L, st));
   R2L_TRY(transpose(u, E, M, E, uT, Mp, len, L, st));
   R2L_TRY(gemm_f32(ddbcT, (int)Mp, uT, (int)Mp, gr->x_proj_w, E, ldd, E, (int)Mp, nullptr, ldd, err, gpart, gpb,
                    st));
 
-  // ---- conv + SiLU: dpre, dx (into dxz), dconv_w, dconv_b; dz into dxz
-  float* dpre = (float*)(ws + q.dpre);
+  // ---- conv + SiLU: dx (into dxz and dxzᵀ), dconv_w, dconv_b; dz into dxz and dxzᵀ
   bf16* dxz16 = (bf16*)(ws + q.dxz16);
-  K::conv_silu_bwd_pre_kernel<<<grid_for(M * E, 256), 256, 0, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E,
-                                                                   len, L, M, dpre);
-  R2L_LAUNCH_CHECK();
-  K::conv_bwd_dx_kernel<<<grid_for(M * E, 256), 256, 0, st>>>(dpre, w->conv_w, E, len, L, M, dxz16, 2LL * E);
-  K::to_bf16_rows_kernel<float><<<grid_for(M * E, 256), 256, 0, st>>>(dz, E, (int)M, E, dxz16 + E, 2LL * E, len, L);
+  bf16* dxzT = (bf16*)(ws + q.dxzT);
   float* cpart = (float*)(ws + q.cpart);
-  K::conv_bwd_params_kernel<<<dim3((unsigned)((E + 127) / 128), (unsigned)nrc), 128, 0, st>>>(dpre, xz, 2LL * E, E,
-                                                                                             len, L, M, cpart);
-  K::conv_bwd_reduce_kernel<<<(E + 127) / 128, 128, 0, st>>>(cpart, (int)nrc, E, gr->conv_w, gr->conv_b);
+  if (cudaFuncSetAttribute(K::conv_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::CONV_SMEM) !=
+      cudaSuccess)
+    return R2L_ERR_CUDA;
+  K::conv_bwd_kernel<<<dim3((unsigned)((E + K::CONV_CH - 1) / K::CONV_CH), (unsigned)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS)),
+                       256, K::CONV_SMEM, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E, len, L, M, dxz16, 2LL * E, dxzT, Mp,
+                                     cpart);
   R2L_LAUNCH_CHECK();
+  K::chunk_sum_kernel<1><<<(5 * E + 31) / 32, 256, 0, st>>>(cpart, (int)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS), 5 * E,
+                                                            E, gr->conv_w, gr->conv_b);
+  R2L_LAUNCH_CHECK();
+  R2L_TRY(cvt_transpose(dz, E, M, E, dxz16 + E, 2LL * E, dxzT + (size_t)E * Mp, Mp, len, L, st));
 
   // ---- in_proj: dh = dh⁺ + [dx | dz]·W_in, dW_in = [dx | dz]ᵀ·h
   float* dhtmp = (float*)(ws + q.dhtmp);
   R2L_TRY(gemm_f32(dxz16, 2 * E, winT, 2 * E, dhtmp, d, M, d, 2 * E, len, L, err, gpart, gpb, st));
-  K::add_rows_kernel<<<grid_for(M * d, 256), 256, 0, st>>>(dh_out, dhtmp, d, len, L, M, dh);
+  K::add_rows_kernel<<<(unsigned)std::min<long long>(M, 148 * 8), 256, 0, st>>>(dh_out, dhtmp, d, len, L, M, dh);
   R2L_LAUNCH_CHECK();
-  bf16* dxzT = (bf16*)(ws + q.dxzT);
   bf16* hT = (bf16*)(ws + q.hT);
-  R2L_TRY(transpose(dxz16, 2LL * E, M, 2 * E, dxzT, Mp, len, L, st));
   R2L_TRY(transpose((const bf16*)hidden, d, M, d, hT, Mp, len, L, st));
   R2L_TRY(gemm_f32(dxzT, (int)Mp, hT, (int)Mp, gr->in_proj_w, d, 2LL * E, d, (int)Mp, nullptr, 2 * E, err, gpart,
                    gpb, st));

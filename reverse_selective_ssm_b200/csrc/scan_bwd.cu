@@ -38,6 +38,10 @@
 // columns.
 #include <cuda_runtime.h>
 
+#include <cmath>
+#include <cstring>
+#include <type_traits>
+
 #include "common.cuh"
 #include "scan_bwd.h"
 
@@ -81,6 +85,8 @@ struct Args {
   float* pD;               // [B][nc][E]
   float* pb;               // [B][nc][E]
   float* pbc;              // [E/CPB][B·L][32] per-block partial dB | dC
+  int nbc;                 // channel blocks in pbc
+  uint32_t lnbits[16];     // float log(1) … log(16): the power-path A_log
 };
 
 __device__ __forceinline__ int seq_len(const Args& a, int b) {
@@ -591,13 +597,25 @@ __global__ void reduce_bc_kernel(const Args a) {
   if (t >= M * 32) return;
   const long long row = t >> 5;
   const int col = (int)(t & 31);
-  const int nb = a.E / CPB;
+  const int nb = a.nbc;
   float acc = 0.0f;
   for (int cb = 0; cb < nb; ++cb) acc += a.pbc[((size_t)cb * M + row) * 32 + col];
   a.dbc[row * a.ld_dbc + col] = acc;
 }
 
 }  // namespace sbwd
+}  // namespace r2l
+
+#include "scan_bwd_seq.cuh"
+
+namespace r2l {
+
+// The walk along each sequence (scan_bwd_seq.cuh) runs when the chunk length
+// is left to the library and one 32-channel block per (sequence, block) gives
+// the GPU at least four blocks per SM; otherwise the chunked kernels above.
+static bool use_seq(int B, int E, int chunk_tokens) {
+  return chunk_tokens == 0 && (long long)B * (E / sbwd::QC) >= 4LL * 148;
+}
 
 int scan_bwd_chunk_tokens(int chunk_tokens) {
   if (chunk_tokens <= 0) return 16;
@@ -605,6 +623,7 @@ int scan_bwd_chunk_tokens(int chunk_tokens) {
 }
 
 bool scan_bwd_supported(int B, int L, int E, int chunk_tokens) {
+  if (use_seq(B, E, chunk_tokens)) return E % sbwd::QC == 0 && B <= 65535;
   const int T = scan_bwd_chunk_tokens(chunk_tokens);
   const long long nc = (L + T - 1) / T;
   const long long nseg = ((long long)B * nc + sbwd::RSEG - 1) / sbwd::RSEG;
@@ -612,10 +631,15 @@ bool scan_bwd_supported(int B, int L, int E, int chunk_tokens) {
 }
 
 size_t scan_bwd_scratch_bytes(int B, int L, int E, int chunk_tokens) {
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  if (use_seq(B, E, chunk_tokens)) {
+    const size_t nc = (size_t)((L + sbwd::QS - 1) / sbwd::QS);
+    return al((size_t)B * nc * E * 16 * 4) + al((size_t)B * E * 16 * 4) + 2 * al((size_t)B * E * 4) +
+           al((size_t)(E / sbwd::QC) * B * L * 32 * 4);
+  }
   const int T = scan_bwd_chunk_tokens(chunk_tokens);
   const size_t nc = (size_t)((L + T - 1) / T);
   const size_t cells = (size_t)B * nc * E;
-  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t nseg = (cells / E + sbwd::RSEG - 1) / sbwd::RSEG;
   return al(cells * 16 * 4) * 3 + al(cells * 4) * 4 + al((size_t)(E / sbwd::CPB) * B * L * 32 * 4) +
          al(nseg * E * 16 * 3 * 4);
@@ -633,8 +657,30 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   a.nc = (g.L + a.T - 1) / a.T;
   a.lengths = g.lengths;
   a.status = g.status;
-  const size_t cells = (size_t)g.B * a.nc * g.E;
+  for (int m = 0; m < 16; ++m) {
+    const float v = (float)std::log((double)(m + 1));
+    std::memcpy(&a.lnbits[m], &v, sizeof(v));
+  }
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  const long long M = (long long)g.B * g.L;
+  if (use_seq(g.B, g.E, g.chunk_tokens)) {
+    a.T = QS;
+    a.nc = (g.L + QS - 1) / QS;
+    char* p = (char*)scratch;
+    a.hcar = (float*)p; p += al((size_t)g.B * a.nc * g.E * 16 * 4);
+    a.pA = (float*)p;   p += al((size_t)g.B * g.E * 16 * 4);
+    a.pD = (float*)p;   p += al((size_t)g.B * g.E * 4);
+    a.pb = (float*)p;   p += al((size_t)g.B * g.E * 4);
+    a.pbc = (float*)p;
+    a.nbc = g.E / QC;
+    const dim3 grid(g.E / QC, g.B);
+    seq_ckpt_kernel<<<grid, QT, 0, st>>>(a);
+    seq_final_kernel<<<grid, QT, 0, st>>>(a);
+    seq_reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a);
+    reduce_bc_kernel<<<(unsigned)((M * 32 + 255) / 256), 256, 0, st>>>(a);
+    return cudaPeekAtLastError();
+  }
+  const size_t cells = (size_t)g.B * a.nc * g.E;
   char* p = (char*)scratch;
   a.hcar = (float*)p; p += al(cells * 16 * 4);
   a.gcar = (float*)p; p += al(cells * 16 * 4);
@@ -644,6 +690,7 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   a.pD = (float*)p;   p += al(cells * 4);
   a.pb = (float*)p;   p += al(cells * 4);
   a.pbc = (float*)p;  p += al((size_t)(g.E / CPB) * g.B * g.L * 32 * 4);
+  a.nbc = g.E / CPB;
   float* seg = (float*)p;
   const int nseg = (int)(((size_t)g.B * a.nc + RSEG - 1) / RSEG);
 
@@ -662,7 +709,6 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
   final_kernel<<<grid, THREADS, fsmem, st>>>(a);
   reduce_params_seg_kernel<<<dim3((unsigned)((g.E * 16 + 255) / 256), nseg), 256, 0, st>>>(a, seg);
   reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a, seg, nseg);
-  const long long M = (long long)g.B * g.L;
   reduce_bc_kernel<<<(unsigned)((M * 32 + 255) / 256), 256, 0, st>>>(a);
   return cudaPeekAtLastError();
 }

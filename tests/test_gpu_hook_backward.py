@@ -33,8 +33,7 @@ def _lib():
     bd.load()
 
 
-def make(B, L, seed, lengths=None, ln="seeded", x_proj_std=0.8, D_value=0.5):
-    dims = S.BIG
+def make(B, L, seed, lengths=None, ln="seeded", x_proj_std=0.8, D_value=0.5, dims=S.BIG):
     h = S.make_hidden(B, L, dims.d_model, torch.bfloat16, seed=seed)
     if lengths is not None:
         h = S.poison_padding(h, lengths)
@@ -131,6 +130,19 @@ def test_hook_backward_ragged_against_oracle():
     hh = hhat_pair(dims, h, w, 0.7, lengths)
     compare(got, run_oracle(h, w, 0.7, dh_out, lengths), h, dh_out, lengths,
             ds_check=(0.7, dh_out, lengths) + hh)
+
+
+def test_hook_backward_odd_sizes():
+    """d_inner 192 (the conv gradient's 128-channel tiles end part-way), d_model
+    136, dt_rank 8, and B·L = 2 × 75 positions (not a multiple of 8: the
+    transposed operands carry zero columns past the last position), ragged."""
+    dims = S.Dims(d_model=136, d_inner=192, d_state=16, dt_rank=8, d_conv=4)
+    lengths = torch.tensor([75, 38], dtype=torch.int32)
+    _, h, w, dh_out = make(2, 75, seed=86, lengths=lengths, dims=dims)
+    got = run_gpu(dims, h, w, 0.9, dh_out, lengths)
+    hh = hhat_pair(dims, h, w, 0.9, lengths)
+    compare(got, run_oracle(h, w, 0.9, dh_out, lengths), h, dh_out, lengths,
+            ds_check=(0.9, dh_out, lengths) + hh)
 
 
 def test_hook_backward_without_layernorm():

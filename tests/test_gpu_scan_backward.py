@@ -6,7 +6,10 @@ its softplus(Δ) input and SiLU(z) gate.
 Covered: ragged lengths that end chunks part-way and an empty sequence (with
 NaN in every padding row of every input), chunk lengths 1, 7, 16 and 32,
 bitwise reproducibility, the full d_inner of 4096 (64 channel blocks in the
-dB | dC reduction), and the B = 8 × L = 4096 batch on sampled channels.
+dB | dC reduction), and the B = 8 × L = 4096 batch on sampled channels.  At
+B = 8 × d_inner 4096 the library walks each sequence in one block
+(scan_bwd_seq.cuh): that path is covered with ragged lengths, the power and
+the general decays in one call, bf16 inputs and reproducibility.
 Tolerance: max |a − b| / max |b| ≤ 1e-4 per output (fp32 against fp64).
 """
 import numpy as np
@@ -145,3 +148,43 @@ def test_scan_backward_bf16_inputs(chunk):
     c["z"] = c["z"].to(torch.bfloat16).float()
     got = run_gpu(c, B, L, E, lengths, chunk, act=torch.bfloat16)
     compare(got, oracle(c, B, L, E, lengths), B, L, E, lengths)
+
+
+def walk_case(seed, mixed_A):
+    """B = 8 × d_inner 4096: 1024 blocks of 32 channels, enough for the walk
+    along each sequence.  Lengths end chunks part-way, one sequence is empty,
+    one has a single position, one fills L = 70 (its last chunk runs past L).
+    With mixed_A every other 32-channel block gets a random A, so one call
+    runs blocks on the power path and blocks on the general path."""
+    B, L, E = 8, 70, 4096
+    lengths = torch.tensor([70, 33, 0, 1, 16, 17, 64, 50], dtype=torch.int32)
+    c = S.make_scan_bwd_case(B, L, E, seed=seed, lengths=lengths)
+    if mixed_A:
+        g = torch.Generator().manual_seed(seed + 1)
+        rnd = torch.log(torch.rand((E, 16), generator=g) * 15.0 + 0.5)
+        blk = (torch.arange(E) // 32) % 2 == 1
+        c["A_log"][blk] = rnd[blk]
+    return c, B, L, E, lengths
+
+
+@pytest.mark.parametrize("mixed_A", [False, True])
+def test_scan_backward_walk_along_sequences(mixed_A):
+    c, B, L, E, lengths = walk_case(67, mixed_A)
+    got = run_gpu(c, B, L, E, lengths)
+    compare(got, oracle(c, B, L, E, lengths), B, L, E, lengths)
+
+
+def test_scan_backward_walk_bf16_inputs():
+    c, B, L, E, lengths = walk_case(68, True)
+    for k in ("u", "z"):
+        c[k] = c[k].to(torch.bfloat16).to(torch.float32)
+    got = run_gpu(c, B, L, E, lengths, act=torch.bfloat16)
+    compare(got, oracle(c, B, L, E, lengths), B, L, E, lengths)
+
+
+def test_scan_backward_walk_reproducible():
+    c, B, L, E, lengths = walk_case(69, True)
+    a = run_gpu(c, B, L, E, lengths)
+    b = run_gpu(c, B, L, E, lengths)
+    for k in OUTS:
+        assert torch.equal(a[k].view(torch.int32), b[k].view(torch.int32)), k
