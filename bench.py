@@ -83,7 +83,7 @@ STAGE_SOURCES = {
     "out_proj": ["gemm_tc.cuh", "tc_gemm.cu", "tc_gemm.h"] + _COMMON,
     "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh", "scan_split.cuh"] + _COMMON,
     "ln_residual": ["simt_kernels.cuh"] + _COMMON,
-    "scan_bwd": ["scan_bwd.cu", "scan_bwd.h"] + _COMMON,
+    "scan_bwd": ["scan_bwd.cu", "scan_bwd.h", "scan_bwd_seq.cuh"] + _COMMON,
 }
 
 
@@ -724,7 +724,20 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
 # ---------------------------------------------------------------- scan gradient
 
 BWD_METRIC = "R2L reverse-scan backward tokens/sec at B=8,L=4096,E=4096 (fp32)"
-BWD_LAUNCHES = 6          # kernels one r2l_reverse_scan_backward call launches
+B200_SCAN_BWD_BLOCK = 32  # channels per block of the walk along each sequence
+
+
+def bwd_walks_sequences(B, E):
+    """The library's path choice for chunk_tokens = 0: one 32-channel block
+    walks each sequence when that gives at least 4 blocks per SM."""
+    return B * (E // B200_SCAN_BWD_BLOCK) >= 4 * B200_SMS
+
+
+def bwd_launches(B, E):
+    """Kernels one r2l_reverse_scan_backward call launches: checkpoints,
+    gradient, two reductions on the walk; state, carry, gradient and three
+    reductions on the chunked path."""
+    return 4 if bwd_walks_sequences(B, E) else 6
 
 
 def bwd_bytes_per_token(E):
@@ -833,15 +846,17 @@ def run_scan_backward(args, rank, world, local_rank):
                 "logUniform[1e-3,1e-1] step; A=-(1..16); D=1)",
         "config": {"workload": f"reverse-scan gradient fp32 B={B} L={L} E={E} N=16", "B": B, "L": L,
                    "d_inner": E, "d_state": 16, "chunk_tokens": 16,
+                   "path": ("one 32-channel block walks each sequence, H checkpoints every 16 positions"
+                            if bwd_walks_sequences(B, E) else "chunks of 16 positions with H and G carries"),
                    "l2": "inputs larger than L2 (~4 GB read and written per step), no flush",
                    "parallelism": f"dp{world}: one independent batch per GPU, no collective"},
-        "roofline": {"kernel": f"r2l_reverse_scan_backward (the {BWD_LAUNCHES} launches of one call)",
+        "roofline": {"kernel": f"r2l_reverse_scan_backward (the {bwd_launches(B, E)} launches of one call)",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "peak_source": f"{peak_kind} HBM copy", "algorithmic_per_launch": nbytes,
                      "bytes_per_token": bwd_bytes_per_token(E), "ms_per_launch": round(per_call, 4),
                      "traffic": read_traffic("scan_bwd", tag)},
-        "gpu_launches": BWD_LAUNCHES * K, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
+        "gpu_launches": bwd_launches(B, E) * K, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_backward(host, B, L, E)
@@ -901,6 +916,18 @@ def hook_bwd_gemm_flops(case):
     T = float(case.valid_tokens)
     fwd = 2.0 * T * (d * 2 * E + E * (R + 2 * N) + R * E + E * d)
     return fwd + 2.0 * fwd
+
+
+def hook_bwd_launches(case):
+    """Kernels one r2l_sidecar_backward call launches at the bench's shapes
+    (as the ncu launch list shows them): the recomputed forward (6) and dt_raw,
+    4 weight transposes, the gate and LayerNorm gradient (4, or 2 without
+    LayerNorm), the scan gradient, and per projection its input-gradient GEMM,
+    weight-gradient GEMM (dt_proj and x_proj with a split-K sum) and operand
+    conversions, the conv gradient and its column sum, and dh = dh+ + dx."""
+    w = case.weights[0]
+    ln = 4 if w.get("ln_w") is not None else 2
+    return 6 + 1 + 4 + ln + bwd_launches(case.B, case.dims.d_inner) + 22
 
 
 def run_hook_backward(args, rank, world, local_rank):
@@ -1013,7 +1040,7 @@ def run_hook_backward(args, rank, world, local_rank):
                      "bound": "tensor", "achieved": round(achieved, 2), "peak": tpeak, "unit": "TFLOP/s",
                      "frac": round(achieved / tpeak, 4), "peak_source": tnote, "algorithmic_per_launch": flops,
                      "ms_per_launch": round(per_call, 4), "traffic": None},
-        "gpu_launches": None, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
+        "gpu_launches": hook_bwd_launches(case) * K, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_hook_backward(case, dh_host)

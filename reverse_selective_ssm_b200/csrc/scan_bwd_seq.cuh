@@ -21,8 +21,9 @@
 // Threads: two per channel, lanes j and j+16 of a warp, thread h holding the
 // states 8h … 8h+7 as four f32x2 pairs.  Per position a channel's two halves
 // of ⟨C, H⟩, Σ G ⊙ B and Σ gh ⊙ A meet by one xor-16 shuffle each; dB | dC
-// over the warp's 16 channels is a 15-shuffle reduce-scatter that leaves each
-// lane one of the 32 columns, and the block's two warps are summed in order.
+// over the warp's 16 channels goes through a per-warp shared-memory transpose
+// (each lane sums one of the 32 columns over the channels in a fixed pairwise
+// tree), and the block's two warps are summed in order.
 //
 // Padding positions (i ≥ the sequence's length) are staged as zeros: their
 // decay is 1 and their input 0, so H stays 0 past the end and every gradient
@@ -45,6 +46,10 @@ constexpr int QMINB = 7;        // resident blocks per SM the registers allow
 // stores of 4-channel groups (one group per lane) fall in distinct banks.
 constexpr int QCP = QC + QC / 4;
 __device__ __forceinline__ int qi(int ch) { return ch + (ch >> 2); }
+// Row stride of the dB | dC transpose buffer: 36 words, so the eight 16-byte
+// stores of a wavefront (channels j … j+7) start in distinct bank groups and a
+// column read (one word per channel) touches 32 distinct banks.
+constexpr int QXB = 36;
 
 struct QLane {
   int w, j, h, cl, c, b, n, nck;
@@ -192,6 +197,7 @@ struct QSmem {
   float4 bc[QS][8];       // B | C
   float red[2][QS][32];   // dB | dC per warp
   float4 hb[QS / QH - 1][2][QT];   // H at positions 4, 8, 12 of the chunk
+  float xb[2][16][QXB];   // per warp: one position's dB | dC by channel (row) and column
 };
 
 // Stage chunk rows s … s+15 of the block's 32 channels (zeros past the end).
@@ -289,37 +295,37 @@ __device__ __forceinline__ void qgstep(const QLane& l, QSmem& S, int r, const fl
   pc += __shfl_xor_sync(0xffffffffu, pc, 16);
   sa += __shfl_xor_sync(0xffffffffu, sa, 16);
   sb += __shfl_xor_sync(0xffffffffu, sb, 16);
-  // dB (values 0-7) and dC (8-15) of states 8h … 8h+7 over the warp's 16
-  // channels: reduce-scatter on lane bits 3, 2, 1, 0
-  const bool b3 = l.j & 8, b2 = l.j & 4, b1 = l.j & 2, b0 = l.j & 1;
-  float w8[8];
+  // dB (columns 8h … 8h+7) and dC (16 + 8h …) over the warp's 16 channels:
+  // the warp writes its 16 × 32 values by channel, then lane c sums column c
+  // over the channels (a fixed tree: bitwise reproducible)
+  float* xr = &S.xb[l.w][l.j][0];
+  __syncwarp();
+  *reinterpret_cast<float4*>(xr + 8 * l.h) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(xr + 8 * l.h + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  *reinterpret_cast<float4*>(xr + 16 + 8 * l.h) = make_float4(v[8], v[9], v[10], v[11]);
+  *reinterpret_cast<float4*>(xr + 16 + 8 * l.h + 4) = make_float4(v[12], v[13], v[14], v[15]);
+  __syncwarp();
+  {
+    const int col = l.j + 16 * l.h;                     // the lane index
+    float t[16];
 #pragma unroll
-  for (int t = 0; t < 8; ++t)
-    w8[t] = (b3 ? v[t + 8] : v[t]) + __shfl_xor_sync(0xffffffffu, b3 ? v[t] : v[t + 8], 8);
-  float w4[4];
+    for (int ch = 0; ch < 16; ++ch) t[ch] = S.xb[l.w][ch][col];
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
-    w4[t] = (b2 ? w8[t + 4] : w8[t]) + __shfl_xor_sync(0xffffffffu, b2 ? w8[t] : w8[t + 4], 4);
-  float w2[2];
+    for (int w = 8; w >= 1; w >>= 1)                    // a fixed pairwise tree
 #pragma unroll
-  for (int t = 0; t < 2; ++t)
-    w2[t] = (b1 ? w4[t + 2] : w4[t]) + __shfl_xor_sync(0xffffffffu, b1 ? w4[t] : w4[t + 2], 2);
-  const float w1 = (b0 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b0 ? w2[0] : w2[1], 1);
-  // value j: dB of state 8h + j (j < 8), dC of state 8h + j − 8
-  S.red[l.w][r][(l.j < 8 ? 0 : 8) + 8 * l.h + l.j] = w1;
+      for (int i = 0; i < w; ++i) t[i] += t[i + w];
+    S.red[l.w][r][col] = t[0];
+  }
+  // the gradients (both halves of a channel hold the same sums) go over the
+  // row's staged scalars, which no later step reads
   const float p = fmaf(Dc, uu, pc);
   const float2 s2 = S.sc2[r][qi(l.cl)];
-  // the row's gradients go over its staged scalars, which no later step reads
+  const float ddt = fmaf(sb, uu, sa) * s2.y;
   float* o = reinterpret_cast<float*>(&S.sc[r][qi(l.cl)]);
-  if (l.h == 0) {
-    const float ddt = fmaf(sb, uu, sa) * s2.y;
-    o[0] = fmaf(Dc, dp, delta * sb);
-    o[1] = ddt;
-    q.dD = fmaf(dp, uu, q.dD);
-    q.db += ddt;
-  } else {
-    o[2] = p * s2.x;
-  }
+  o[2 * l.h] = l.h ? p * s2.x : fmaf(Dc, dp, delta * sb);
+  o[1] = ddt;
+  q.dD = fmaf(dp, uu, q.dD);
+  q.db += ddt;
   qdecays<POW>(delta, l.h, l.A, q.ap);                  // a_r, for G at r + 1
 }
 
