@@ -13,8 +13,8 @@
 //      every 16-position chunk (hck[b][k] = H_{16(k+1)}, zero past the end);
 //   2. seq_final_kernel walks the chunks left to right.  Per chunk it stages
 //      the per-(position, channel) scalars once and walks H from the
-//      checkpoint over positions 15 … 4, keeping the states at positions 12, 8
-//      and 4 in shared memory.  Then per group of 4 positions, left to right,
+//      checkpoint (loaded with the chunk's inputs) over positions 15 … 4, keeping
+//      the states at positions 12, 8 and 4 in shared memory.  Then per group of 4 positions, left to right,
 //      it recomputes the group's H into registers from the state on its right
 //      and walks G over it (28 H steps per 16 positions).  The G step needs
 //      a_i ⊙ H_{i+1}, which is H_i − Δ_i u_i B_i, so only H_i is kept.
@@ -42,10 +42,12 @@ constexpr int QT = 2 * QC;      // threads per block
 constexpr int QS = 16;          // positions per chunk (the checkpoint spacing)
 constexpr int QH = 4;           // positions of H held in registers
 constexpr int QMINB = 7;        // resident blocks per SM the registers allow
-// Staged per-channel rows are padded by one slot per 4 channels, so a warp's
-// stores of 4-channel groups (one group per lane) fall in distinct banks.
-constexpr int QCP = QC + QC / 4;
-__device__ __forceinline__ int qi(int ch) { return ch + (ch >> 2); }
+// Slot of channel ch = 8a + b in a staged row: b rotated by a within its group
+// of 8.  Both access patterns then hit 8 distinct 16-byte bank groups: the
+// staging stores (one lane per 4-channel group, channels 4q + i for a fixed i)
+// and the walk's reads (8 consecutive channels).
+constexpr int QCP = QC;
+__device__ __forceinline__ int qi(int ch) { return (ch & ~7) | ((ch + (ch >> 3)) & 7); }
 // Row stride of the dB | dC transpose buffer: 36 words, so the eight 16-byte
 // stores of a wavefront (channels j … j+7) start in distinct bank groups and a
 // column read (one word per channel) touches 32 distinct banks.
@@ -196,14 +198,19 @@ struct QSmem {
   float2 sc2[QS][QCP];    // dz factor dy·SiLU'(z), softplus'(v)
   float4 bc[QS][8];       // B | C
   float red[2][QS][32];   // dB | dC per warp
-  float4 hb[QS / QH - 1][2][QT];   // H at positions 4, 8, 12 of the chunk
+  float4 hb[QS / QH][2][QT];   // H at positions 4, 8, 12 of the chunk, and the checkpoint (16)
   float xb[2][16][QXB];   // per warp: one position's dB | dC by channel (row) and column
 };
 
-// Stage chunk rows s … s+15 of the block's 32 channels (zeros past the end).
-__device__ __forceinline__ void qstage(const Args& a, const QLane& l, QSmem& S, int s) {
+// Stage chunk k (rows s … s+15 of the block's 32 channels, zeros past the
+// end): the per-element scalars, B | C, and the thread's checkpoint (loaded
+// with the chunk's inputs, so the H walk starts from shared memory).
+__device__ __forceinline__ void qstage(const Args& a, const QLane& l, QSmem& S, int k) {
   const int c0 = blockIdx.x * QC;
+  const int s = k * QS;
   const int q4 = threadIdx.x & 7, rr = threadIdx.x >> 3;
+  const float* hp = a.hcar + hck_idx(a, l, k);
+  const float4 h0 = ld4(hp), h1 = ld4(hp + 4);
   const float4 dtb = ld4(a.dt_b + c0 + 4 * q4);
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
@@ -245,6 +252,8 @@ __device__ __forceinline__ void qstage(const Args& a, const QLane& l, QSmem& S, 
     S.bc[row][q] = pos < l.n ? ld4(a.bc + ((size_t)l.b * a.L + pos) * a.ldbc + 4 * q)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  S.hb[QS / QH - 1][0][threadIdx.x] = h0;
+  S.hb[QS / QH - 1][1][threadIdx.x] = h1;
 }
 
 struct QAcc {
@@ -345,12 +354,11 @@ __global__ void __launch_bounds__(QT, QMINB) seq_final_kernel(const Args a) {
     constexpr bool POW = decltype(pow_tag)::value;
     for (int k = 0; k < l.nck; ++k) {
       const int s = k * QS;
-      const float* hp = a.hcar + hck_idx(a, l, k);
       __syncthreads();                                    // the last chunk's epilogue is done with S
-      qstage(a, l, S, s);
+      qstage(a, l, S, k);
       __syncthreads();
       {
-        const float4 h0 = ld4(hp), h1 = ld4(hp + 4);
+        const float4 h0 = S.hb[QS / QH - 1][0][threadIdx.x], h1 = S.hb[QS / QH - 1][1][threadIdx.x];
         float2 H[4] = {lo2(h0), hi2(h0), lo2(h1), hi2(h1)};
 #pragma unroll
         for (int r = QS - 1; r >= QH; --r) {
@@ -363,14 +371,7 @@ __global__ void __launch_bounds__(QT, QMINB) seq_final_kernel(const Args a) {
       }
 #pragma unroll 1
       for (int g = 0; g < QS / QH; ++g) {
-        float4 h0, h1;
-        if (g == QS / QH - 1) {
-          h0 = ld4(hp);
-          h1 = ld4(hp + 4);
-        } else {
-          h0 = S.hb[g][0][threadIdx.x];
-          h1 = S.hb[g][1][threadIdx.x];
-        }
+        const float4 h0 = S.hb[g][0][threadIdx.x], h1 = S.hb[g][1][threadIdx.x];
         float2 H[4] = {lo2(h0), hi2(h0), lo2(h1), hi2(h1)};
         float2 Hs[QH][4];
 #pragma unroll
