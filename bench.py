@@ -920,14 +920,18 @@ def hook_bwd_gemm_flops(case):
 
 def hook_bwd_launches(case):
     """Kernels one r2l_sidecar_backward call launches at the bench's shapes
-    (as the ncu launch list shows them): the recomputed forward (6) and dt_raw,
+    (as the ncu launch list shows them): the recomputed forward (6, its scan
+    storing the scan gradient's H checkpoints) and dt_raw,
     4 weight transposes, the gate and LayerNorm gradient (4, or 2 without
     LayerNorm), the scan gradient, and per projection its input-gradient GEMM,
     weight-gradient GEMM (dt_proj and x_proj with a split-K sum) and operand
     conversions, the conv gradient and its column sum, and dh = dh+ + dx."""
     w = case.weights[0]
     ln = 4 if w.get("ln_w") is not None else 2
-    return 6 + 1 + 4 + ln + bwd_launches(case.B, case.dims.d_inner) + 22
+    # on the walk along each sequence the recomputed forward scan stores the H
+    # checkpoints, so the gradient skips its own checkpoint pass
+    scan = bwd_launches(case.B, case.dims.d_inner) - (1 if bwd_walks_sequences(case.B, case.dims.d_inner) else 0)
+    return 6 + 1 + 4 + ln + scan + 22
 
 
 def run_hook_backward(args, rank, world, local_rank):

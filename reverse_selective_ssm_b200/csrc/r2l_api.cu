@@ -243,7 +243,7 @@ r2l_status launch_ln_bf16(int nv, bool has_ln, unsigned blocks, cudaStream_t st,
 template <typename T>
 r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, int B, int L,
                      char* ws, cudaStream_t st, const r2l_debug_out* dbg, Prof* prof, bool residual = true,
-                     const unsigned* a_flag = nullptr) {
+                     const unsigned* a_flag = nullptr, float* hck = nullptr, int* hck_written = nullptr) {
   Prof dummy;
   if (!prof) prof = &dummy;
   const long long M = p.M;
@@ -337,6 +337,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     sa.forward = fwd ? 1 : 0;
     sa.dr = dr; sa.lddr = R;
     sa.wdt = (const bf16*)w->dt_proj_w;
+    sa.hck = hck;
+    sa.hck_written = hck_written;
     int nl = 0;
     if (r2l::scan_bf16(sa, st, &nl) != cudaSuccess) return R2L_ERR_CUDA;
     prof->launches += nl - 1;
@@ -630,7 +632,7 @@ struct BwdPlan {
   Plan f;                                        // the forward's regions
   long long Mp;                                  // positions rounded up to 8 (K of the weight gradients)
   size_t dt32, winT, woutT, wxT, wdtT, stats, dsrow, do16, lnpart, dy, doT, yT, dus, dz, ddt, dbcs, sbwd, sbwd_bytes,
-      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, total;
+      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, hck, total;
 };
 
 long long row_chunks(long long M) { return (M + r2l::bwd::ROW_CHUNK - 1) / r2l::bwd::ROW_CHUNK; }
@@ -644,6 +646,7 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   size_t off = p.total;
   auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, kAlign); return at; };
   q->dt32 = take(M * E * 4);
+  q->hck = take((size_t)B * ((L + 15) / 16) * E * 16 * 4);   // the forward's H checkpoints
   q->winT = take(d * 2 * E * 2);
   q->woutT = take(E * d * 2);
   q->wxT = take(E * ldd * 2);
@@ -758,8 +761,12 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
 
   // ---- the forward's intermediates: xz, u, Δr|B|C, Δr (bf16), y, o; dt_raw in fp32
   R2L_TRY(prep(p, ws, lengths, B, L, st));
-  // run_layer with residual = false reads hidden and writes nothing to it
-  R2L_TRY(run_layer<bf16>((bf16*)const_cast<void*>(hidden), w, p, g, B, L, ws, st, nullptr, nullptr, false));
+  // run_layer with residual = false reads hidden and writes nothing to it; its
+  // scan stores H every 16 positions for the scan gradient where it can
+  float* hck = (float*)(ws + q.hck);
+  int hck_written = 0;
+  R2L_TRY(run_layer<bf16>((bf16*)const_cast<void*>(hidden), w, p, g, B, L, ws, st, nullptr, nullptr, false, nullptr,
+                          hck, &hck_written));
   const bf16* xz = (const bf16*)(ws + p.xz);
   const bf16* u = (const bf16*)(ws + p.u);
   const float* dbc = (const float*)(ws + p.dbc);
@@ -826,6 +833,7 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
     a.dA_log = gr->A_log; a.dD = gr->D; a.ddt_b = gr->dt_proj_b;
     a.B = B; a.L = L; a.E = E; a.chunk_tokens = 0; a.lengths = len;
     a.status = err;
+    a.hck = hck_written ? hck : nullptr;
     char* sw = ws + q.sbwd;
     if (cudaMemsetAsync(sw, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
     if (r2l::scan_bwd_f32(a, sw + align_up(16, kAlign), st) != cudaSuccess) return R2L_ERR_CUDA;

@@ -667,14 +667,15 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
     a.T = QS;
     a.nc = (g.L + QS - 1) / QS;
     char* p = (char*)scratch;
-    a.hcar = (float*)p; p += al((size_t)g.B * a.nc * g.E * 16 * 4);
+    a.hcar = g.hck ? const_cast<float*>(g.hck) : (float*)p;   // seq_final_kernel only reads them
+    p += al((size_t)g.B * a.nc * g.E * 16 * 4);
     a.pA = (float*)p;   p += al((size_t)g.B * g.E * 16 * 4);
     a.pD = (float*)p;   p += al((size_t)g.B * g.E * 4);
     a.pb = (float*)p;   p += al((size_t)g.B * g.E * 4);
     a.pbc = (float*)p;
     a.nbc = g.E / QC;
     const dim3 grid(g.E / QC, g.B);
-    seq_ckpt_kernel<<<grid, QT, 0, st>>>(a);
+    if (!g.hck) seq_ckpt_kernel<<<grid, QT, 0, st>>>(a);
     seq_final_kernel<<<grid, QT, 0, st>>>(a);
     seq_reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a);
     reduce_bc_kernel<<<(unsigned)((M * 32 + 255) / 256), 256, 0, st>>>(a);

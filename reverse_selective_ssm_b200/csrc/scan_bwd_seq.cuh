@@ -10,7 +10,9 @@
 // states, and the parameter sums accumulate in registers over the sequence.
 // Two launches do the work:
 //   1. seq_ckpt_kernel walks H right to left and stores it at the right end of
-//      every 16-position chunk (hck[b][k] = H_{16(k+1)}, zero past the end);
+//      every 16-position chunk (hck[b][k] = H_{16(k+1)}, zero past the end).
+//      A training-mode forward (the two-thread scan with checkpoints) stores
+//      the same states, and then this launch is skipped;
 //   2. seq_final_kernel walks the chunks left to right.  Per chunk it stages
 //      the per-(position, channel) scalars once and walks H from the
 //      checkpoint (loaded with the chunk's inputs) over positions 15 … 4, keeping
@@ -209,8 +211,12 @@ __device__ __forceinline__ void qstage(const Args& a, const QLane& l, QSmem& S, 
   const int c0 = blockIdx.x * QC;
   const int s = k * QS;
   const int q4 = threadIdx.x & 7, rr = threadIdx.x >> 3;
+  // the last chunk starts from H = 0 (nothing lies past the sequence's end);
+  // a training-mode forward leaves that checkpoint unwritten
   const float* hp = a.hcar + hck_idx(a, l, k);
-  const float4 h0 = ld4(hp), h1 = ld4(hp + 4);
+  const bool last = k == l.nck - 1;
+  const float4 h0 = last ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(hp);
+  const float4 h1 = last ? make_float4(0.f, 0.f, 0.f, 0.f) : ld4(hp + 4);
   const float4 dtb = ld4(a.dt_b + c0 + 4 * q4);
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {

@@ -106,6 +106,8 @@ struct Params {
   int force_general;
   const unsigned* a_general;  // 0: A is exactly −(1..16) (the power path), decided once per call
   int fwd;              // left-to-right block (chunk carry direction)
+  float* hck;           // training mode: H at every position 16(k+1) < len, [B][nc16][E][16] (else null)
+  int nc16;             // ⌈L/16⌉
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -111,9 +111,14 @@ cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaS
       !make_tmap_2d(&tdr, a.dr, 2, DT_R, M, a.lddr * 2, 64, TS, 128) ||
       !make_tmap_2d(&tw, a.wdt, 2, DT_R, a.E, (long long)DT_R * 2, 64, CHP, 128))
     return cudaErrorInvalidValue;
+  // training mode (p.hck): the final pass also stores the scan gradient's checkpoints
+  const bool ckpt = !FWD && p.hck != nullptr;
   cudaError_t e = cudaFuncSetAttribute(pair::scan_pair_kernel<true, FWD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sp::BYTES);
   if (e != cudaSuccess) return e;
+  if (ckpt && (e = cudaFuncSetAttribute(pair::scan_pair_kernel<true, false, true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sp::BYTES)) != cudaSuccess)
+    return e;
   const dim3 grid((a.E + CHP - 1) / CHP, nc, a.B);
   if (nc > 1) {
     if ((e = cudaFuncSetAttribute(pair::scan_pair_kernel<false, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -125,7 +130,10 @@ cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaS
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     if (launches) *launches += 2;
   }
-  pair::scan_pair_kernel<true, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+  if (ckpt)
+    pair::scan_pair_kernel<true, false, true><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+  else
+    pair::scan_pair_kernel<true, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;
@@ -205,6 +213,13 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.a_general = a.a_general;
   if (!a.force_general && !a.a_general) return cudaErrorInvalidValue;
   p.fwd = a.forward;
+  p.hck = nullptr;
+  p.nc16 = (a.L + 15) / 16;
+  if (a.hck_written) *a.hck_written = 0;
+  if (a.hck && a.dt_mma && !a.forward && R2L_SCAN_IMPL == 1) {   // only the two-thread kernel writes them
+    p.hck = a.hck;
+    if (a.hck_written) *a.hck_written = 1;
+  }
   if (a.dt_mma) {
     if (!a.dr || !a.wdt || (a.lddr % 8)) return cudaErrorInvalidValue;
     return a.forward ? launch<true, true>(a, p, nc, st, launches) : launch<true, false>(a, p, nc, st, launches);

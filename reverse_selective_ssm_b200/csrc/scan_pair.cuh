@@ -181,11 +181,13 @@ __device__ __forceinline__ void pair_decays(const PCtx& cx, float dec, float2 (&
 // outside [jlo, jhi) (a tile that crosses the chunk's start or end) leave the
 // state untouched and write nothing.  Without FINAL (the chunked scheme's
 // first pass) only the state and this thread's Σ Δ over its tokens advance.
-template <bool FINAL, bool POW, bool FULL, bool FWD>
+// CKPT (training mode): after token jck the state is stored at ck (the
+// checkpoint of the scan gradient: H at a position that is a multiple of 16).
+template <bool FINAL, bool POW, bool FULL, bool FWD, bool CKPT>
 __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float& sumd, const bf16* su, bf16* sz,
                                           bf16* yg, long long ldy, bool store_ok, int jlo, int jhi,
                                           const float (&dto)[8], uint32_t ph, uint64_t* bcready, uint64_t* bcfree,
-                                          uint32_t t_bc, unsigned* err, bool& ok) {
+                                          uint32_t t_bc, unsigned* err, bool& ok, int jck, float* ck) {
   const int lane = threadIdx.x & 31;
   const int h = lane >> 4;
   // With FINAL, u and z of this thread's tokens are read one sub-tile ahead:
@@ -270,6 +272,14 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float&
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           H[q] = __ffma2_rn(a[q], H[q], __fmul2_rn(du2, make_float2(bv[2 * q], bv[2 * q + 1])));
+        if (CKPT && j == jck) {
+          const int h = lane >> 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            ck[4 * q + h] = H[q].x;
+            ck[4 * q + 2 + h] = H[q].y;
+          }
+        }
         if (FINAL) {
           float2 acc = __fmul2_rn(make_float2(bv[8], bv[9]), H[0]);
 #pragma unroll
@@ -300,7 +310,7 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float&
   }
 }
 
-template <bool FINAL, bool POW, bool FWD>
+template <bool FINAL, bool POW, bool FWD, bool CKPT>
 __device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], float& sumd, uint8_t* smem, uint64_t* full,
                                              uint64_t* empty, uint64_t* dtready, uint64_t* bcready, uint64_t* bcfree,
                                              uint32_t tmem_base, int ntiles, int s0, int e0, int b, int c, int cl,
@@ -344,12 +354,23 @@ __device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], flo
     bf16* sz = reinterpret_cast<bf16*>(smem + S::Z) + st * TS * CHP + cl;
     bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
     const uint32_t gph = (uint32_t)it & 1u;   // each group region is used once per tile
+    // the tile's checkpoint position: its one token at a multiple of 16 (past 0)
+    int jck = -1;
+    float* ck = nullptr;
+    if (CKPT && cvalid) {
+      const int j = (16 - (((tbase % 16) + 16) % 16)) % 16;
+      const int P = tbase + j;
+      if (P >= 16 && j >= jlo && j < jhi) {
+        jck = j;
+        ck = p.hck + (((long long)b * p.nc16 + (P / 16 - 1)) * p.E + c) * 16;
+      }
+    }
     if (full_tile)
-      pair_tile<FINAL, POW, true, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready, bcfree,
-                                       t_lane + P_BC_COL0, p.err, ok);
+      pair_tile<FINAL, POW, true, FWD, CKPT>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready,
+                                             bcfree, t_lane + P_BC_COL0, p.err, ok, jck, ck);
     else
-      pair_tile<FINAL, POW, false, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready,
-                                        bcfree, t_lane + P_BC_COL0, p.err, ok);
+      pair_tile<FINAL, POW, false, FWD, CKPT>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready,
+                                              bcfree, t_lane + P_BC_COL0, p.err, ok, jck, ck);
     if (!ok) break;
     if (FINAL && full_tile) sm100::fence_proxy_async_smem();   // y tile visible to the TMA store
     sm100::tc_fence_before();
@@ -362,7 +383,7 @@ __device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], flo
 // FINAL: y, starting from the carried state H_in(k) when sequences are split
 // (zero with one chunk).  Otherwise the chunked scheme's first pass: the
 // chunk's end state from a zero start and Σ Δ over it, into the carry buffer.
-template <bool FINAL, bool FWD>
+template <bool FINAL, bool FWD, bool CKPT = false>
 __global__ void __launch_bounds__(SmemPair::THREADS, 1)
 scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_z,
                  const __grid_constant__ CUtensorMap tm_dr, const __grid_constant__ CUtensorMap tm_bc,
@@ -466,11 +487,11 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
     H[kk] = (FINAL && cst) ? make_float2(cst[4 * kk + h], cst[4 * kk + 2 + h]) : make_float2(0.0f, 0.0f);
   float sumd = 0.0f;
   if (use_pow)
-    pair_compute<FINAL, true, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
-                                   e0, b, c, cl, cvalid, p);
+    pair_compute<FINAL, true, FWD, CKPT>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles,
+                                         s0, e0, b, c, cl, cvalid, p);
   else
-    pair_compute<FINAL, false, FWD>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base, ntiles, s0,
-                                    e0, b, c, cl, cvalid, p);
+    pair_compute<FINAL, false, FWD, CKPT>(cx, H, sumd, smem, full, empty, dtready, bcready, bcfree, tmem_base,
+                                          ntiles, s0, e0, b, c, cl, cvalid, p);
   if (!FINAL) {
     // chunk end state S_k and Σ Δ (each thread summed Δ over its own tokens)
     const float total = sumd + __shfl_xor_sync(0xffffffffu, sumd, 16);

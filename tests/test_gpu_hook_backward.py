@@ -145,6 +145,19 @@ def test_hook_backward_odd_sizes():
             ds_check=(0.9, dh_out, lengths) + hh)
 
 
+def test_hook_backward_batch_of_eight():
+    """B = 8 × L = 96 at workload-1 widths: at batch 8 the scan gradient walks
+    each sequence in one block, from the H checkpoints that the recomputed
+    forward scan stores every 16 positions.  Ragged lengths end checkpoint
+    chunks part-way; one sequence has a single position."""
+    lengths = torch.tensor([96, 17, 64, 1, 80, 33, 96, 48], dtype=torch.int32)
+    dims, h, w, dh_out = make(8, 96, seed=87, lengths=lengths)
+    got = run_gpu(dims, h, w, 0.6, dh_out, lengths)
+    hh = hhat_pair(dims, h, w, 0.6, lengths)
+    compare(got, run_oracle(h, w, 0.6, dh_out, lengths), h, dh_out, lengths,
+            ds_check=(0.6, dh_out, lengths) + hh)
+
+
 def test_hook_backward_without_layernorm():
     """No LayerNorm (ĥ = o), s = −1.2, one sequence of 128."""
     dims, h, w, dh_out = make(1, 128, seed=82, ln="none")
