@@ -444,11 +444,11 @@ __global__ void __launch_bounds__(256) conv_bwd_kernel(
     rows(std::true_type{});
   else
     rows(std::false_type{});
-  // the transpose: rows r0 … r0+15 of channels c and c+1 (zero past M, up to ldT)
+  // the transpose (when asked for): rows r0 … r0+15 of channels c and c+1 (zero past M, up to ldT)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const long long m = r0 + 8 * h;
-    if (live && m < ldT) {
+    if (dxzT != nullptr && live && m < ldT) {
       *reinterpret_cast<uint4*>(dxzT + (long long)c * ldT + m) =
           make_uint4(packA[4 * h], packA[4 * h + 1], packA[4 * h + 2], packA[4 * h + 3]);
       *reinterpret_cast<uint4*>(dxzT + (long long)(c + 1) * ldT + m) =
@@ -470,6 +470,22 @@ __global__ void __launch_bounds__(256) conv_bwd_kernel(
       acc.y += red[(gq * 64 + p) * 5 + k].y;
     }
     *reinterpret_cast<float2*>(part + ((long long)blockIdx.y * 5 + k) * E + c) = acc;
+  }
+}
+
+// Rows i ≥ len_b of sequence b of a bf16 [B·L, cols] array (row stride ld)
+// set to zero: one block per sequence, 16-byte stores (cols a multiple of 8).
+// Activations the weight-gradient GEMMs read position-major must be finite
+// on padding rows, where the gradient operand is zero.
+__global__ void __launch_bounds__(256) zero_padding_rows_kernel(bf16* __restrict__ x, long long ld, int cols,
+                                                                const int* __restrict__ len, int L) {
+  const int b = blockIdx.x;
+  const int n = len[b];
+  const int c8 = cols / 8;
+  const long long rows = (long long)(L - n) * c8;
+  for (long long t = threadIdx.x; t < rows; t += blockDim.x) {
+    const long long m = (long long)b * L + n + t / c8;
+    *reinterpret_cast<uint4*>(x + m * ld + 8 * (t % c8)) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

@@ -140,7 +140,12 @@ __device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[
 // `splits` slices of Mp rows, Mp = M rounded up to whole tiles), and a
 // separate kernel adds the slices in a fixed order.  For short, wide-K GEMMs
 // with fewer tiles than SMs.
-template <int BN, typename TOut, int MB = 1>
+// AMN / BMN: A (B) is stored MN-major, as [K, M] ([K, N]) with the M (N)
+// index contiguous; it is loaded in boxes of 64 MN elements × 64 K rows and
+// read through the MN-major descriptor.  The weight gradients of the
+// projections contract over positions, and their operands are activations
+// and gradients stored position-major, i.e. MN-major.
+template <int BN, typename TOut, int MB = 1, int AMN = 0, int BMN = 0>
 __global__ void __launch_bounds__(TcGemmCfg<BN, TOut, MB>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, bf16* __restrict__ C2, int ldc2, int c2_cols,
@@ -148,6 +153,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                int splits) {
   using Cfg = TcGemmCfg<BN, TOut, MB>;
   constexpr int BM = Cfg::BM, BK = Cfg::BK, STAGES = Cfg::STAGES, NACC = Cfg::NACC;
+  static_assert(!BMN || BN % 64 == 0, "an MN-major B tile is whole 64-column boxes");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -213,8 +219,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!sm100::mbar_wait(&empty[stage], phase ^ 1u, err)) { ok = false; break; }
           sm100::mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          sm100::tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
-          sm100::tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+          if (AMN) {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i)
+              sm100::tma_load_2d(sA + stage * Cfg::A_BYTES + i * 8192, &tmA, mb * BM + 64 * i, kb * BK, &full[stage]);
+          } else {
+            sm100::tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
+          }
+          if (BMN) {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i)
+              sm100::tma_load_2d(sB + stage * Cfg::B_BYTES + i * 8192, &tmB, nb * BN + 64 * i, kb * BK, &full[stage]);
+          } else {
+            sm100::tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+          }
           ++issued[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -227,7 +245,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = sm100::idesc_bf16_f32(128, BN);
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32_mn(128, BN, AMN != 0, BMN != 0);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -247,9 +265,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
 #pragma unroll
-            for (int mb = 0; mb < MB; ++mb)   // rows 128·mb …: accumulator columns [BN·mb, BN·mb + BN)
-              sm100::mma_bf16(d_tmem + (uint32_t)(mb * BN), sm100::smem_desc_k128(a0 + mb * (128 * 128) + k * 32),
-                              sm100::smem_desc_k128(b0 + k * 32), idesc, (kb != kb0) | (k != 0));
+            for (int mb = 0; mb < MB; ++mb) {  // rows 128·mb …: accumulator columns [BN·mb, BN·mb + BN)
+              // K-major: 16 K elements are 32 bytes along a 128-byte row; MN-major:
+              // 16 K rows are two 1024-byte atoms, and 128 M rows are two 8 KB boxes
+              const uint64_t da = AMN ? sm100::smem_desc_mn128(a0 + mb * (2 * 8192) + k * 2048)
+                                      : sm100::smem_desc_k128(a0 + mb * (128 * 128) + k * 32);
+              const uint64_t db = BMN ? sm100::smem_desc_mn128(b0 + k * 2048) : sm100::smem_desc_k128(b0 + k * 32);
+              sm100::mma_bf16(d_tmem + (uint32_t)(mb * BN), da, db, idesc, (kb != kb0) | (k != 0));
+            }
           }
           sm100::mma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

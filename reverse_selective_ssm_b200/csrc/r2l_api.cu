@@ -632,7 +632,7 @@ struct BwdPlan {
   Plan f;                                        // the forward's regions
   long long Mp;                                  // positions rounded up to 8 (K of the weight gradients)
   size_t dt32, winT, woutT, wxT, wdtT, stats, dsrow, do16, lnpart, dy, doT, yT, dus, dz, ddt, dbcs, sbwd, sbwd_bytes,
-      ddt16, ddtT, drT, ddr, ddbc16, ddbcT, uT, dux, cpart, dxz16, dxzT, hT, dhtmp, gpart, gpart_bytes, hck, total;
+      ddt16, ddr, ddbc16, dux, cpart, dxz16, hT, dhtmp, gpart, gpart_bytes, hck, total;
 };
 
 long long row_chunks(long long M) { return (M + r2l::bwd::ROW_CHUNK - 1) / r2l::bwd::ROW_CHUNK; }
@@ -656,8 +656,6 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   q->do16 = take(M * d * 2);
   q->lnpart = take((size_t)row_chunks(p.M) * 2 * d * 4);
   q->dy = take(M * E * 4);
-  q->doT = take(d * Mp * 2);
-  q->yT = take(E * Mp * 2);
   q->dus = take(M * E * 4);
   q->dz = take(M * E * 4);
   q->ddt = take(M * E * 4);
@@ -668,16 +666,11 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   if (q->sbwd_bytes == 0) return false;
   q->sbwd = take(q->sbwd_bytes);
   q->ddt16 = take(M * E * 2);
-  q->ddtT = take(E * Mp * 2);
-  q->drT = take(R * Mp * 2);
   q->ddr = take(M * R * 4);
   q->ddbc16 = take(M * ldd * 2);
-  q->ddbcT = take(ldd * Mp * 2);
-  q->uT = take(E * Mp * 2);
   q->dux = take(M * E * 4);
   q->cpart = take((size_t)row_chunks(p.M) * 5 * E * 4);
   q->dxz16 = take(M * 2 * E * 2);
-  q->dxzT = take(2 * E * Mp * 2);
   q->hT = take(d * Mp * 2);
   q->dhtmp = take(M * d * 4);
   // split-K scratch: the largest any fp32-output GEMM below asks for
@@ -685,13 +678,13 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   auto need = [&](long long m, int n, int k) { gp = std::max(gp, r2l::tc_gemm_partial_bytes(m, n, k)); };
   need(p.M, p.E, p.R);                 // dt_raw
   need(p.M, p.E, p.d);                 // dy
-  need(p.d, p.E, (int)q->Mp);          // dW_out
+  need(p.d, p.E, (int)p.M);            // dW_out
   need(p.M, p.R, p.E);                 // dΔr
-  need(p.E, p.R, (int)q->Mp);          // dW_dt
+  need(p.E, p.R, (int)p.M);            // dW_dt
   need(p.M, p.E, p.ldd);               // du_x
-  need(p.ldd, p.E, (int)q->Mp);        // dW_x
+  need(p.ldd, p.E, (int)p.M);          // dW_x
   need(p.M, p.d, 2 * p.E);             // dh
-  need(2LL * p.E, p.d, (int)q->Mp);    // dW_in
+  need(2LL * p.E, p.d, (int)p.M);      // dW_in
   q->gpart_bytes = gp;
   q->gpart = take(gp);
   q->total = off;
@@ -718,11 +711,14 @@ r2l_status transpose(const TIn* in, long long ld_in, long long M, int C, bf16* o
   return cvt_transpose<TIn>(in, ld_in, M, C, nullptr, 0, outT, ldT, len, L, st);
 }
 
-// C[m, n] = Σ_k A[m, k]·B[n, k], bf16 operands, fp32 result.
+// C[m, n] = Σ_k A[m, k]·B[n, k], bf16 operands, fp32 result.  a_mn / b_mn: A
+// stored [K, M] / B stored [K, N] (position-major operands of a weight gradient).
 r2l_status gemm_f32(const bf16* A, int lda, const bf16* Bm, int ldb, float* C, int ldc, long long M, int N, int K,
-                    const int* len, int L, unsigned* err, float* partial, size_t partial_bytes, cudaStream_t st) {
+                    const int* len, int L, unsigned* err, float* partial, size_t partial_bytes, cudaStream_t st,
+                    bool a_mn = false, bool b_mn = false) {
   r2l::TcGemm g{};
   g.A = A; g.lda = lda; g.B = Bm; g.ldb = ldb; g.C = C; g.ldc = ldc; g.c_fp32 = true;
+  g.a_mn = a_mn; g.b_mn = b_mn;
   g.M = (int)M; g.N = N; g.K = K; g.len = len; g.L = L; g.err = err;
   g.partial = partial; g.partial_bytes = partial_bytes;
   return r2l::tc_gemm(g, st) == cudaSuccess ? R2L_OK : R2L_ERR_CUDA;
@@ -814,11 +810,13 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   // ---- out_proj: dy = do·W_out, dW_out = doᵀ·y
   float* dy = (float*)(ws + q.dy);
   R2L_TRY(gemm_f32(do16, d, woutT, d, dy, E, M, E, d, len, L, err, gpart, gpb, st));
-  bf16* doT = (bf16*)(ws + q.doT);
-  bf16* yT = (bf16*)(ws + q.yT);
-  R2L_TRY(transpose(do16, d, M, d, doT, Mp, len, L, st));
-  R2L_TRY(transpose(y, E, M, E, yT, Mp, len, L, st));
-  R2L_TRY(gemm_f32(doT, (int)Mp, yT, (int)Mp, gr->out_proj_w, E, d, E, (int)Mp, nullptr, d, err, gpart, gpb, st));
+  // the weight gradients read their operands position-major (MN-major); the
+  // gradient side is zero on padding rows, the activation side is zeroed there
+  K::zero_padding_rows_kernel<<<B, 256, 0, st>>>(const_cast<bf16*>(y), E, E, len, L);
+  K::zero_padding_rows_kernel<<<B, 256, 0, st>>>(const_cast<bf16*>(u), E, E, len, L);
+  K::zero_padding_rows_kernel<<<B, 256, 0, st>>>(const_cast<bf16*>(dr), R, R, len, L);
+  R2L_LAUNCH_CHECK();
+  R2L_TRY(gemm_f32(do16, d, y, E, gr->out_proj_w, E, d, E, (int)M, nullptr, d, err, gpart, gpb, st, true, true));
 
   // ---- ❷ the scan (bf16 u and z, fp32 dt_raw, B|C and dy)
   float* dus = (float*)(ws + q.dus);
@@ -841,51 +839,46 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
 
   // ---- dt_proj: dΔr = ddt_raw·W_dt, dW_dt = ddt_rawᵀ·Δr
   bf16* ddt16 = (bf16*)(ws + q.ddt16);
-  bf16* ddtT = (bf16*)(ws + q.ddtT);
-  R2L_TRY(cvt_transpose(ddt, E, M, E, ddt16, E, ddtT, Mp, len, L, st));
+  R2L_TRY(cvt_transpose(ddt, E, M, E, ddt16, E, (bf16*)nullptr, 0, len, L, st));
   float* ddr = (float*)(ws + q.ddr);
   R2L_TRY(gemm_f32(ddt16, E, wdtT, E, ddr, R, M, R, E, len, L, err, gpart, gpb, st));
-  bf16* drT = (bf16*)(ws + q.drT);
-  R2L_TRY(transpose(dr, R, M, R, drT, Mp, len, L, st));
-  R2L_TRY(gemm_f32(ddtT, (int)Mp, drT, (int)Mp, gr->dt_proj_w, R, E, R, (int)Mp, nullptr, E, err, gpart, gpb, st));
+  R2L_TRY(gemm_f32(ddt16, E, dr, R, gr->dt_proj_w, R, E, R, (int)M, nullptr, E, err, gpart, gpb, st, true, true));
 
   // ---- x_proj: d[Δr|B|C] → du_x = d[Δr|B|C]·W_x, dW_x = d[Δr|B|C]ᵀ·u
   bf16* ddbc16 = (bf16*)(ws + q.ddbc16);
-  bf16* ddbcT = (bf16*)(ws + q.ddbcT);
-  R2L_TRY(cvt_transpose(ddr, R, M, R, ddbc16, ldd, ddbcT, Mp, len, L, st));
-  R2L_TRY(cvt_transpose(dbcs, 2LL * p.N, M, 2 * p.N, ddbc16 + R, ldd, ddbcT + (size_t)R * Mp, Mp, len, L, st));
+  R2L_TRY(cvt_transpose(ddr, R, M, R, ddbc16, ldd, (bf16*)nullptr, 0, len, L, st));
+  R2L_TRY(cvt_transpose(dbcs, 2LL * p.N, M, 2 * p.N, ddbc16 + R, ldd, (bf16*)nullptr, 0, len, L, st));
   float* dux = (float*)(ws + q.dux);
   R2L_TRY(gemm_f32(ddbc16, ldd, wxT, ldd, dux, E, M, E, ldd, len, L, err, gpart, gpb, st));
-  bf16* uT = (bf16*)(ws + q.uT);
-  R2L_TRY(transpose(u, E, M, E, uT, Mp, len, L, st));
-  R2L_TRY(gemm_f32(ddbcT, (int)Mp, uT, (int)Mp, gr->x_proj_w, E, ldd, E, (int)Mp, nullptr, ldd, err, gpart, gpb,
-                   st));
+  R2L_TRY(gemm_f32(ddbc16, ldd, u, E, gr->x_proj_w, E, ldd, E, (int)M, nullptr, ldd, err, gpart, gpb, st, true,
+                   true));
 
-  // ---- conv + SiLU: dx (into dxz and dxzᵀ), dconv_w, dconv_b; dz into dxz and dxzᵀ
+  // ---- conv + SiLU: dx (into dxz), dconv_w, dconv_b; dz into dxz
   bf16* dxz16 = (bf16*)(ws + q.dxz16);
-  bf16* dxzT = (bf16*)(ws + q.dxzT);
   float* cpart = (float*)(ws + q.cpart);
   if (cudaFuncSetAttribute(K::conv_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::CONV_SMEM) !=
       cudaSuccess)
     return R2L_ERR_CUDA;
   K::conv_bwd_kernel<<<dim3((unsigned)((E + K::CONV_CH - 1) / K::CONV_CH), (unsigned)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS)),
-                       256, K::CONV_SMEM, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E, len, L, M, dxz16, 2LL * E, dxzT, Mp,
+                       256, K::CONV_SMEM, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E, len, L, M, dxz16, 2LL * E, nullptr, Mp,
                                      cpart);
   R2L_LAUNCH_CHECK();
   K::chunk_sum_kernel<1><<<(5 * E + 31) / 32, 256, 0, st>>>(cpart, (int)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS), 5 * E,
                                                             E, gr->conv_w, gr->conv_b);
   R2L_LAUNCH_CHECK();
-  R2L_TRY(cvt_transpose(dz, E, M, E, dxz16 + E, 2LL * E, dxzT + (size_t)E * Mp, Mp, len, L, st));
+  R2L_TRY(cvt_transpose(dz, E, M, E, dxz16 + E, 2LL * E, (bf16*)nullptr, 0, len, L, st));
 
   // ---- in_proj: dh = dh⁺ + [dx | dz]·W_in, dW_in = [dx | dz]ᵀ·h
   float* dhtmp = (float*)(ws + q.dhtmp);
   R2L_TRY(gemm_f32(dxz16, 2 * E, winT, 2 * E, dhtmp, d, M, d, 2 * E, len, L, err, gpart, gpb, st));
   K::add_rows_kernel<<<(unsigned)std::min<long long>(M, 148 * 8), 256, 0, st>>>(dh_out, dhtmp, d, len, L, M, dh);
   R2L_LAUNCH_CHECK();
+  // h is the caller's (its padding rows may hold anything): transposed with
+  // padding zeroed, and read K-major
   bf16* hT = (bf16*)(ws + q.hT);
   R2L_TRY(transpose((const bf16*)hidden, d, M, d, hT, Mp, len, L, st));
-  R2L_TRY(gemm_f32(dxzT, (int)Mp, hT, (int)Mp, gr->in_proj_w, d, 2LL * E, d, (int)Mp, nullptr, 2 * E, err, gpart,
-                   gpb, st));
+  R2L_TRY(gemm_f32(dxz16, 2 * E, hT, (int)Mp, gr->in_proj_w, d, 2LL * E, d, (int)M, nullptr, 2 * E, err, gpart, gpb,
+                   st, true, false));
   return R2L_OK;
 }
 

@@ -170,6 +170,23 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major tile written by TMA with
+// 128-byte swizzle in boxes of 64 MN elements × 64 K rows: each K row holds 64
+// consecutive MN elements (128 bytes), 8 K rows form a 1024-byte swizzle atom,
+// and the boxes of successive 64-element MN blocks follow each other.  Fields
+// as for the K-major form, with the leading byte offset = the stride between
+// 64-element MN blocks (one box, 8 KB) and the stride byte offset = the stride
+// between 8-row groups along K (1024 bytes).
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(8192u >> 4) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
 // Shared-memory matrix descriptor for a K-major operand without swizzle: 8-row
 // core matrices of 16 bytes per row (128 contiguous bytes), `lbo` bytes
 // between the core matrices adjacent along K, `sbo` bytes between the 8-row
@@ -207,6 +224,12 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
 // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same with A and/or B MN-major (bits 15 and 16: the operand is stored
+// transposed, its M or N index contiguous).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
 }
 
 // 32 lanes x 16 consecutive fp32 columns of TMEM into registers (one row per

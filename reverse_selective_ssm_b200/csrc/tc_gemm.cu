@@ -69,15 +69,20 @@ int choose_splits(long long tiles, int num_k) {
   return (num_k + kps - 1) / kps;
 }
 
-template <int BN, typename TOut, int MB = 1>
+template <int BN, typename TOut, int MB = 1, int AMN = 0, int BMN = 0>
 cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   using Cfg = TcGemmCfg<BN, TOut, MB>;
   CUtensorMap ta, tb, tc;
-  if (!make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, 128)) return cudaErrorInvalidValue;
+  // K-major: boxes of 64 K × BM (BN) rows; MN-major: boxes of 64 M (N) × 64 K rows
+  if (AMN ? !make_tmap_2d(&ta, g.A, 2, g.M, g.K, (long long)g.lda * 2, 64, Cfg::BK, 128)
+          : !make_tmap_2d(&ta, g.A, 2, g.K, g.M, (long long)g.lda * 2, Cfg::BK, Cfg::BM, 128))
+    return cudaErrorInvalidValue;
+  if (BMN ? !make_tmap_2d(&tb, g.B, 2, g.N, g.K, (long long)g.ldb * 2, 64, Cfg::BK, 128)
+          : !make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, 128))
+    return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tc, g.C, (int)sizeof(TOut), g.N, g.M, (long long)g.ldc * sizeof(TOut), 32, 32, Cfg::STG_SWIZZLE))
     return cudaErrorInvalidValue;
-  auto kern = gemm_tc_kernel<BN, TOut, MB>;
+  auto kern = gemm_tc_kernel<BN, TOut, MB, AMN, BMN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const long long num_m = (g.M + Cfg::BM - 1) / Cfg::BM;
@@ -125,6 +130,22 @@ cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
   return launch<256, TOut>(g, st);
 }
 
+// fp32-output GEMMs with MN-major operands (the weight gradients): the tile
+// width as dispatch() picks it, in whole 64-column boxes when B is MN-major.
+template <int AMN, int BMN>
+cudaError_t dispatch_mn(const TcGemm& g, cudaStream_t st) {
+  if (g.N % 256 == 0) {
+    if ((long long)((g.M + 127) / 128) * (g.N / 256) < sm_count()) return launch<128, float, 1, AMN, BMN>(g, st);
+    return launch<256, float, 1, AMN, BMN>(g, st);
+  }
+  if (g.N <= 64) return launch<64, float, 1, AMN, BMN>(g, st);
+  if (g.N <= 128) return launch<128, float, 1, AMN, BMN>(g, st);
+  if constexpr (!BMN)
+    if (g.N <= 160) return launch<160, float, 1, AMN, BMN>(g, st);
+  if (g.N % 128 == 0) return launch<128, float, 1, AMN, BMN>(g, st);
+  return launch<256, float, 1, AMN, BMN>(g, st);
+}
+
 template <bool FWD>
 cudaError_t launch_convx(const ConvX& g, cudaStream_t st) {
   namespace cx = convx;
@@ -170,8 +191,13 @@ cudaError_t convx_gemm(const ConvX& g, cudaStream_t st) {
 
 cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;
-  if ((g.lda % 8) || (g.ldb % 8) || (g.K % 8)) return cudaErrorInvalidValue;  // TMA: 16-byte strides
+  // TMA: 16-byte row strides; a K-major operand's K is its inner extent
+  if ((g.lda % 8) || (g.ldb % 8) || (!g.a_mn && (g.K % 8))) return cudaErrorInvalidValue;
   if ((g.ldc * (g.c_fp32 ? 4 : 2)) % 16) return cudaErrorInvalidValue;
+  if (g.a_mn || g.b_mn) {
+    if (!g.c_fp32 || !g.a_mn || g.C2) return cudaErrorInvalidValue;
+    return g.b_mn ? dispatch_mn<1, 1>(g, st) : dispatch_mn<1, 0>(g, st);
+  }
   return g.c_fp32 ? dispatch<float>(g, st) : dispatch<bf16>(g, st);
 }
 

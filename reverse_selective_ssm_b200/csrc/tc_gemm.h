@@ -7,10 +7,13 @@
 namespace r2l {
 
 struct TcGemm {
-  const __nv_bfloat16* A;  // [M, K] row stride lda (elements), 16-byte aligned
+  const __nv_bfloat16* A;  // [M, K] row stride lda (elements), 16-byte aligned; [K, M] when a_mn
   int lda;
-  const __nv_bfloat16* B;  // [N, K] row stride ldb
+  const __nv_bfloat16* B;  // [N, K] row stride ldb; [K, N] when b_mn
   int ldb;
+  // MN-major operands (fp32 C only): A stored [K, M], B stored [K, N], rows of
+  // stride lda / ldb.  Supported: a_mn alone, or a_mn with b_mn.
+  bool a_mn, b_mn;
   void* C;                 // [M, N] row stride ldc; bf16, or fp32 when c_fp32
   int ldc;
   bool c_fp32;
