@@ -921,17 +921,18 @@ def hook_bwd_gemm_flops(case):
 def hook_bwd_launches(case):
     """Kernels one r2l_sidecar_backward call launches at the bench's shapes
     (as the ncu launch list shows them): the recomputed forward (6, its scan
-    storing the scan gradient's H checkpoints) and dt_raw,
-    4 weight transposes, the gate and LayerNorm gradient (4, or 2 without
-    LayerNorm), the scan gradient, and per projection its input-gradient GEMM,
-    weight-gradient GEMM (dt_proj and x_proj with a split-K sum) and operand
-    conversions, the conv gradient and its column sum, and dh = dh+ + dx."""
+    storing the scan gradient's H checkpoints) and dt_raw, 4 weight
+    transposes, the gate and LayerNorm gradient (4, or 2 without LayerNorm),
+    the scan gradient, and 21 more: the padding rows of 3 activations zeroed,
+    per projection its input-gradient and weight-gradient GEMMs (dt_proj and
+    x_proj with a split-K sum) and operand conversions, the conv gradient and
+    its column sum, dh = dh+ + dx, and h transposed."""
     w = case.weights[0]
     ln = 4 if w.get("ln_w") is not None else 2
-    # on the walk along each sequence the recomputed forward scan stores the H
-    # checkpoints, so the gradient skips its own checkpoint pass
-    scan = bwd_launches(case.B, case.dims.d_inner) - (1 if bwd_walks_sequences(case.B, case.dims.d_inner) else 0)
-    return 6 + 1 + 4 + ln + scan + 22
+    # (on the walk along each sequence the recomputed forward scan stores the H
+    # checkpoints of sequences whose length is a multiple of 16, and the
+    # gradient's checkpoint pass launches but fills only the others)
+    return 6 + 1 + 4 + ln + bwd_launches(case.B, case.dims.d_inner) + 21
 
 
 def run_hook_backward(args, rank, world, local_rank):

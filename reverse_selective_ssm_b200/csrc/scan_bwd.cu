@@ -86,6 +86,7 @@ struct Args {
   float* pb;               // [B][nc][E]
   float* pbc;              // [E/CPB][B·L][32] per-block partial dB | dC
   int nbc;                 // channel blocks in pbc
+  int ckpt_ragged_only;    // the checkpoint pass skips sequences whose length is a multiple of 16
   uint32_t lnbits[16];     // float log(1) … log(16): the power-path A_log
 };
 
@@ -667,7 +668,8 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
     a.T = QS;
     a.nc = (g.L + QS - 1) / QS;
     char* p = (char*)scratch;
-    a.hcar = g.hck ? const_cast<float*>(g.hck) : (float*)p;   // seq_final_kernel only reads them
+    a.hcar = g.hck ? g.hck : (float*)p;
+    a.ckpt_ragged_only = g.hck ? 1 : 0;
     p += al((size_t)g.B * a.nc * g.E * 16 * 4);
     a.pA = (float*)p;   p += al((size_t)g.B * g.E * 16 * 4);
     a.pD = (float*)p;   p += al((size_t)g.B * g.E * 4);
@@ -675,7 +677,7 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
     a.pbc = (float*)p;
     a.nbc = g.E / QC;
     const dim3 grid(g.E / QC, g.B);
-    if (!g.hck) seq_ckpt_kernel<<<grid, QT, 0, st>>>(a);
+    seq_ckpt_kernel<<<grid, QT, 0, st>>>(a);
     seq_final_kernel<<<grid, QT, 0, st>>>(a);
     seq_reduce_params_kernel<<<(unsigned)((g.E * 16 + 255) / 256), 256, 0, st>>>(a);
     reduce_bc_kernel<<<(unsigned)((M * 32 + 255) / 256), 256, 0, st>>>(a);

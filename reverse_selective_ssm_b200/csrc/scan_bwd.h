@@ -19,10 +19,12 @@ struct ScanBwdArgs {
   int B, L, E, chunk_tokens;
   const int* lengths;   // device [B] or null
   unsigned* status;     // device status word (R2L_DEVFLAG_* bits)
-  // H at every position 16(k+1) < len, [B][⌈L/16⌉][E][16], stored by a
-  // training-mode forward (null: the gradient computes them); read by the walk
-  // along each sequence only
-  const float* hck;
+  // [B][⌈L/16⌉][E][16]: H at every position 16(k+1) < len, which a
+  // training-mode forward has stored for every sequence whose length is a
+  // multiple of 16; the gradient computes the other sequences' into it (null:
+  // it computes all of them in its own scratch).  Used by the walk along each
+  // sequence only.
+  float* hck;
 };
 
 int scan_bwd_chunk_tokens(int chunk_tokens);

@@ -12,7 +12,8 @@
 //   1. seq_ckpt_kernel walks H right to left and stores it at the right end of
 //      every 16-position chunk (hck[b][k] = H_{16(k+1)}, zero past the end).
 //      A training-mode forward (the two-thread scan with checkpoints) stores
-//      the same states, and then this launch is skipped;
+//      the same states for every sequence whose length is a multiple of 16,
+//      and then this launch only fills in the other sequences;
 //   2. seq_final_kernel walks the chunks left to right.  Per chunk it stages
 //      the per-(position, channel) scalars once and walks H from the
 //      checkpoint (loaded with the chunk's inputs) over positions 15 … 4, keeping
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(QT, QMINB) seq_ckpt_kernel(const Args a) {
   __shared__ float4 bs[2][QS][4];       // B
   bool pow;
   const QLane l = qlane(a, pow);
+  if (a.ckpt_ragged_only && l.n % QS == 0) return;    // stored by the training-mode forward
   const int c0 = blockIdx.x * QC;
   const int q4 = threadIdx.x & 7, rr = threadIdx.x >> 3;
   const float4 dtb = ld4(a.dt_b + c0 + 4 * q4);

@@ -32,8 +32,9 @@ struct ScanArgs {
   int dt_mma;                                  // compute dt_raw = Δr·W_dtᵀ inside the scan (dt_rank 128)
   int forward;                                 // left-to-right block
   // training mode: H at every position 16(k+1) < len into hck[B][⌈L/16⌉][E][16]
-  // (the scan gradient's checkpoints).  Only the two-thread kernel (right to
-  // left, dt_proj fused) writes them; *hck_written (when set) says whether it did.
+  // (the scan gradient's checkpoints), for every sequence whose length is a
+  // multiple of 16.  Only the two-thread kernel (right to left, dt_proj fused)
+  // writes them; *hck_written (when set) says whether it did.
   float* hck;
   int* hck_written;
 };

@@ -181,13 +181,11 @@ __device__ __forceinline__ void pair_decays(const PCtx& cx, float dec, float2 (&
 // outside [jlo, jhi) (a tile that crosses the chunk's start or end) leave the
 // state untouched and write nothing.  Without FINAL (the chunked scheme's
 // first pass) only the state and this thread's Σ Δ over its tokens advance.
-// CKPT (training mode): after token jck the state is stored at ck (the
-// checkpoint of the scan gradient: H at a position that is a multiple of 16).
-template <bool FINAL, bool POW, bool FULL, bool FWD, bool CKPT>
+template <bool FINAL, bool POW, bool FULL, bool FWD>
 __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float& sumd, const bf16* su, bf16* sz,
                                           bf16* yg, long long ldy, bool store_ok, int jlo, int jhi,
                                           const float (&dto)[8], uint32_t ph, uint64_t* bcready, uint64_t* bcfree,
-                                          uint32_t t_bc, unsigned* err, bool& ok, int jck, float* ck) {
+                                          uint32_t t_bc, unsigned* err, bool& ok) {
   const int lane = threadIdx.x & 31;
   const int h = lane >> 4;
   // With FINAL, u and z of this thread's tokens are read one sub-tile ahead:
@@ -272,14 +270,6 @@ __device__ __forceinline__ void pair_tile(const PCtx& cx, float2 (&H)[4], float&
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           H[q] = __ffma2_rn(a[q], H[q], __fmul2_rn(du2, make_float2(bv[2 * q], bv[2 * q + 1])));
-        if (CKPT && j == jck) {
-          const int h = lane >> 4;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            ck[4 * q + h] = H[q].x;
-            ck[4 * q + 2 + h] = H[q].y;
-          }
-        }
         if (FINAL) {
           float2 acc = __fmul2_rn(make_float2(bv[8], bv[9]), H[0]);
 #pragma unroll
@@ -354,23 +344,33 @@ __device__ __forceinline__ void pair_compute(const PCtx& cx, float2 (&H)[4], flo
     bf16* sz = reinterpret_cast<bf16*>(smem + S::Z) + st * TS * CHP + cl;
     bf16* yg = p.y + ((long long)b * p.L + tbase) * p.ldy + c;
     const uint32_t gph = (uint32_t)it & 1u;   // each group region is used once per tile
-    // the tile's checkpoint position: its one token at a multiple of 16 (past 0)
-    int jck = -1;
-    float* ck = nullptr;
-    if (CKPT && cvalid) {
-      const int j = (16 - (((tbase % 16) + 16) % 16)) % 16;
-      const int P = tbase + j;
-      if (P >= 16 && j >= jlo && j < jhi) {
-        jck = j;
-        ck = p.hck + (((long long)b * p.nc16 + (P / 16 - 1)) * p.E + c) * 16;
+    if (full_tile)
+      pair_tile<FINAL, POW, true, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready, bcfree,
+                                       t_lane + P_BC_COL0, p.err, ok);
+    else
+      pair_tile<FINAL, POW, false, FWD>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready,
+                                        bcfree, t_lane + P_BC_COL0, p.err, ok);
+    // training mode: when the chunk ends at a multiple of 16 (the sequence's
+    // length is one), every tile starts at one, and the state after the tile
+    // is the scan gradient's checkpoint H_tbase.  Thread h holds the states
+    // 4q + 2e + h; one exchange with the partner (lane ± 16) gives it the 8
+    // consecutive states 8h … 8h+7, stored as two 16-byte vectors.
+    if (CKPT && ok && (e0 % 16) == 0 && tbase >= 16) {
+      const int h = lane >> 4;
+      const float2 s0 = h ? H[0] : H[2], s1 = h ? H[1] : H[3];
+      float r[4];
+      r[0] = __shfl_xor_sync(0xffffffffu, s0.x, 16);
+      r[1] = __shfl_xor_sync(0xffffffffu, s0.y, 16);
+      r[2] = __shfl_xor_sync(0xffffffffu, s1.x, 16);
+      r[3] = __shfl_xor_sync(0xffffffffu, s1.y, 16);
+      if (cvalid) {
+        const float2 k0 = h ? H[2] : H[0], k1 = h ? H[3] : H[1];
+        float4* d4 = reinterpret_cast<float4*>(p.hck + (((long long)b * p.nc16 + (tbase / 16 - 1)) * p.E + c) * 16 +
+                                               8 * h);
+        d4[0] = h ? make_float4(r[0], k0.x, r[1], k0.y) : make_float4(k0.x, r[0], k0.y, r[1]);
+        d4[1] = h ? make_float4(r[2], k1.x, r[3], k1.y) : make_float4(k1.x, r[2], k1.y, r[3]);
       }
     }
-    if (full_tile)
-      pair_tile<FINAL, POW, true, FWD, CKPT>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, 0, TS, dto, gph, bcready,
-                                             bcfree, t_lane + P_BC_COL0, p.err, ok, jck, ck);
-    else
-      pair_tile<FINAL, POW, false, FWD, CKPT>(cx, H, sumd, su, sz, yg, p.ldy, cvalid, jlo, jhi, dto, gph, bcready,
-                                              bcfree, t_lane + P_BC_COL0, p.err, ok, jck, ck);
     if (!ok) break;
     if (FINAL && full_tile) sm100::fence_proxy_async_smem();   // y tile visible to the TMA store
     sm100::tc_fence_before();
