@@ -923,16 +923,18 @@ def hook_bwd_launches(case):
     (as the ncu launch list shows them): the recomputed forward (6, its scan
     storing the scan gradient's H checkpoints) and dt_raw, 4 weight
     transposes, the gate and LayerNorm gradient (4, or 2 without LayerNorm),
-    the scan gradient, and 21 more: the padding rows of 3 activations zeroed,
+    the scan gradient, and 19 more: the padding rows of 3 activations zeroed,
     per projection its input-gradient and weight-gradient GEMMs (dt_proj and
     x_proj with a split-K sum) and operand conversions, the conv gradient and
-    its column sum, dh = dh+ + dx, and h transposed."""
+    its column sum, dh = dh+ + dx, and h transposed; on the chunked scan
+    gradient also ddt_raw and dz converted to bf16 (the walk writes them so)."""
     w = case.weights[0]
     ln = 4 if w.get("ln_w") is not None else 2
     # (on the walk along each sequence the recomputed forward scan stores the H
     # checkpoints of sequences whose length is a multiple of 16, and the
     # gradient's checkpoint pass launches but fills only the others)
-    return 6 + 1 + 4 + ln + bwd_launches(case.B, case.dims.d_inner) + 21
+    walk = bwd_walks_sequences(case.B, case.dims.d_inner)
+    return 6 + 1 + 4 + ln + bwd_launches(case.B, case.dims.d_inner) + 19 + (0 if walk else 2)
 
 
 def run_hook_backward(args, rank, world, local_rank):

@@ -199,6 +199,112 @@ struct RowWalk {
   }
 };
 
+// The same with the row held in registers, for d = 256·NK: lane ℓ takes the
+// 8-column groups 8ℓ + 256k (k < NK), read once as 16-byte vectors.
+template <bool HAS_LN, int NK>
+__global__ void __launch_bounds__(256) ln_gate_bwd_rows_reg_kernel(const bf16* __restrict__ o,
+                                                                   const float* __restrict__ dh_out,
+                                                                   const float* __restrict__ gamma,
+                                                                   const float* __restrict__ beta, float g, int d,
+                                                                   const int* __restrict__ len, int L, long long M,
+                                                                   float2* __restrict__ stats,
+                                                                   float* __restrict__ ds_row,
+                                                                   bf16* __restrict__ dout) {
+  const long long m = blockIdx.x * 8LL + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  bf16* drow = dout + m * d;
+  if (!valid_row(len, L, m)) {
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+      *reinterpret_cast<uint4*>(drow + 8 * lane + 256 * k) = make_uint4(0u, 0u, 0u, 0u);
+    if (lane == 0) {
+      ds_row[m] = 0.0f;
+      stats[m] = make_float2(0.0f, 0.0f);
+    }
+    return;
+  }
+  float ov[NK][8], gv[NK][8];
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const int j = 8 * lane + 256 * k;
+    load8(o + m * d + j, ov[k]);
+    load8(dh_out + m * d + j, gv[k]);
+  }
+  float mu = 0.0f, rstd = 1.0f;
+  if (HAS_LN) {
+    float sum = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += ov[k][i];
+#pragma unroll
+    for (int x = 16; x; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
+    mu = sum / (float)d;
+    float q = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t = ov[k][i] - mu;
+        q += t * t;
+      }
+#pragma unroll
+    for (int x = 16; x; x >>= 1) q += __shfl_xor_sync(0xffffffffu, q, x);
+    rstd = rsqrtf(q / (float)d + 1e-5f);
+  }
+  float sh = 0.0f, s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const int j = 8 * lane + 256 * k;
+    if (HAS_LN) {
+      float gm[8], bt[8];
+      load8(gamma + j, gm);
+      load8(beta + j, bt);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float nh = (ov[k][i] - mu) * rstd;
+        sh += gv[k][i] * (gm[i] * nh + bt[i]);
+        const float gg = g * gv[k][i] * gm[i];
+        s1 += gg;
+        s2 += gg * nh;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sh += gv[k][i] * ov[k][i];
+    }
+  }
+#pragma unroll
+  for (int x = 16; x; x >>= 1) {
+    sh += __shfl_xor_sync(0xffffffffu, sh, x);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, x);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, x);
+  }
+  const float m1 = s1 / (float)d, m2 = s2 / (float)d;
+#pragma unroll
+  for (int k = 0; k < NK; ++k) {
+    const int j = 8 * lane + 256 * k;
+    float dv[8];
+    if (HAS_LN) {
+      float gm[8];
+      load8(gamma + j, gm);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float nh = (ov[k][i] - mu) * rstd;
+        dv[i] = rstd * (gm[i] * (g * gv[k][i]) - m1 - nh * m2);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dv[i] = g * gv[k][i];
+    }
+    *reinterpret_cast<uint4*>(drow + j) = pack8(dv);
+  }
+  if (lane == 0) {
+    ds_row[m] = sh;
+    stats[m] = make_float2(mu, rstd);
+  }
+}
+
 // ❸ column sums, chunk y of ROW_CHUNK rows: dγ and dβ partials
 // part[y][0][j] = Σ ĝ ⊙ n̂, part[y][1][j] = Σ ĝ over the chunk's valid rows.
 // Each thread takes four columns (one 16-byte load of dh⁺, one 8-byte load of o

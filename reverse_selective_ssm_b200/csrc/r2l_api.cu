@@ -788,7 +788,13 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   bf16* do16 = (bf16*)(ws + q.do16);
   const bool has_ln = w->ln_w != nullptr;
   const unsigned rblocks = (unsigned)((M + 7) / 8);
-  if (has_ln)
+  if (d == 2048 && has_ln)   // the row in registers (16-byte loads, one pass over memory)
+    K::ln_gate_bwd_rows_reg_kernel<true, 8><<<rblocks, 256, 0, st>>>(o, dh_out, w->ln_w, w->ln_b, g, d, len, L, M,
+                                                                     stats, dsrow, do16);
+  else if (d == 2048)
+    K::ln_gate_bwd_rows_reg_kernel<false, 8><<<rblocks, 256, 0, st>>>(o, dh_out, nullptr, nullptr, g, d, len, L, M,
+                                                                      stats, dsrow, do16);
+  else if (has_ln)
     K::ln_gate_bwd_rows_kernel<true><<<rblocks, 256, 0, st>>>(o, dh_out, w->ln_w, w->ln_b, g, d, len, L, M, stats,
                                                               dsrow, do16);
   else
@@ -818,7 +824,11 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   R2L_LAUNCH_CHECK();
   R2L_TRY(gemm_f32(do16, d, y, E, gr->out_proj_w, E, d, E, (int)M, nullptr, d, err, gpart, gpb, st, true, true));
 
-  // ---- ❷ the scan (bf16 u and z, fp32 dt_raw, B|C and dy)
+  // ---- ❷ the scan (bf16 u and z, fp32 dt_raw, B|C and dy); on the walk along
+  // each sequence it writes ddt_raw and dz in bf16 itself
+  const bool walks = r2l::scan_bwd_walks(B, E, 0);
+  bf16* ddt16 = (bf16*)(ws + q.ddt16);
+  bf16* dxz16 = (bf16*)(ws + q.dxz16);
   float* dus = (float*)(ws + q.dus);
   float* dz = (float*)(ws + q.dz);
   float* ddt = (float*)(ws + q.ddt);
@@ -832,14 +842,17 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
     a.B = B; a.L = L; a.E = E; a.chunk_tokens = 0; a.lengths = len;
     a.status = err;
     a.hck = hck_written ? hck : nullptr;
+    if (walks) {   // ddt_raw and dz straight to the bf16 GEMM operands
+      a.ddt16 = ddt16; a.ld_ddt16 = E;
+      a.dz16 = dxz16 + E; a.ld_dz16 = 2LL * E;
+    }
     char* sw = ws + q.sbwd;
     if (cudaMemsetAsync(sw, 0, 16, st) != cudaSuccess) return R2L_ERR_CUDA;
     if (r2l::scan_bwd_f32(a, sw + align_up(16, kAlign), st) != cudaSuccess) return R2L_ERR_CUDA;
   }
 
   // ---- dt_proj: dΔr = ddt_raw·W_dt, dW_dt = ddt_rawᵀ·Δr
-  bf16* ddt16 = (bf16*)(ws + q.ddt16);
-  R2L_TRY(cvt_transpose(ddt, E, M, E, ddt16, E, (bf16*)nullptr, 0, len, L, st));
+  if (!walks) R2L_TRY(cvt_transpose(ddt, E, M, E, ddt16, E, (bf16*)nullptr, 0, len, L, st));
   float* ddr = (float*)(ws + q.ddr);
   R2L_TRY(gemm_f32(ddt16, E, wdtT, E, ddr, R, M, R, E, len, L, err, gpart, gpb, st));
   R2L_TRY(gemm_f32(ddt16, E, dr, R, gr->dt_proj_w, R, E, R, (int)M, nullptr, E, err, gpart, gpb, st, true, true));
@@ -854,7 +867,6 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
                    true));
 
   // ---- conv + SiLU: dx (into dxz), dconv_w, dconv_b; dz into dxz
-  bf16* dxz16 = (bf16*)(ws + q.dxz16);
   float* cpart = (float*)(ws + q.cpart);
   if (cudaFuncSetAttribute(K::conv_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::CONV_SMEM) !=
       cudaSuccess)
@@ -866,7 +878,7 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   K::chunk_sum_kernel<1><<<(5 * E + 31) / 32, 256, 0, st>>>(cpart, (int)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS), 5 * E,
                                                             E, gr->conv_w, gr->conv_b);
   R2L_LAUNCH_CHECK();
-  R2L_TRY(cvt_transpose(dz, E, M, E, dxz16 + E, 2LL * E, (bf16*)nullptr, 0, len, L, st));
+  if (!walks) R2L_TRY(cvt_transpose(dz, E, M, E, dxz16 + E, 2LL * E, (bf16*)nullptr, 0, len, L, st));
 
   // ---- in_proj: dh = dh⁺ + [dx | dz]·W_in, dW_in = [dx | dz]ᵀ·h
   float* dhtmp = (float*)(ws + q.dhtmp);

@@ -87,6 +87,10 @@ struct Args {
   float* pbc;              // [E/CPB][B·L][32] per-block partial dB | dC
   int nbc;                 // channel blocks in pbc
   int ckpt_ragged_only;    // the checkpoint pass skips sequences whose length is a multiple of 16
+  bf16* ddt16;             // bf16 ddt_raw and dz instead of fp32 (the walk only), or null
+  long long ld_ddt16;
+  bf16* dz16;
+  long long ld_dz16;
   uint32_t lnbits[16];     // float log(1) … log(16): the power-path A_log
 };
 
@@ -618,6 +622,8 @@ static bool use_seq(int B, int E, int chunk_tokens) {
   return chunk_tokens == 0 && (long long)B * (E / sbwd::QC) >= 4LL * 148;
 }
 
+bool scan_bwd_walks(int B, int E, int chunk_tokens) { return use_seq(B, E, chunk_tokens); }
+
 int scan_bwd_chunk_tokens(int chunk_tokens) {
   if (chunk_tokens <= 0) return 16;
   return chunk_tokens > SCAN_BWD_MAX_CHUNK ? SCAN_BWD_MAX_CHUNK : chunk_tokens;
@@ -668,6 +674,7 @@ cudaError_t scan_bwd_f32(const ScanBwdArgs& g, void* scratch, cudaStream_t st) {
     a.T = QS;
     a.nc = (g.L + QS - 1) / QS;
     char* p = (char*)scratch;
+    a.ddt16 = g.ddt16; a.ld_ddt16 = g.ld_ddt16; a.dz16 = g.dz16; a.ld_dz16 = g.ld_dz16;
     a.hcar = g.hck ? g.hck : (float*)p;
     a.ckpt_ragged_only = g.hck ? 1 : 0;
     p += al((size_t)g.B * a.nc * g.E * 16 * 4);

@@ -25,7 +25,17 @@ struct ScanBwdArgs {
   // it computes all of them in its own scratch).  Used by the walk along each
   // sequence only.
   float* hck;
+  // bf16 copies of ddt_raw and dz written instead of the fp32 arrays (rows of
+  // stride ld_ddt16 / ld_dz16), by the walk along each sequence only
+  // (scan_bwd_walks); null: fp32
+  __nv_bfloat16* ddt16;
+  long long ld_ddt16;
+  __nv_bfloat16* dz16;
+  long long ld_dz16;
 };
+
+// Whether a call of this shape takes the walk along each sequence.
+bool scan_bwd_walks(int B, int E, int chunk_tokens);
 
 int scan_bwd_chunk_tokens(int chunk_tokens);
 bool scan_bwd_supported(int B, int L, int E, int chunk_tokens);   // grid limits of the launches

@@ -401,8 +401,16 @@ __global__ void __launch_bounds__(QT, QMINB) seq_final_kernel(const Args a) {
         const float4 v = make_float4(src[4 * qi(4 * qq)], src[4 * qi(4 * qq + 1)], src[4 * qi(4 * qq + 2)],
                                      src[4 * qi(4 * qq + 3)]);
         const size_t row = bl + s + r;
-        float* dst = arr == 0 ? a.du + row * a.E : arr == 1 ? a.ddt + row * a.E : a.dz + row * a.ld_dz;
-        st4(dst + c0 + 4 * qq, v);
+        bf16* d16 = arr == 1 ? a.ddt16 : arr == 2 ? a.dz16 : nullptr;
+        if (d16) {
+          const long long ld = arr == 1 ? a.ld_ddt16 : a.ld_dz16;
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+          *reinterpret_cast<uint2*>(d16 + row * ld + c0 + 4 * qq) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        } else {
+          float* dst = arr == 0 ? a.du + row * a.E : arr == 1 ? a.ddt + row * a.E : a.dz + row * a.ld_dz;
+          st4(dst + c0 + 4 * qq, v);
+        }
       }
       for (int i = threadIdx.x; i < QS * 8; i += QT) {
         const int r = i / 8, qq = i & 7;
@@ -425,8 +433,10 @@ __global__ void __launch_bounds__(QT, QMINB) seq_final_kernel(const Args a) {
     const size_t row = bl + l.nck * QS + (size_t)(i / 8);
     const int qq = (int)(i & 7);
     st4(a.du + row * a.E + c0 + 4 * qq, zero);
-    st4(a.ddt + row * a.E + c0 + 4 * qq, zero);
-    st4(a.dz + row * a.ld_dz + c0 + 4 * qq, zero);
+    if (a.ddt16) *reinterpret_cast<uint2*>(a.ddt16 + row * a.ld_ddt16 + c0 + 4 * qq) = make_uint2(0u, 0u);
+    else st4(a.ddt + row * a.E + c0 + 4 * qq, zero);
+    if (a.dz16) *reinterpret_cast<uint2*>(a.dz16 + row * a.ld_dz16 + c0 + 4 * qq) = make_uint2(0u, 0u);
+    else st4(a.dz + row * a.ld_dz + c0 + 4 * qq, zero);
     st4(a.pbc + ((size_t)blockIdx.x * a.B * a.L + row) * 32 + 4 * qq, zero);
   }
   float* pa = a.pA + ((size_t)l.b * a.E + l.c) * 16 + 8 * l.h;
