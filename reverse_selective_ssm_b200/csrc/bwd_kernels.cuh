@@ -393,27 +393,29 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
-// conv + SiLU, over a tile of 64 rows × 128 channels.  With W = 4 taps,
+// conv + SiLU, over a tile of 32 rows × 128 channels.  With W = 4 taps,
 // w_k = conv_w[c][W−1−k] multiplying x_{i+k}:
 //   pre_i  = conv_b + Σ_k w_k·x_{i+k}   (x_j = 0 for j ≥ the sequence's length)
 //   dpre_i = (du_s + du_x)_i · SiLU'(pre_i)   (0 on padding rows)
 //   dx_j   = Σ_k w_k·dpre_{j−k}   (k ≤ j: the same sequence)
-// The block first stages x (rows m0−3 … m0+66), du_s and du_x (rows m0−3 …
-// m0+63) in shared memory by 16-byte asynchronous copies, all in flight at
+// The block first stages x (rows m0−3 … m0+34), du_s and du_x (rows m0−3 …
+// m0+31) in shared memory by 16-byte asynchronous copies, all in flight at
 // once, padding rows as zero.  Thread (p, grp) then takes the channel pair c,
 // c+1 (c = 2p within the tile) and rows r0 = m0 + 16·grp … r0+15; dpre of the
 // three rows above r0 is recomputed, so every tile is independent.  dx goes out
 // as bf16 twice: into dxz (row-major) and into dxzT[c][r0 …] (its transpose, 16
 // consecutive positions per channel: two 16-byte stores).  The chunk's
 // parameter partials part[y][k][c] = Σ dpre_i·x_{i+k} (tap W−1−k) and
-// part[y][4][c] = Σ dpre_i are summed over the four row groups in order.
-constexpr int CONV_ROWS = 64;
+// part[y][4][c] = Σ dpre_i are summed over the row groups in order.
+constexpr int CONV_ROWS = 32;
+constexpr int CONV_GRP = CONV_ROWS / 16;          // 16-row groups: threads (p, grp)
+constexpr int CONV_THREADS = 64 * CONV_GRP;
 constexpr int CONV_CH = 128;
 constexpr int CONV_XROWS = CONV_ROWS + 6;
 constexpr int CONV_DROWS = CONV_ROWS + 3;
 constexpr size_t CONV_SMEM = 2 * (size_t)CONV_DROWS * 64 * sizeof(float2) + (size_t)CONV_XROWS * 64 * 4;
 
-__global__ void __launch_bounds__(256) conv_bwd_kernel(
+__global__ void __launch_bounds__(CONV_THREADS) conv_bwd_kernel(
     const bf16* __restrict__ x, long long ldx, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
     const float* __restrict__ du_s, const float* __restrict__ du_x, int E, const int* __restrict__ len, int L,
     long long M, bf16* __restrict__ dxz, long long lddxz, bf16* __restrict__ dxzT, long long ldT,
@@ -435,13 +437,13 @@ __global__ void __launch_bounds__(256) conv_bwd_kernel(
     rowok[threadIdx.x] = m >= 0 && m < M && valid_row(len, L, m);
   }
   __syncthreads();
-  for (int k = threadIdx.x; k < CONV_XROWS * 16; k += 256) {            // x: 16 × 16 B per row
+  for (int k = threadIdx.x; k < CONV_XROWS * 16; k += CONV_THREADS) {   // x: 16 × 16 B per row
     const int r = k >> 4, q = k & 15;
     const bool ok = rowok[r] && 8 * q < nch;
     const long long m = ok ? m0 - HALO + r : 0;
     cp_async16(xs + r * 64 + 4 * q, x + m * ldx + (ok ? c0 + 8 * q : 0), ok);
   }
-  for (int k = threadIdx.x; k < CONV_DROWS * 32; k += 256) {            // du_s, du_x: 32 × 16 B per row
+  for (int k = threadIdx.x; k < CONV_DROWS * 32; k += CONV_THREADS) {   // du_s, du_x: 32 × 16 B per row
     const int r = k >> 5, q = k & 31;
     const bool ok = rowok[r] && 4 * q < nch;
     const long long off = ok ? (m0 - HALO + r) * E + c0 + 4 * q : 0;
@@ -571,7 +573,7 @@ __global__ void __launch_bounds__(256) conv_bwd_kernel(
   for (int k = 0; k < 5; ++k) {
     float2 acc = red[p * 5 + k];
 #pragma unroll
-    for (int gq = 1; gq < 4; ++gq) {
+    for (int gq = 1; gq < CONV_GRP; ++gq) {
       acc.x += red[(gq * 64 + p) * 5 + k].x;
       acc.y += red[(gq * 64 + p) * 5 + k].y;
     }

@@ -669,7 +669,7 @@ bool make_bwd_plan(const r2l_dims* dm, int B, int L, BwdPlan* q) {
   q->ddr = take(M * R * 4);
   q->ddbc16 = take(M * ldd * 2);
   q->dux = take(M * E * 4);
-  q->cpart = take((size_t)row_chunks(p.M) * 5 * E * 4);
+  q->cpart = take((size_t)((q->Mp + r2l::bwd::CONV_ROWS - 1) / r2l::bwd::CONV_ROWS) * 5 * E * 4);
   q->dxz16 = take(M * 2 * E * 2);
   q->hT = take(d * Mp * 2);
   q->dhtmp = take(M * d * 4);
@@ -872,7 +872,7 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
       cudaSuccess)
     return R2L_ERR_CUDA;
   K::conv_bwd_kernel<<<dim3((unsigned)((E + K::CONV_CH - 1) / K::CONV_CH), (unsigned)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS)),
-                       256, K::CONV_SMEM, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E, len, L, M, dxz16, 2LL * E, nullptr, Mp,
+                       K::CONV_THREADS, K::CONV_SMEM, st>>>(xz, 2LL * E, w->conv_w, w->conv_b, dus, dux, E, len, L, M, dxz16, 2LL * E, nullptr, Mp,
                                      cpart);
   R2L_LAUNCH_CHECK();
   K::chunk_sum_kernel<1><<<(5 * E + 31) / 32, 256, 0, st>>>(cpart, (int)((Mp + K::CONV_ROWS - 1) / K::CONV_ROWS), 5 * E,
