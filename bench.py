@@ -988,6 +988,40 @@ def run_hook_backward(args, rank, world, local_rank):
     clk = clocks.stop() if rank == 0 else None
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
 
+    # a training step of the hook: the training forward (h+ into its own
+    # buffer, the intermediates and checkpoints left in the workspace), then the
+    # gradient without recomputing the forward
+    out_buf = torch.empty_like(h)
+    sdims = bd.dims_of(case.dims, case.dtype, bd.R2L_FLAG_SAVED_FORWARD)
+
+    def train_step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        bd.sidecar_forward_train(h, w, dims, case.s[0], lengths, workspace=ws, out=out_buf, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        bd.sidecar_backward(h, w, sdims, case.s[0], dh_out, grads, lengths, workspace=ws, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(max(2, args.warmup)):
+        train_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for k in range(K):
+        train_step(evs[k])
+    torch.cuda.synchronize()
+    barrier()
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    step_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][2]), world, dev)
+    train = {"ms_per_step": round(step_ms / K, 4),
+             "tokens_per_s": round(whole_job_rate(case.valid_tokens, world, K, step_ms), 1),
+             "forward_ms": round(fwd_ms / K, 4), "backward_ms": round(bwd_ms / K, 4),
+             "api": "r2l_sidecar_forward_train, then r2l_sidecar_backward with R2L_FLAG_SAVED_FORWARD"}
+
     e2e = None
     if not args.no_e2e:
         # the hidden states and dh⁺ come from pinned host memory and dh, ds and every
@@ -1048,6 +1082,7 @@ def run_hook_backward(args, rank, world, local_rank):
                      "frac": round(achieved / tpeak, 4), "peak_source": tnote, "algorithmic_per_launch": flops,
                      "ms_per_launch": round(per_call, 4), "traffic": None},
         "gpu_launches": hook_bwd_launches(case) * K, "clocks": clk, "e2e": e2e, "source_sha": source_sha(),
+        "train_step": train,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_hook_backward(case, dh_host)

@@ -86,6 +86,9 @@ typedef enum {
 #define R2L_FLAG_FORWARD_SCAN 0x2u  /* run the block left to right instead: causal conv and a
                                        forward scan (the "L2R Mamba" control of Table 4); every
                                        other step is unchanged                                    */
+#define R2L_FLAG_SAVED_FORWARD 0x4u /* r2l_sidecar_backward only: the workspace holds this hook's
+                                       forward from r2l_sidecar_forward_train, so the forward is
+                                       not recomputed                                             */
 /* Device status bits, reported by r2l_get_device_status(). */
 #define R2L_DEVFLAG_LENGTH_CLAMPED 0x1u   /* a lengths[b] was outside [0, L] and was clamped */
 #define R2L_DEVFLAG_TIMEOUT 0x2u          /* a kernel gave up waiting on a pipeline barrier (results invalid) */
@@ -326,7 +329,8 @@ R2L_API size_t r2l_sidecar_backward_workspace_size(const r2l_dims *dims, int B, 
  *   *ds   fp32 scalar     ∂L/∂s = (1 − tanh²(s)) Σ dh_out ⊙ ĥ (device pointer)
  *   grads                 ∂L/∂(every parameter), summed over the batch
  *
- * The forward is recomputed into the workspace, then the chain rule runs in
+ * The forward is recomputed into the workspace (unless R2L_FLAG_SAVED_FORWARD
+ * says r2l_sidecar_forward_train left it there), then the chain rule runs in
  * reverse: gate, LayerNorm, out_proj, the scan (bf16 u and z, fp32 state),
  * dt_proj, x_proj, conv + SiLU, in_proj.  GEMM operands are bf16 (gradients
  * rounded once to bf16 where they feed a GEMM), accumulation fp32; every
@@ -344,6 +348,24 @@ R2L_API r2l_status r2l_sidecar_backward(const void *hidden, const r2l_weights *w
                                         float s, int B, int L, const int32_t *lengths, const float *dh_out,
                                         float *dh, float *ds, const r2l_grads *grads, void *workspace,
                                         size_t workspace_bytes, void *stream);
+
+/* The hook's forward for training (the R2LM-PI setting, §3.4 and §4.1):
+ * out = h⁺ = h + tanh(s)·ĥ as r2l_sidecar_forward computes it, written to
+ * `out` (act dtype [B, L, d], 16-byte aligned, not aliasing hidden: padding
+ * rows are copied from hidden; hidden is not written, since the gradient reads
+ * it again), and everything r2l_sidecar_backward needs left in `workspace`
+ * (≥ r2l_sidecar_backward_workspace_size(dims, B, L) bytes): the forward's
+ * intermediates, dt_raw in fp32, and the H checkpoints of its scan gradient
+ * (every 16 positions, for sequences whose length is a multiple of 16, with
+ * dt_rank 128).  A later r2l_sidecar_backward with R2L_FLAG_SAVED_FORWARD in
+ * dims->flags and the same hidden, weights, other dims, s, B, L, lengths and
+ * workspace (untouched in between) skips its recomputation of the forward.
+ * Supported shapes and errors as r2l_sidecar_backward; out == hidden returns
+ * R2L_ERR_INVALID_ARG.  Runs the layer even when tanh(s) == 0 (the gradient
+ * needs ĥ for ds).                                                            */
+R2L_API r2l_status r2l_sidecar_forward_train(const void *hidden, void *out, const r2l_weights *weights,
+                                             const r2l_dims *dims, float s, int B, int L, const int32_t *lengths,
+                                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream`, then reads the device status word that the last
  * forward call on `workspace` wrote.  *flags_out receives the R2L_DEVFLAG_*

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(PKG, "libr2l.so")
 R2L_BF16, R2L_FP32 = 0, 1
 R2L_FLAG_GENERAL_A = 0x1
 R2L_FLAG_FORWARD_SCAN = 0x2
+R2L_FLAG_SAVED_FORWARD = 0x4
 R2L_DEVFLAG_LENGTH_CLAMPED = 0x1
 
 STATUS = {0: "R2L_OK", 1: "R2L_ERR_INVALID_ARG", 2: "R2L_ERR_UNSUPPORTED", 3: "R2L_ERR_ALIGNMENT",
@@ -28,7 +29,8 @@ EXPORTS = ("r2l_abi_version", "r2l_status_string", "r2l_workspace_size", "r2l_si
            "r2l_sidecar_forward_debug", "r2l_sidecar_forward_profiled", "r2l_sidecar_stack",
            "r2l_get_device_status", "r2l_reverse_scan_workspace_size", "r2l_reverse_scan",
            "r2l_reverse_scan_noalloc", "r2l_reverse_scan_backward_workspace_size",
-           "r2l_reverse_scan_backward", "r2l_sidecar_backward_workspace_size", "r2l_sidecar_backward")
+           "r2l_reverse_scan_backward", "r2l_sidecar_backward_workspace_size", "r2l_sidecar_backward",
+           "r2l_sidecar_forward_train")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -117,6 +119,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.r2l_sidecar_backward.restype = ci
     lib.r2l_sidecar_backward.argtypes = [vp, ctypes.POINTER(Weights), ctypes.POINTER(Dims), cf, ci, ci, vp, vp, vp,
                                          vp, ctypes.POINTER(Grads), vp, ctypes.c_size_t, vp]
+    lib.r2l_sidecar_forward_train.restype = ci
+    lib.r2l_sidecar_forward_train.argtypes = [vp, vp, ctypes.POINTER(Weights), ctypes.POINTER(Dims), cf, ci, ci, vp,
+                                              vp, ctypes.c_size_t, vp]
     lib.r2l_get_device_status.restype = ci
     lib.r2l_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -333,6 +338,27 @@ def alloc_grads(weights: Dict[str, Optional[torch.Tensor]], device="cuda") -> Di
     weight is None)."""
     return {k: None if v is None else torch.empty(v.shape, dtype=torch.float32, device=device)
             for k, v in weights.items()}
+
+
+def sidecar_forward_train(hidden: torch.Tensor, weights, dims: Dims, s: float, lengths=None,
+                          workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None,
+                          check: bool = True):
+    """r2l_sidecar_forward_train: returns (out = h⁺, workspace); hidden is not
+    written.  Pass the same workspace to sidecar_backward with dims carrying
+    R2L_FLAG_SAVED_FORWARD to skip the forward's recomputation."""
+    lib = load()
+    B, L = hidden.shape[0], hidden.shape[1]
+    if workspace is None:
+        workspace = torch.empty(max(sidecar_backward_workspace_size(dims, B, L), 16), dtype=torch.uint8,
+                                device=hidden.device)
+    if out is None:
+        out = torch.empty_like(hidden)
+    w = weights if isinstance(weights, Weights) else weights_struct(weights)
+    st = lib.r2l_sidecar_forward_train(_ptr(hidden), _ptr(out), ctypes.byref(w), ctypes.byref(dims), float(s), B, L,
+                                       _ptr(lengths), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if check and st != 0:
+        raise R2LError(st, "r2l_sidecar_forward_train")
+    return out, workspace
 
 
 def sidecar_backward(hidden: torch.Tensor, weights, dims: Dims, s: float, dh_out: torch.Tensor,

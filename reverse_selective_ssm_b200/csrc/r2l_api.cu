@@ -737,6 +737,21 @@ r2l_status check_grads(const r2l_grads* gr, const r2l_weights* w) {
   return R2L_OK;
 }
 
+// The forward as the gradient needs it, into the backward's workspace: the
+// layer on `target` (in place with the residual, or reading it only), its
+// scan storing the scan gradient's checkpoints where it can (*hck_written),
+// and dt_raw = Δr·W_dtᵀ in fp32.
+r2l_status forward_for_backward(bf16* target, bool residual, const r2l_weights* w, const BwdPlan& q, float g, int B,
+                                int L, const int32_t* lengths, char* ws, cudaStream_t st, int* hck_written) {
+  const Plan& p = q.f;
+  R2L_TRY(prep(p, ws, lengths, B, L, st));
+  R2L_TRY(run_layer<bf16>(target, w, p, g, B, L, ws, st, nullptr, nullptr, residual, nullptr, (float*)(ws + q.hck),
+                          hck_written));
+  return gemm_f32((const bf16*)(ws + p.dr), p.R, (const bf16*)w->dt_proj_w, p.R, (float*)(ws + q.dt32), p.E, p.M,
+                  p.E, p.R, (const int*)(ws + p.len), L, (unsigned*)(ws + p.status), (float*)(ws + q.gpart),
+                  q.gpart_bytes, st);
+}
+
 r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dims* dims, float s, int B, int L,
                          const int32_t* lengths, const float* dh_out, float* dh, float* ds, const r2l_grads* gr,
                          void* workspace, size_t workspace_bytes, cudaStream_t st) {
@@ -755,22 +770,26 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   const float g = (float)gd;
   const float dgate = (float)(1.0 - gd * gd);   // d tanh(s) / ds
 
-  // ---- the forward's intermediates: xz, u, Δr|B|C, Δr (bf16), y, o; dt_raw in fp32
-  R2L_TRY(prep(p, ws, lengths, B, L, st));
-  // run_layer with residual = false reads hidden and writes nothing to it; its
-  // scan stores H every 16 positions for the scan gradient where it can
+  // ---- the forward's intermediates: xz, u, Δr|B|C, Δr (bf16), y, o; dt_raw in
+  // fp32; the scan gradient's checkpoints.  Recomputed here, or left in the
+  // workspace by r2l_sidecar_forward_train (R2L_FLAG_SAVED_FORWARD).
   float* hck = (float*)(ws + q.hck);
   int hck_written = 0;
-  R2L_TRY(run_layer<bf16>((bf16*)const_cast<void*>(hidden), w, p, g, B, L, ws, st, nullptr, nullptr, false, nullptr,
-                          hck, &hck_written));
+  if (dims->flags & R2L_FLAG_SAVED_FORWARD) {
+    R2L_TRY(prep(p, ws, lengths, B, L, st));
+    hck_written = r2l::scan_writes_checkpoints(R, false) ? 1 : 0;
+  } else {
+    // hidden is only read (no residual)
+    R2L_TRY(forward_for_backward((bf16*)const_cast<void*>(hidden), false, w, q, g, B, L, lengths, ws, st,
+                                 &hck_written));
+  }
   const bf16* xz = (const bf16*)(ws + p.xz);
   const bf16* u = (const bf16*)(ws + p.u);
   const float* dbc = (const float*)(ws + p.dbc);
   const bf16* dr = (const bf16*)(ws + p.dr);
   const bf16* y = (const bf16*)(ws + p.y);
   const bf16* o = (const bf16*)(ws + p.o);
-  float* dt32 = (float*)(ws + q.dt32);
-  R2L_TRY(gemm_f32(dr, R, (const bf16*)w->dt_proj_w, R, dt32, E, M, E, R, len, L, err, gpart, gpb, st));
+  const float* dt32 = (const float*)(ws + q.dt32);
 
   // ---- weights transposed once: W_outᵀ [E, d], W_dtᵀ [R, E], W_xᵀ [E, R+2N], W_inᵀ [d, 2E]
   bf16* woutT = (bf16*)(ws + q.woutT);
@@ -905,10 +924,11 @@ size_t r2l_sidecar_backward_workspace_size(const r2l_dims* dims, int B, int L) {
   return q.total;
 }
 
-r2l_status r2l_sidecar_backward(const void* hidden, const r2l_weights* weights, const r2l_dims* dims, float s, int B,
-                                int L, const int32_t* lengths, const float* dh_out, float* dh, float* ds,
-                                const r2l_grads* grads, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!hidden || !dims || !dh_out || !dh || !ds) return R2L_ERR_INVALID_ARG;
+namespace {
+// The checks r2l_sidecar_backward and r2l_sidecar_forward_train share.
+r2l_status check_train_call(const void* hidden, const r2l_weights* weights, const r2l_dims* dims, int B, int L,
+                            const int32_t* lengths, void* workspace, size_t workspace_bytes) {
+  if (!hidden || !dims) return R2L_ERR_INVALID_ARG;
   Plan p;
   if (!make_plan(dims, B, L, &p)) return R2L_ERR_INVALID_ARG;
   if (dims->d_state != 16 || dims->d_conv != 4) return R2L_ERR_UNSUPPORTED;
@@ -916,14 +936,43 @@ r2l_status r2l_sidecar_backward(const void* hidden, const r2l_weights* weights, 
   if ((dims->d_model % 8) || (dims->d_inner % 64) || (dims->dt_rank % 8)) return R2L_ERR_UNSUPPORTED;
   if (L > 65535 || B > 65535 || (p.M + 63) / 64 > 65535) return R2L_ERR_UNSUPPORTED;
   R2L_TRY(check_weights(weights));
-  R2L_TRY(check_grads(grads, weights));
-  for (const void* q : {hidden, (const void*)dh_out, (const void*)dh})
-    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
-  if (((uintptr_t)ds & 3u) || (lengths && ((uintptr_t)lengths & 3u))) return R2L_ERR_ALIGNMENT;
+  if (!aligned16(hidden)) return R2L_ERR_ALIGNMENT;
+  if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
   BwdPlan q;
   if (!make_bwd_plan(dims, B, L, &q)) return R2L_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < q.total) return R2L_ERR_WORKSPACE;
   if (!aligned16(workspace)) return R2L_ERR_ALIGNMENT;
+  return R2L_OK;
+}
+}  // namespace
+
+r2l_status r2l_sidecar_forward_train(const void* hidden, void* out, const r2l_weights* weights, const r2l_dims* dims,
+                                     float s, int B, int L, const int32_t* lengths, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!out || out == hidden) return R2L_ERR_INVALID_ARG;
+  R2L_TRY(check_train_call(hidden, weights, dims, B, L, lengths, workspace, workspace_bytes));
+  if (!aligned16(out)) return R2L_ERR_ALIGNMENT;
+  BwdPlan q;
+  make_bwd_plan(dims, B, L, &q);
+  cudaStream_t st = (cudaStream_t)stream;
+  // h⁺ is formed in `out` (a copy of h, updated in place on valid rows); h,
+  // which the gradient reads again, stays as it is
+  if (cudaMemcpyAsync(out, hidden, (size_t)q.f.M * q.f.d * sizeof(bf16), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return R2L_ERR_CUDA;
+  int hck_written = 0;
+  return forward_for_backward((bf16*)out, true, weights, q, (float)std::tanh((double)s), B, L, lengths,
+                              (char*)workspace, st, &hck_written);
+}
+
+r2l_status r2l_sidecar_backward(const void* hidden, const r2l_weights* weights, const r2l_dims* dims, float s, int B,
+                                int L, const int32_t* lengths, const float* dh_out, float* dh, float* ds,
+                                const r2l_grads* grads, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dh_out || !dh || !ds) return R2L_ERR_INVALID_ARG;
+  R2L_TRY(check_train_call(hidden, weights, dims, B, L, lengths, workspace, workspace_bytes));
+  R2L_TRY(check_grads(grads, weights));
+  for (const void* q : {(const void*)dh_out, (const void*)dh})
+    if (!aligned16(q)) return R2L_ERR_ALIGNMENT;
+  if ((uintptr_t)ds & 3u) return R2L_ERR_ALIGNMENT;
   return backward_impl(hidden, weights, dims, s, B, L, lengths, dh_out, dh, ds, grads, workspace, workspace_bytes,
                        (cudaStream_t)stream);
 }

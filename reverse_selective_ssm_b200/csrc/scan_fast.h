@@ -46,6 +46,9 @@ int scan_auto_chunk_tokens(int B, int L, int E, bool pair = false);
 int scan_resolve_chunk_tokens(int B, int L, int E, int chunk_tokens, bool pair = false);
 // Bytes of carry scratch the scan needs for this shape and chunk length.
 size_t scan_carry_bytes(int B, int L, int E, int chunk_tokens, bool pair = false);
+// Whether a bf16 scan with this dt_rank and direction stores the scan
+// gradient's checkpoints when given a buffer (ScanArgs::hck).
+bool scan_writes_checkpoints(int dt_rank, bool forward);
 // Enqueue the scan (1 or 3 launches).  Returns the number of kernels launched
 // through *launches when not null.
 cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches);

@@ -185,6 +185,10 @@ cudaError_t launch(const ScanArgs& a, const rscan::Params& p, int nc, cudaStream
 
 }  // namespace
 
+bool scan_writes_checkpoints(int dt_rank, bool forward) {
+  return dt_rank == kScanFusedDtRank && !forward && R2L_SCAN_IMPL == 1;
+}
+
 cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   using namespace rscan;
   if (launches) *launches = 0;
@@ -216,7 +220,7 @@ cudaError_t scan_bf16(const ScanArgs& a, cudaStream_t st, int* launches) {
   p.hck = nullptr;
   p.nc16 = (a.L + 15) / 16;
   if (a.hck_written) *a.hck_written = 0;
-  if (a.hck && a.dt_mma && !a.forward && R2L_SCAN_IMPL == 1) {   // only the two-thread kernel writes them
+  if (a.hck && a.dt_mma && scan_writes_checkpoints(kScanFusedDtRank, a.forward != 0)) {   // the two-thread kernel
     p.hck = a.hck;
     if (a.hck_written) *a.hck_written = 1;
   }

@@ -216,3 +216,29 @@ def test_hook_backward_argument_checks(lib):
     assert _hook_bwd(lib, ws=None) == 4
     assert _hook_bwd(lib, ws_bytes=16) == 4
     assert _hook_bwd(lib, ws=FAKE + 8) == 3
+
+
+def _train_fwd(lib, dims=None, B=2, L=40, hidden=FAKE, out=FAKE + 1024, ws=FAKE, ws_bytes=None, lengths=None):
+    dims = dims or bd.make_dims(64, 128, dt_rank=8)
+    w = _weights()
+    if ws_bytes is None:
+        ws_bytes = bd.sidecar_backward_workspace_size(dims, B, L) or 1
+    return lib.r2l_sidecar_forward_train(hidden, out, ctypes.byref(w), ctypes.byref(dims), 0.5, B, L, lengths, ws,
+                                         ws_bytes, None)
+
+
+def test_train_forward_argument_checks(lib):
+    """r2l_sidecar_forward_train rejects bad arguments on the host: an output
+    that aliases the input (the gradient reads the input again), shapes the
+    gradient does not support, a workspace smaller than the gradient's."""
+    assert _train_fwd(lib, out=None) == 1
+    assert _train_fwd(lib, out=FAKE) == 1                                       # out == hidden
+    assert _train_fwd(lib, hidden=None) == 1
+    assert _train_fwd(lib, B=0) == 1
+    assert _train_fwd(lib, dims=bd.make_dims(64, 128, dt_rank=8, dtype=torch.float32)) == 2
+    assert _train_fwd(lib, dims=bd.make_dims(64, 128, dt_rank=8, flags=bd.R2L_FLAG_FORWARD_SCAN)) == 2
+    assert _train_fwd(lib, out=FAKE + 1032) == 3
+    assert _train_fwd(lib, lengths=FAKE + 2) == 3
+    assert _train_fwd(lib, ws=None) == 4
+    dims = bd.make_dims(64, 128, dt_rank=8)
+    assert _train_fwd(lib, ws_bytes=bd.workspace_size(dims, 2, 40)) == 4        # the forward's alone is too small

@@ -199,3 +199,41 @@ def test_hook_backward_zero_gate():
         assert torch.count_nonzero(grads[k]) == 0, k
     want = run_oracle(h, w, 0.0, dh_out)
     check_ds(ds, want["ds"], 0.0, dh_out, None, *hhat_pair(dims, h, w, 0.0, None))
+
+
+@pytest.mark.parametrize("B,L,lens,seed", [(8, 96, [96, 17, 64, 1, 80, 33, 96, 48], 88), (2, 160, [160, 97], 89)])
+def test_saved_forward_matches_recompute(B, L, lens, seed):
+    """r2l_sidecar_forward_train followed by r2l_sidecar_backward with
+    R2L_FLAG_SAVED_FORWARD gives, bit for bit, what r2l_sidecar_backward alone
+    gives (it recomputes the same forward); the training forward's output is
+    r2l_sidecar_forward's, and the input is left untouched.  B = 8: the walk
+    along each sequence, from the training forward's checkpoints where the
+    length is a multiple of 16; B = 2: the chunked scan gradient."""
+    dev = "cuda"
+    lengths = torch.tensor(lens, dtype=torch.int32)
+    dims, h, w, dh_out = make(B, L, seed=seed, lengths=lengths)
+    bdims = bd.dims_of(dims, torch.bfloat16)
+    wdev = bd.weights_to_device(w, dev)
+    hd, ln, gd = h.to(dev), lengths.to(dev), dh_out.to(dev)
+    h_before = hd.clone()
+    g1 = bd.alloc_grads(wdev, dev)
+    dh1, ds1 = bd.sidecar_backward(hd, wdev, bdims, 0.6, gd, g1, ln)
+    out, ws = bd.sidecar_forward_train(hd, wdev, bdims, 0.6, ln)
+    g2 = bd.alloc_grads(wdev, dev)
+    for v in g2.values():
+        if v is not None:
+            v.fill_(float("nan"))
+    sdims = bd.dims_of(dims, torch.bfloat16, bd.R2L_FLAG_SAVED_FORWARD)
+    dh2, ds2 = bd.sidecar_backward(hd, wdev, sdims, 0.6, gd, g2, ln, workspace=ws)
+    torch.cuda.synchronize()
+    st, flags = bd.get_device_status(ws)
+    assert st == 0 and flags == 0, (st, flags)
+    assert torch.equal(hd.view(torch.int16), h_before.view(torch.int16)), "input written"
+    assert torch.equal(dh1.view(torch.int32), dh2.view(torch.int32))
+    assert torch.equal(ds1.view(torch.int32), ds2.view(torch.int32))
+    for k in PARAMS:
+        assert torch.equal(g1[k].view(torch.int32), g2[k].view(torch.int32)), k
+    h_fwd = hd.clone()
+    bd.sidecar_forward(h_fwd, wdev, bdims, 0.6, ln)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), h_fwd.view(torch.int16))
