@@ -595,7 +595,9 @@ __global__ void reduce_params_kernel(const Args a, const float* seg, int nseg) {
   }
 }
 
-// 6b. dB | dC: sum of the per-block partials in block order.
+// 6b. dB | dC: sum of the per-block partials in a fixed order (four
+// interleaved running sums over the blocks, cb ≡ 0, 1, 2, 3 mod 4, then
+// combined pairwise), so four loads per thread are in flight.
 __global__ void reduce_bc_kernel(const Args a) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // row·32 + col
   const long long M = (long long)a.B * a.L;
@@ -603,9 +605,18 @@ __global__ void reduce_bc_kernel(const Args a) {
   const long long row = t >> 5;
   const int col = (int)(t & 31);
   const int nb = a.nbc;
-  float acc = 0.0f;
-  for (int cb = 0; cb < nb; ++cb) acc += a.pbc[((size_t)cb * M + row) * 32 + col];
-  a.dbc[row * a.ld_dbc + col] = acc;
+  const float* p = a.pbc + row * 32 + col;
+  const size_t stride = (size_t)M * 32;
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  int cb = 0;
+  for (; cb + 4 <= nb; cb += 4) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] += p[(size_t)(cb + i) * stride];
+  }
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    if (cb + i < nb) acc[i] += p[(size_t)(cb + i) * stride];
+  a.dbc[row * a.ld_dbc + col] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 }  // namespace sbwd
