@@ -84,6 +84,7 @@ STAGE_SOURCES = {
     "scan": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh", "scan_split.cuh"] + _COMMON,
     "ln_residual": ["simt_kernels.cuh"] + _COMMON,
     "scan_bwd": ["scan_bwd.cu", "scan_bwd.h", "scan_bwd_seq.cuh"] + _COMMON,
+    "scan_general": ["scan_fast.cuh", "scan_fast.h", "scan_launch.cu", "scan_pair.cuh", "scan_split.cuh"] + _COMMON,
 }
 
 
