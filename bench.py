@@ -633,15 +633,20 @@ def cpu_baseline(case, sample_seqs=(0, 1)):
                       f"numpy float64 oracle, {dt:.1f} s"}
 
 
+E2E_BUFFERS = 3  # device buffers of the pipelined host-to-host loop
+
+
 def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev):
     """Tokens/s through r2l_sidecar_forward with the hidden states coming from
     and going back to pinned host memory every step.
 
     value: a pipelined serving loop. Step k's host-to-device copy runs on one
     stream, its forward on another and its device-to-host copy on a third, over
-    two device buffers. So the inbound copy of step k+1 and the outbound copy
-    of step k-1 overlap the forward of step k. The forward calls stay ordered
-    on one stream, so they share one workspace.
+    E2E_BUFFERS device buffers. So the inbound copy of step k+1 and the outbound
+    copy of step k-1 overlap the forward of step k. With three buffers the
+    inbound copy of step k+1 does not wait for the outbound copy of step k-2,
+    so the two directions of the link run at once (with two they alternate).
+    The forward calls stay ordered on one stream, so they share one workspace.
     serial_value: copy in, forward, copy out, one after the other on one stream."""
     import torch
     from reverse_selective_ssm_b200 import binding as bd
@@ -675,11 +680,12 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
     ms_serial = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     # pipelined
-    bufs = [h, torch.empty_like(h)]
+    nb = E2E_BUFFERS
+    bufs = [h] + [torch.empty_like(h) for _ in range(nb - 1)]
     s_in, s_fw, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_fw = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_fw = [torch.cuda.Event() for _ in range(nb)]
+    ev_out = [torch.cuda.Event() for _ in range(nb)]
 
     def pipelined(n, t_start=None, t_end=None):
         if t_start is not None:
@@ -687,9 +693,9 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
             s_fw.wait_event(t_start)
             s_out.wait_event(t_start)
         for k in range(n):
-            i = k & 1
-            if k >= 2:
-                s_in.wait_event(ev_out[i])          # buffer i is free once step k-2 is copied out
+            i = k % nb
+            if k >= nb:
+                s_in.wait_event(ev_out[i])          # buffer i is free once step k-nb is copied out
             with torch.cuda.stream(s_in):
                 bufs[i].copy_(h_host, non_blocking=True)
             ev_in[i].record(s_in)
@@ -705,7 +711,7 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
             s_out.wait_stream(s_fw)
             t_end.record(s_out)
 
-    pipelined(max(2, args.warmup))
+    pipelined(max(nb, args.warmup))
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -718,8 +724,9 @@ def run_e2e(args, case, h, wdev, dims, lengths, ws, stream, barrier, world, dev)
             "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
             "serial_value": round(whole_job_rate(case.valid_tokens, world, K, ms_serial), 1),
             "api": "r2l_sidecar_forward via binding, pinned host hidden in/out",
-            "schedule": "pipelined: copy-in, forward and copy-out of successive steps on three streams over "
-                        "two device buffers (serial_value: one stream, no overlap)"}
+            "device_buffers": nb,
+            "schedule": f"pipelined: copy-in, forward and copy-out of successive steps on three streams over "
+                        f"{nb} device buffers (serial_value: one stream, no overlap)"}
 
 
 # ---------------------------------------------------------------- scan gradient
