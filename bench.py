@@ -424,6 +424,11 @@ def run_ours(args, rank, world, local_rank):
         # always the stream current at call time (the capture stream under a graph)
         st = torch.cuda.current_stream()
         launches = 0
+        if events is None and hooks > 1:
+            # a stack of hooks is one r2l_sidecar_stack call: one length check and
+            # one A_log check for all hooks
+            bd.sidecar_stack(h, wdev, dims, case.s, lengths, ws, st)
+            return launches
         for k in range(hooks):
             if events is not None:
                 launches += bd.sidecar_forward_profiled(h, wdev[k], dims, case.s[k], events[k], lengths, ws, st)
@@ -600,7 +605,8 @@ def run_graph(args, case, step, barrier, rank, world, local_rank, dev):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": {"workload": case.name, "B": case.B, "L": case.L, "hooks": hooks,
-                                         "cuda_graph": True, "per_hook_us": round(ms / K / hooks * 1e3, 2)},
+                                         "cuda_graph": True, "per_hook_us": round(ms / K / hooks * 1e3, 2),
+                                         "api": "r2l_sidecar_stack" if hooks > 1 else "r2l_sidecar_forward"},
         "clocks": clk, "source_sha": source_sha(),
     }
 

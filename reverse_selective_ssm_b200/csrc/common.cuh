@@ -23,6 +23,20 @@ __device__ __forceinline__ float silu_f(float v) { return v / (1.0f + expf(-v));
 // softplus(v) = log(1 + exp(v)), and v itself above 20 (Δ parameterisation).
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
 
+// Programmatic dependent launch.  grid_dep_wait: block until the grids this
+// one was launched behind have completed and their writes are visible (it
+// returns at once in a grid launched without the programmatic attribute).
+// grid_dep_launch: let the next grid of the stream, when launched with the
+// attribute, start once every CTA of this grid has issued it or exited.
+// A kernel launched with the attribute (launch_pdl.h) calls grid_dep_wait
+// before it touches global memory that earlier kernels of the stream write or
+// read, and before it allocates tensor memory; it calls grid_dep_launch only
+// after its own grid_dep_wait.  So at most two grids of a stream are resident
+// at once, the later one waiting, and a tensor-memory allocation never waits
+// for a grid that is still running.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Row m = b*L + i of a right-padded [B, L, ·] batch is valid when i < len[b].
 __device__ __forceinline__ bool row_valid(const int* len, int L, long long m) {
   const long long b = m / L;

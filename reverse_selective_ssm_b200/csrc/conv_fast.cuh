@@ -71,6 +71,8 @@ __global__ void __launch_bounds__(THREADS)
 conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u, int E,
                       const float* __restrict__ conv_w, const float* __restrict__ conv_b,
                       const int* __restrict__ len, int L) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int cg = blockIdx.x * THREADS + threadIdx.x;
   const int c0 = cg * 8;
   const int t0 = blockIdx.y * CT;

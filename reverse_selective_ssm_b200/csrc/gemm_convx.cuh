@@ -192,11 +192,13 @@ gemm_convx_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     sm100::prefetch_tmap(&tmW4);
     sm100::prefetch_tmap(&tmCB);
   }
+  grid_dep_wait();
   if (warp == 1) sm100::tmem_alloc(tmem_slot, TMEM_COLS);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_launch();
 
   auto tile_live = [&](long long t) -> bool {
     if (!a.len) return true;

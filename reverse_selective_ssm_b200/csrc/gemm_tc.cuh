@@ -189,11 +189,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     sm100::prefetch_tmap(&tmB);
     sm100::prefetch_tmap(&tmC);
   }
+  grid_dep_wait();
   if (warp == 1) sm100::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_launch();
 
   auto tile_live = [&](long long t) -> bool {
     if (!len) return true;

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "simt_kernels.cuh"
 #include "scan_simple.cuh"
+#include "launch_pdl.h"
 #include "tc_gemm.h"
 #include "scan_fast.h"
 #include "scan_bwd.h"
@@ -217,10 +218,12 @@ r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long l
 template <int NV>
 r2l_status ln_bf16_nv(bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o, const float* lw,
                       const float* lb, float g, int d, const int* len, int L, long long M, float* hhat) {
-  if (has_ln)
-    r2l::ln_residual_bf16_kernel<NV, true><<<blocks, 128, 0, st>>>(h, o, lw, lb, g, d, len, L, M, hhat);
-  else
-    r2l::ln_residual_bf16_kernel<NV, false><<<blocks, 128, 0, st>>>(h, o, lw, lb, g, d, len, L, M, hhat);
+  const cudaError_t e =
+      has_ln ? r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, true>, dim3(blocks), dim3(128), 0, st, h, o, lw, lb, g,
+                               d, len, L, M, hhat)
+             : r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, false>, dim3(blocks), dim3(128), 0, st, h, o, lw, lb,
+                               g, d, len, L, M, hhat);
+  if (e != cudaSuccess) return R2L_ERR_CUDA;
   R2L_LAUNCH_CHECK();
   return R2L_OK;
 }
@@ -288,10 +291,12 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     if constexpr (kTC) {
       namespace cv = r2l::conv;
       dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
-      if (fwd)
-        cv::conv_silu_bf16_kernel<true><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
-      else
-        cv::conv_silu_bf16_kernel<false><<<grid, cv::THREADS, 0, st>>>(xz, 2 * E, u, E, w->conv_w, w->conv_b, len, L);
+      const cudaError_t e =
+          fwd ? r2l::launch_pdl(cv::conv_silu_bf16_kernel<true>, grid, dim3(cv::THREADS), 0, st, (const bf16*)xz, 2 * E,
+                                u, E, (const float*)w->conv_w, (const float*)w->conv_b, (const int*)len, L)
+              : r2l::launch_pdl(cv::conv_silu_bf16_kernel<false>, grid, dim3(cv::THREADS), 0, st, (const bf16*)xz,
+                                2 * E, u, E, (const float*)w->conv_w, (const float*)w->conv_b, (const int*)len, L);
+      if (e != cudaSuccess) return R2L_ERR_CUDA;
       R2L_LAUNCH_CHECK();
     } else {
       dim3 grid((E + 127) / 128, L, B);

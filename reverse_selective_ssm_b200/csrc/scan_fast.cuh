@@ -500,6 +500,8 @@ __device__ __forceinline__ uint32_t opnd_row(int n) { return (uint32_t)((n >> 3)
 // each chunk from the right (from the left with fwd), in place (see the
 // header comment, step 2).
 __global__ void chunk_carry_kernel(const Params p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
   if (c >= p.E) return;

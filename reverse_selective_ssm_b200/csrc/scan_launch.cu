@@ -2,6 +2,7 @@
 // descriptors for the u / z / dt_raw / B|C tiles, and the launch sequence.
 #include <cuda.h>
 
+#include "launch_pdl.h"
 #include "scan_fast.cuh"
 #include "scan_fast.h"
 #include "scan_pair.cuh"
@@ -124,16 +125,20 @@ cudaError_t launch_pair(const ScanArgs& a, const rscan::Params& p, int nc, cudaS
     if ((e = cudaFuncSetAttribute(pair::scan_pair_kernel<false, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)Sp::BYTES)) != cudaSuccess)
       return e;
-    pair::scan_pair_kernel<false, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-    chunk_carry_kernel<<<dim3((a.E + 127) / 128, a.B), 128, 0, st>>>(p);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(pair::scan_pair_kernel<false, FWD>, grid, dim3(Sp::THREADS), Sp::BYTES, st, tu, tz, tdr,
+                        tbc, ty, tw, p)) != cudaSuccess)
+      return e;
+    if ((e = launch_pdl(chunk_carry_kernel, dim3((a.E + 127) / 128, a.B), dim3(128), 0, st, p)) != cudaSuccess)
+      return e;
     if (launches) *launches += 2;
   }
   if (ckpt)
-    pair::scan_pair_kernel<true, false, true><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+    e = launch_pdl(pair::scan_pair_kernel<true, false, true>, grid, dim3(Sp::THREADS), Sp::BYTES, st, tu, tz, tdr,
+                   tbc, ty, tw, p);
   else
-    pair::scan_pair_kernel<true, FWD><<<grid, Sp::THREADS, Sp::BYTES, st>>>(tu, tz, tdr, tbc, ty, tw, p);
+    e = launch_pdl(pair::scan_pair_kernel<true, FWD>, grid, dim3(Sp::THREADS), Sp::BYTES, st, tu, tz, tdr, tbc, ty,
+                   tw, p);
+  if (e != cudaSuccess) return e;
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaSuccess;

@@ -401,6 +401,8 @@ scan_pair_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant
   uint64_t* bcfree = bcready + NG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::SLOT);
 
+  grid_dep_wait();
+  grid_dep_launch();
   const int cb = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;

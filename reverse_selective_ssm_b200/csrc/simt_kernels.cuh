@@ -232,6 +232,8 @@ __global__ void __launch_bounds__(128)
 ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const float* __restrict__ ln_w,
                         const float* __restrict__ ln_b, float g, int d, const int* __restrict__ len, int L,
                         long long M, float* __restrict__ hhat_out) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;

@@ -6,17 +6,19 @@
 
 #include "gemm_convx.cuh"
 #include "gemm_tc.cuh"
+#include "launch_pdl.h"
 #include "tc_gemm.h"
 #include "tmap.h"
 
 namespace r2l {
-namespace {
 
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
 }
+
+namespace {
 
 // 256 × 256 tiles (two M = 128 MMA blocks per CTA) for 256-multiple N (0: 128 × BN only).
 #ifndef R2L_GEMM_MB2
@@ -36,6 +38,8 @@ int sm_count() {
 __global__ void splitk_sum_kernel(const float* __restrict__ P, int splits, long long Mp, int N,
                                   float* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols,
                                   int M, const int* __restrict__ len, int L) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int m = blockIdx.x;
   if (m >= M) return;
   const bool valid = !len || row_valid(len, L, m);
@@ -44,6 +48,45 @@ __global__ void splitk_sum_kernel(const float* __restrict__ P, int splits, long 
     for (int sp = 0; sp < splits; ++sp) acc += P[((long long)sp * Mp + m) * N + c];
     C[(long long)m * ldc + c] = acc;
     if (C2 && valid && c < c2_cols) C2[(long long)m * ldc2 + c] = __float2bfloat16_rn(acc);
+  }
+}
+
+// The same sum, four columns per thread (N and ldc multiples of 4, P and C
+// 16-byte aligned): up to eight slices' loads are in flight before their adds,
+// which keep the order above, so both kernels give the same bits.
+__global__ void splitk_sum4_kernel(const float* __restrict__ P, int splits, long long Mp, int N,
+                                   float* __restrict__ C, int ldc, bf16* __restrict__ C2, int ldc2, int c2_cols,
+                                   int M, const int* __restrict__ len, int L) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int n4 = N >> 2;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)M * n4) return;
+  const int m = (int)(idx / n4);
+  const int c = (int)(idx - (long long)m * n4) * 4;
+  const float* p = P + (long long)m * N + c;
+  const long long slice = Mp * N;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (s0 + i < splits) v[i] = *reinterpret_cast<const float4*>(p + (s0 + i) * slice);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (s0 + i < splits) {
+        acc.x += v[i].x;
+        acc.y += v[i].y;
+        acc.z += v[i].z;
+        acc.w += v[i].w;
+      }
+  }
+  *reinterpret_cast<float4*>(C + (long long)m * ldc + c) = acc;
+  if (C2 && c < c2_cols && (!len || row_valid(len, L, m))) {
+    const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (c + i < c2_cols) C2[(long long)m * ldc2 + c + i] = __float2bfloat16_rn(a[i]);
   }
 }
 
@@ -101,12 +144,23 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   const long long units = tiles * splits;
   const int grid = (int)(units < sm_count() ? units : sm_count());
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(ta, tb, tc, g.C2, g.ldc2, g.c2_cols,
-                                            g.M, g.N, g.K, g.len, g.L, g.err, splits);
+  const cudaError_t el = launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, ta, tb, tc, g.C2,
+                                    g.ldc2, g.c2_cols, g.M, g.N, g.K, g.len, g.L, g.err, splits);
+  if (el != cudaSuccess) return el;
   cudaError_t e2 = cudaPeekAtLastError();
   if (e2 != cudaSuccess || splits == 1) return e2;
-  splitk_sum_kernel<<<g.M, 128, 0, st>>>(g.partial, splits, num_m * Cfg::BM, g.N, reinterpret_cast<float*>(g.C),
-                                         g.ldc, g.C2, g.ldc2, g.c2_cols, g.M, g.len, g.L);
+  if (((g.N | g.ldc) & 3) == 0 && ((reinterpret_cast<uintptr_t>(g.partial) | reinterpret_cast<uintptr_t>(g.C)) & 15) == 0) {
+    const long long n = (long long)g.M * (g.N / 4);
+    const cudaError_t es = launch_pdl(splitk_sum4_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
+                                      (const float*)g.partial, splits, (long long)(num_m * Cfg::BM), g.N,
+                                      reinterpret_cast<float*>(g.C), g.ldc, g.C2, g.ldc2, g.c2_cols, g.M, g.len, g.L);
+    if (es != cudaSuccess) return es;
+  } else {
+    const cudaError_t es = launch_pdl(splitk_sum_kernel, dim3((unsigned)g.M), dim3(128), 0, st,
+                                      (const float*)g.partial, splits, (long long)(num_m * Cfg::BM), g.N,
+                                      reinterpret_cast<float*>(g.C), g.ldc, g.C2, g.ldc2, g.c2_cols, g.M, g.len, g.L);
+    if (es != cudaSuccess) return es;
+  }
   return cudaPeekAtLastError();
 }
 
@@ -114,10 +168,11 @@ template <typename TOut>
 cudaError_t dispatch(const TcGemm& g, cudaStream_t st) {
   // widest tile that divides N; else the narrowest that covers it; else 256 with a ragged edge
   if (g.N % 256 == 0) {
-    // 256 × 256 tiles only when there are enough of them to give every SM one
+    // 256 × 256 tiles when there are enough of them for three SMs in four: one
+    // wave of them beats 1.7 waves of 128 × 256 tiles (M = 1024, N = 8192)
     if constexpr (std::is_same<TOut, bf16>::value)
       if (R2L_GEMM_MB2 && g.K >= R2L_GEMM_MB2_MIN_K &&
-          (long long)((g.M + 255) / 256) * (g.N / 256) >= sm_count())
+          (long long)((g.M + 255) / 256) * (g.N / 256) * 4 >= (long long)sm_count() * 3)
         return launch<256, TOut, 2>(g, st);
     // fewer 128 × 256 tiles than SMs: 128-wide tiles give twice as many
     if ((long long)((g.M + 127) / 128) * (g.N / 256) < sm_count()) return launch<128, TOut>(g, st);
@@ -166,7 +221,8 @@ cudaError_t launch_convx(const ConvX& g, cudaStream_t st) {
   a.x = g.x; a.ldx = g.ldx; a.conv_w = g.conv_w; a.conv_b = g.conv_b; a.u = g.u; a.ldu = g.ldu;
   a.M = g.M; a.K = g.E; a.C2 = g.C2; a.ldc2 = g.ldc2; a.c2_cols = g.c2_cols; a.len = g.len; a.L = g.L;
   a.err = g.err;
-  kern<<<grid, cx::THREADS, cx::SMEM_BYTES, st>>>(tx, tb, tc, tw4, tcb, a);
+  const cudaError_t el = launch_pdl(kern, dim3(grid), dim3(cx::THREADS), cx::SMEM_BYTES, st, tx, tb, tc, tw4, tcb, a);
+  if (el != cudaSuccess) return el;
   return cudaPeekAtLastError();
 }
 

@@ -28,6 +28,9 @@ struct TcGemm {
   size_t partial_bytes;
 };
 
+// Streaming multiprocessors of the current device (148 on B200).
+int sm_count();
+
 // Scratch an fp32-output GEMM of this shape uses for split-K partial sums
 // (0 when it runs unsplit).  With less, it runs unsplit.
 size_t tc_gemm_partial_bytes(long long M, int N, int K);
