@@ -39,8 +39,9 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Byte offsets of the workspace regions for a [B, L] batch.
 struct Plan {
-  size_t status, len, aflags, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, total;
+  size_t status, len, aflags, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, osplit, osplit_bytes, total;
   int chunk_tokens;  // scan chunk length (bf16 path)
+  int osplits;       // out_proj K splits left to the LayerNorm kernel (0: o stored by the GEMM)
   long long M;
   int E, d, R, N, ldd;
   size_t act;
@@ -81,6 +82,12 @@ bool make_plan(const r2l_dims* dm, int B, int L, Plan* p) {
   p->xsplit = off;
   p->xsplit_bytes = dm->dtype == R2L_BF16 ? r2l::tc_gemm_partial_bytes(p->M, p->ldd, p->E) : 0;
   off = align_up(off + p->xsplit_bytes, kAlign);
+  // out_proj of a batch whose 128 × 256 tiles do not fill the SMs (bf16 path,
+  // d ≤ 2048): K-split fp32 partial sums that the LayerNorm kernel adds
+  p->osplits = dm->dtype == R2L_BF16 && p->d <= 2048 ? r2l::tc_gemm_kept_splits(p->M, p->d, p->E) : 0;
+  p->osplit = off;
+  p->osplit_bytes = (size_t)p->osplits * (size_t)((p->M + 127) / 128 * 128) * p->d * sizeof(float);
+  off = align_up(off + p->osplit_bytes, kAlign);
   p->total = off;
   return true;
 }
@@ -215,14 +222,26 @@ r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long l
 }
 
 // LayerNorm + gated residual for bf16 rows of d <= 2048 (nv = ceil(d / 256)).
+// With ps (the out_proj partial sums of a small batch, `splits` slices of
+// `slice` floats) o is added up from them, and written to `o` only when
+// o_keep is set (the debug entry point).
 template <int NV>
 r2l_status ln_bf16_nv(bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o, const float* lw,
-                      const float* lb, float g, int d, const int* len, int L, long long M, float* hhat) {
-  const cudaError_t e =
-      has_ln ? r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, true>, dim3(blocks), dim3(128), 0, st, h, o, lw, lb, g,
-                               d, len, L, M, hhat)
-             : r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, false>, dim3(blocks), dim3(128), 0, st, h, o, lw, lb,
-                               g, d, len, L, M, hhat);
+                      const float* lb, float g, int d, const int* len, int L, long long M, float* hhat,
+                      const float* ps, int splits, long long slice, bool o_keep) {
+  cudaError_t e;
+  const dim3 grid(blocks), block(128);
+  bf16* o_out = o_keep ? const_cast<bf16*>(o) : nullptr;
+  if (ps)
+    e = has_ln ? r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, true, true>, grid, block, 0, st, h, o, lw, lb, g, d,
+                                 len, L, M, hhat, ps, splits, slice, o_out)
+               : r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, false, true>, grid, block, 0, st, h, o, lw, lb, g, d,
+                                 len, L, M, hhat, ps, splits, slice, o_out);
+  else
+    e = has_ln ? r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, true>, grid, block, 0, st, h, o, lw, lb, g, d, len,
+                                 L, M, hhat, (const float*)nullptr, 0, 0LL, (bf16*)nullptr)
+               : r2l::launch_pdl(r2l::ln_residual_bf16_kernel<NV, false>, grid, block, 0, st, h, o, lw, lb, g, d, len,
+                                 L, M, hhat, (const float*)nullptr, 0, 0LL, (bf16*)nullptr);
   if (e != cudaSuccess) return R2L_ERR_CUDA;
   R2L_LAUNCH_CHECK();
   return R2L_OK;
@@ -230,16 +249,17 @@ r2l_status ln_bf16_nv(bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, co
 
 r2l_status launch_ln_bf16(int nv, bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o,
                           const float* lw, const float* lb, float g, int d, const int* len, int L, long long M,
-                          float* hhat) {
+                          float* hhat, const float* ps = nullptr, int splits = 0, long long slice = 0,
+                          bool o_keep = false) {
   switch (nv) {
-    case 1: return ln_bf16_nv<1>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 2: return ln_bf16_nv<2>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 3: return ln_bf16_nv<3>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 4: return ln_bf16_nv<4>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 5: return ln_bf16_nv<5>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 6: return ln_bf16_nv<6>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    case 7: return ln_bf16_nv<7>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
-    default: return ln_bf16_nv<8>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat);
+    case 1: return ln_bf16_nv<1>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 2: return ln_bf16_nv<2>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 3: return ln_bf16_nv<3>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 4: return ln_bf16_nv<4>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 5: return ln_bf16_nv<5>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 6: return ln_bf16_nv<6>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    case 7: return ln_bf16_nv<7>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
+    default: return ln_bf16_nv<8>(has_ln, blocks, st, h, o, lw, lb, g, d, len, L, M, hhat, ps, splits, slice, o_keep);
   }
 }
 
@@ -353,10 +373,30 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
                                                      w->D, w->dt_proj_b, y, E, len, L, fwd);
     R2L_LAUNCH_CHECK();
   }
-  // a6: o = y · W_outᵀ
+  // a6: o = y · W_outᵀ.  A small batch (few 128 × 256 tiles) splits K and
+  // leaves fp32 partial sums, which the LayerNorm kernel adds (and stores o
+  // from); without the LayerNorm step (the gradient's recomputed forward) the
+  // split-K sum kernel stores o, with the same additions in the same order.
   R2L_TRY(prof->mark(R2L_STAGE_OUT_PROJ, st));
   prof->launches++;
-  R2L_TRY(proj(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, err, st));
+  const bool osplit = kTC && p.osplits > 0 && d <= 2048;
+  const long long Mp = (M + 127) / 128 * 128;
+  if (osplit) {
+    r2l::TcGemm gm{};
+    gm.A = (const bf16*)y; gm.lda = E; gm.B = (const bf16*)w->out_proj_w; gm.ldb = E;
+    gm.C = nullptr; gm.ldc = d; gm.c_fp32 = true; gm.keep_partials = true;
+    gm.M = (int)M; gm.N = d; gm.K = E; gm.len = len; gm.L = L; gm.err = err;
+    gm.partial = (float*)(ws + p.osplit); gm.partial_bytes = p.osplit_bytes;
+    if (r2l::tc_gemm(gm, st) != cudaSuccess) return R2L_ERR_CUDA;
+    if (!residual) {
+      prof->launches++;
+      float* ps = (float*)(ws + p.osplit);
+      if (r2l::tc_gemm_add_partials(ps, p.osplits, Mp, d, ps, d, (bf16*)o, d, d, (int)M, len, L, st) != cudaSuccess)
+        return R2L_ERR_CUDA;
+    }
+  } else {
+    R2L_TRY(proj(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, err, st));
+  }
 
   if (dbg) {
     const size_t rowsE = (size_t)M;
@@ -365,7 +405,10 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     if (dbg->u && cudaMemcpyAsync(dbg->u, u, rowsE * E * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
     if (dbg->dbc && cudaMemcpyAsync(dbg->dbc, dbc, rowsE * p.ldd * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
     if (dbg->y && cudaMemcpyAsync(dbg->y, y, rowsE * E * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
-    if (dbg->o && cudaMemcpyAsync(dbg->o, o, rowsE * d * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return R2L_ERR_CUDA;
+    // with the split out_proj and the LayerNorm step, o is copied once that has stored it
+    if (dbg->o && !(osplit && residual) &&
+        cudaMemcpyAsync(dbg->o, o, rowsE * d * es, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return R2L_ERR_CUDA;
   }
   // stop here when only the intermediates are wanted (the hook's gradient)
   if (!residual) return R2L_OK;
@@ -377,7 +420,11 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     const unsigned blocks = (unsigned)((M + 3) / 4);
     const int nv = (d + 255) / 256;
     R2L_TRY(launch_ln_bf16(nv, w->ln_w != nullptr, blocks, st, (bf16*)hidden, (const bf16*)o, w->ln_w, w->ln_b,
-                           g, d, len, L, M, hhat));
+                           g, d, len, L, M, hhat, osplit ? (const float*)(ws + p.osplit) : nullptr, p.osplits,
+                           Mp * d, osplit));
+    if (osplit && dbg && dbg->o &&
+        cudaMemcpyAsync(dbg->o, o, (size_t)M * d * sizeof(T), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return R2L_ERR_CUDA;
   } else if (w->ln_w) {
     r2l::ln_gate_residual_kernel<T, true><<<(unsigned)M, 256, 0, st>>>(hidden, o, w->ln_w, w->ln_b, g, d, len, L, hhat);
     R2L_LAUNCH_CHECK();

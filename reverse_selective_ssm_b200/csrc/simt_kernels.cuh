@@ -227,11 +227,17 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int NV, bool HAS_LN>
+// SPLIT: o arrives as `splits` fp32 partial sums P[s][row][col] (slices of
+// `slice` floats, the K-split out_proj of a small batch); the row's o is their
+// sum in split order rounded to bf16, the value the unsplit GEMM would have
+// stored up to the order of its fp32 additions, and it is written to o_out
+// when that is set.
+template <int NV, bool HAS_LN, bool SPLIT = false>
 __global__ void __launch_bounds__(128)
 ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const float* __restrict__ ln_w,
                         const float* __restrict__ ln_b, float g, int d, const int* __restrict__ len, int L,
-                        long long M, float* __restrict__ hhat_out) {
+                        long long M, float* __restrict__ hhat_out, const float* __restrict__ P = nullptr,
+                        int splits = 0, long long slice = 0, bf16* __restrict__ o_out = nullptr) {
   grid_dep_wait();
   grid_dep_launch();
   const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -247,11 +253,48 @@ ln_residual_bf16_kernel(bf16* __restrict__ h, const bf16* __restrict__ o, const 
   for (int k = 0; k < NV; ++k) {
     const int col = (k * 32 + lane) * 8;
     if (col < d) {
-      oraw[k] = *reinterpret_cast<const uint4*>(orow + col);
+      if (!SPLIT) oraw[k] = *reinterpret_cast<const uint4*>(orow + col);
       hraw_all[k] = *reinterpret_cast<const uint4*>(hrow + col);
     }
   }
   float v[NV][8];
+  if (SPLIT) {
+    // slice by slice, all of a slice's loads of the row in flight at once
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[k][q] = 0.0f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float* prow = P + sp * slice + row * d;
+      float4 pr[NV][2];
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int col = (k * 32 + lane) * 8;
+        if (col < d) {
+          pr[k][0] = *reinterpret_cast<const float4*>(prow + col);
+          pr[k][1] = *reinterpret_cast<const float4*>(prow + col + 4);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int col = (k * 32 + lane) * 8;
+        if (col < d) {
+          v[k][0] += pr[k][0].x; v[k][1] += pr[k][0].y; v[k][2] += pr[k][0].z; v[k][3] += pr[k][0].w;
+          v[k][4] += pr[k][1].x; v[k][5] += pr[k][1].y; v[k][6] += pr[k][1].z; v[k][7] += pr[k][1].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int col = (k * 32 + lane) * 8;
+      if (col < d) {
+        __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&oraw[k]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o2[q] = __floats2bfloat162_rn(v[k][2 * q], v[k][2 * q + 1]);
+        if (o_out) *reinterpret_cast<uint4*>(o_out + row * d + col) = oraw[k];
+      }
+    }
+  }
   float s = 0.0f;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {

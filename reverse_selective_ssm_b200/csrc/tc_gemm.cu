@@ -90,6 +90,31 @@ __global__ void splitk_sum4_kernel(const float* __restrict__ P, int splits, long
   }
 }
 
+}  // namespace
+
+cudaError_t tc_gemm_add_partials(const float* P, int splits, long long Mp, int N, float* C, int ldc, bf16* C2,
+                                 int ldc2, int c2_cols, int M, const int* len, int L, cudaStream_t st) {
+  if ((N | ldc) & 3 || ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(C)) & 15)) return cudaErrorInvalidValue;
+  const long long n = (long long)M * (N / 4);
+  if (n <= 0) return cudaSuccess;
+  return launch_pdl(splitk_sum4_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, P, splits, Mp, N, C, ldc,
+                    C2, ldc2, c2_cols, M, len, L);
+}
+
+int tc_gemm_kept_splits(long long M, int N, int K) {
+  if (N % 256 != 0 || M <= 0) return 0;
+  const long long tiles = (M + 127) / 128 * (N / 256);
+  const int sms = sm_count();
+  if (tiles >= sms) return 0;
+  const int num_k = (K + 63) / 64;
+  int sp = (int)(sms / tiles);             // one wave of (tile, split) units
+  if (sp > 8) sp = 8;
+  while (sp > 1 && num_k / sp < 8) --sp;
+  return sp < 1 ? 1 : sp;
+}
+
+namespace {
+
 int tile_width(int N) {   // the BN dispatch() picks for an fp32-output GEMM of this width
   if (N % 256 == 0) return 256;
   if (N <= 64) return 64;
@@ -123,7 +148,8 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   if (BMN ? !make_tmap_2d(&tb, g.B, 2, g.N, g.K, (long long)g.ldb * 2, 64, Cfg::BK, 128)
           : !make_tmap_2d(&tb, g.B, 2, g.K, g.N, (long long)g.ldb * 2, Cfg::BK, BN, 128))
     return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tc, g.C, (int)sizeof(TOut), g.N, g.M, (long long)g.ldc * sizeof(TOut), 32, 32, Cfg::STG_SWIZZLE))
+  if (!g.keep_partials &&
+      !make_tmap_2d(&tc, g.C, (int)sizeof(TOut), g.N, g.M, (long long)g.ldc * sizeof(TOut), 32, 32, Cfg::STG_SWIZZLE))
     return cudaErrorInvalidValue;
   auto kern = gemm_tc_kernel<BN, TOut, MB, AMN, BMN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
@@ -132,7 +158,18 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   const long long tiles = num_m * ((g.N + BN - 1) / BN);
   int splits = 1;
   if constexpr (std::is_same<TOut, float>::value) {
-    const int sp = choose_splits(tiles, (g.K + Cfg::BK - 1) / Cfg::BK);
+    if (g.keep_partials) {
+      const int sp = tc_gemm_kept_splits(g.M, g.N, g.K);
+      const size_t need = (size_t)sp * num_m * Cfg::BM * g.N * sizeof(float);
+      if (BN != 256 || MB != 1 || sp < 1 || !g.partial || g.partial_bytes < need) return cudaErrorInvalidValue;
+      splits = sp;
+      if (!make_tmap_2d(&tc, g.partial, 4, g.N, (long long)sp * num_m * Cfg::BM, (long long)g.N * 4, 32, 32,
+                        Cfg::STG_SWIZZLE))
+        return cudaErrorInvalidValue;
+    }
+  }
+  if constexpr (std::is_same<TOut, float>::value) {
+    const int sp = g.keep_partials ? 1 : choose_splits(tiles, (g.K + Cfg::BK - 1) / Cfg::BK);
     const size_t need = (size_t)sp * num_m * Cfg::BM * g.N * sizeof(float);
     if (R2L_GEMM_SPLITK && sp > 1 && g.partial && g.partial_bytes >= need) {
       splits = sp;
@@ -148,7 +185,7 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
                                     g.ldc2, g.c2_cols, g.M, g.N, g.K, g.len, g.L, g.err, splits);
   if (el != cudaSuccess) return el;
   cudaError_t e2 = cudaPeekAtLastError();
-  if (e2 != cudaSuccess || splits == 1) return e2;
+  if (e2 != cudaSuccess || splits == 1 || g.keep_partials) return e2;
   if (((g.N | g.ldc) & 3) == 0 && ((reinterpret_cast<uintptr_t>(g.partial) | reinterpret_cast<uintptr_t>(g.C)) & 15) == 0) {
     const long long n = (long long)g.M * (g.N / 4);
     const cudaError_t es = launch_pdl(splitk_sum4_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st,
@@ -249,6 +286,10 @@ cudaError_t tc_gemm(const TcGemm& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return cudaSuccess;
   // TMA: 16-byte row strides; a K-major operand's K is its inner extent
   if ((g.lda % 8) || (g.ldb % 8) || (!g.a_mn && (g.K % 8))) return cudaErrorInvalidValue;
+  if (g.keep_partials) {
+    if (!g.c_fp32 || g.a_mn || g.b_mn || g.C2) return cudaErrorInvalidValue;
+    return launch<256, float>(g, st);
+  }
   if ((g.ldc * (g.c_fp32 ? 4 : 2)) % 16) return cudaErrorInvalidValue;
   if (g.a_mn || g.b_mn) {
     if (!g.c_fp32 || !g.a_mn || g.C2) return cudaErrorInvalidValue;

@@ -26,10 +26,26 @@ struct TcGemm {
   unsigned* err;           // device status word (timeout flag)
   float* partial;          // optional scratch for split-K partial sums (fp32 C only), or null
   size_t partial_bytes;
+  // keep_partials (fp32 C only): run on 128 × 256 tiles with tc_gemm_kept_splits
+  // splits and leave the partial sums in `partial` as [splits][Mp][N], Mp = M
+  // rounded up to 128, for the caller to add in split order; C is not written.
+  bool keep_partials;
 };
 
 // Streaming multiprocessors of the current device (148 on B200).
 int sm_count();
+
+// C2[m, c] = bf16(Σ_s P[s·Mp + m, c]) for c < c2_cols on valid rows (and C = the
+// fp32 sum, which may be P itself), slices added in split order: the sum a
+// keep_partials GEMM leaves to its caller.
+cudaError_t tc_gemm_add_partials(const float* P, int splits, long long Mp, int N, float* C, int ldc,
+                                 __nv_bfloat16* C2, int ldc2, int c2_cols, int M, const int* len, int L,
+                                 cudaStream_t st);
+
+// Splits a keep_partials GEMM of this shape uses: 0 when N is not a multiple
+// of 256 or its 128 × 256 tiles alone fill the SMs; else the fewest splits (at
+// most 8, each of at least 8 K blocks of 64) that give every SM a unit.
+int tc_gemm_kept_splits(long long M, int N, int K);
 
 // Scratch an fp32-output GEMM of this shape uses for split-K partial sums
 // (0 when it runs unsplit).  With less, it runs unsplit.

@@ -2,8 +2,9 @@
 x_proj runs on its own, unsplit or split along K) against the oracle of
 "Bifocal Diffusion Language Models" (arXiv 2606.27732v1, §3.4 steps ❶–❷), at
 three batch sizes: 9600, 3200 and 600 tokens.  Lengths end part-way through a
-thread's 16 tokens; u, Δr, C and y are compared, in both directions, and
-padding rows of h must stay untouched."""
+thread's 16 tokens; u, Δr, C, y, o and ĥ are compared, in both directions,
+and padding rows of h must stay untouched.  At 600 tokens out_proj also runs
+split along K, its partial sums added by the LayerNorm kernel."""
 import numpy as np
 import pytest
 import torch
@@ -65,7 +66,9 @@ def test_conv_small_batches(shape, direction):
         for name, g, w in [("u", S.to_f64(dbg["u"][rows]), inter[b]["u"]),
                            ("dr", dbc[:, :R], inter[b]["dr"]),
                            ("C", dbc[:, R + 16:R + 32], inter[b]["C"]),
-                           ("y", S.to_f64(dbg["y"][rows]), inter[b]["y"])]:
+                           ("y", S.to_f64(dbg["y"][rows]), inter[b]["y"]),
+                           ("o", S.to_f64(dbg["o"][rows]), inter[b]["o"]),
+                           ("hhat", S.to_f64(dbg["hhat"][rows]), inter[b]["hhat"])]:
             if direction == "l2r":
                 w = _flip_rows(w, n)
             e = G.err_norm(g, w)
