@@ -2,9 +2,11 @@
 //   u[i, c] = SiLU(conv_b[c] + Σ_{k=0..3} conv_w[c, 3-k] · x[i+k, c]),   x[j] = 0 for j ≥ len
 // ("Bifocal Diffusion Language Models", arXiv 2606.27732v1, §3.4 steps ❶–❷:
 // the Mamba-1 causal conv seen through the flip).  One thread covers 8
-// channels (16-byte loads and stores) × CT consecutive tokens and keeps the
-// CT + 3 input rows it needs in registers (as packed bf16, unpacked per use),
-// all requested before the first output is computed.
+// channels (16-byte loads and stores) × NT consecutive tokens and keeps the
+// NT + 3 input rows it needs in registers (as packed bf16, unpacked per use),
+// all requested before the first output is computed.  NT = 16, or 8 when 16
+// would give fewer than two blocks per SM (a denoising block of 1024 tokens:
+// 512 blocks instead of 256 spread the work over the SMs more evenly).
 #pragma once
 
 #include "common.cuh"
@@ -12,8 +14,13 @@
 namespace r2l {
 namespace conv {
 
-constexpr int CT = 16;       // tokens per thread
 constexpr int THREADS = 128;
+
+// Tokens per thread for a grid over B sequences of L tokens and E channels.
+inline int tokens_per_thread(int B, int L, int E, int sms) {
+  const long long blocks16 = (long long)((E / 8 + THREADS - 1) / THREADS) * ((L + 15) / 16) * B;
+  return blocks16 < 2LL * sms ? 8 : 16;
+}
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -66,7 +73,7 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
 
 // x: row stride ldx (elements, multiple of 8); u: [B·L, E].  E % 8 == 0.
 // FWD: the causal conv of the left-to-right block (taps on x[i-k], x[j<0] = 0).
-template <bool FWD>
+template <bool FWD, int NT>
 __global__ void __launch_bounds__(THREADS)
 conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u, int E,
                       const float* __restrict__ conv_w, const float* __restrict__ conv_b,
@@ -75,7 +82,7 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
   grid_dep_launch();
   const int cg = blockIdx.x * THREADS + threadIdx.x;
   const int c0 = cg * 8;
-  const int t0 = blockIdx.y * CT;
+  const int t0 = blockIdx.y * NT;
   const int b = blockIdx.z;
   const int n = len[b];
   if (c0 >= E || t0 >= n) return;
@@ -97,9 +104,9 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
   const long long row0 = (long long)b * L + t0;
   // window rows: token t0 + r (reverse block) or t0 - 3 + r (forward block)
   const int first = FWD ? t0 - 3 : t0;
-  uint4 xr[CT + 3];
+  uint4 xr[NT + 3];
 #pragma unroll
-  for (int r = 0; r < CT + 3; ++r) {
+  for (int r = 0; r < NT + 3; ++r) {
     const int tok = first + r;
     xr[r] = (tok >= 0 && tok < n) ? *reinterpret_cast<const uint4*>(x + ((long long)b * L + tok) * ldx + c0)
                                   : make_uint4(0u, 0u, 0u, 0u);
@@ -112,7 +119,7 @@ conv_silu_bf16_kernel(const bf16* __restrict__ x, int ldx, bf16* __restrict__ u,
     win[k][2] = bf2_to_f2(xr[k].z); win[k][3] = bf2_to_f2(xr[k].w);
   }
 #pragma unroll
-  for (int t = 0; t < CT; ++t) {
+  for (int t = 0; t < NT; ++t) {
     {
       const int r = (t + 3) & 3;
       win[r][0] = bf2_to_f2(xr[t + 3].x); win[r][1] = bf2_to_f2(xr[t + 3].y);

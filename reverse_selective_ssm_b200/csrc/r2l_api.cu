@@ -310,12 +310,12 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
     prof->launches++;
     if constexpr (kTC) {
       namespace cv = r2l::conv;
-      dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + cv::CT - 1) / cv::CT, B);
-      const cudaError_t e =
-          fwd ? r2l::launch_pdl(cv::conv_silu_bf16_kernel<true>, grid, dim3(cv::THREADS), 0, st, (const bf16*)xz, 2 * E,
-                                u, E, (const float*)w->conv_w, (const float*)w->conv_b, (const int*)len, L)
-              : r2l::launch_pdl(cv::conv_silu_bf16_kernel<false>, grid, dim3(cv::THREADS), 0, st, (const bf16*)xz,
-                                2 * E, u, E, (const float*)w->conv_w, (const float*)w->conv_b, (const int*)len, L);
+      const int nt = cv::tokens_per_thread(B, L, E, r2l::sm_count());
+      const dim3 grid((E / 8 + cv::THREADS - 1) / cv::THREADS, (L + nt - 1) / nt, B);
+      auto kern = fwd ? (nt == 8 ? cv::conv_silu_bf16_kernel<true, 8> : cv::conv_silu_bf16_kernel<true, 16>)
+                      : (nt == 8 ? cv::conv_silu_bf16_kernel<false, 8> : cv::conv_silu_bf16_kernel<false, 16>);
+      const cudaError_t e = r2l::launch_pdl(kern, grid, dim3(cv::THREADS), 0, st, (const bf16*)xz, 2 * E, u, E,
+                                            (const float*)w->conv_w, (const float*)w->conv_b, (const int*)len, L);
       if (e != cudaSuccess) return R2L_ERR_CUDA;
       R2L_LAUNCH_CHECK();
     } else {

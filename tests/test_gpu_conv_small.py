@@ -1,8 +1,9 @@
 """The separate conv + SiLU kernel (batches below one 128-row tile per SM, where
 x_proj runs on its own, unsplit or split along K) against the oracle of
 "Bifocal Diffusion Language Models" (arXiv 2606.27732v1, §3.4 steps ❶–❷), at
-three batch sizes: 9600, 3200 and 600 tokens.  Lengths end part-way through a
-thread's 16 tokens; u, Δr, C, y, o and ĥ are compared, in both directions,
+three batch sizes: 9600, 3200 and 600 tokens (16 tokens per conv thread at the
+first two, 8 at the last).  Lengths end part-way through a thread's tokens;
+u, Δr, C, y, o and ĥ are compared, in both directions,
 and padding rows of h must stay untouched.  At 600 tokens out_proj also runs
 split along K, its partial sums added by the LayerNorm kernel."""
 import numpy as np
