@@ -112,3 +112,13 @@ def test_hook_backward_gemm_flops():
     per_token = 2 * (2048 * 8192 + 4096 * 160 + 128 * 4096 + 4096 * 2048)
     assert per_token == 52690944
     assert bench.hook_bwd_gemm_flops(case) == 3 * per_token * 8
+
+
+def test_cpu_baseline_of_a_one_sequence_batch():
+    """The forward line's cpu_baseline samples at most the batch's sequences
+    (config 1 and config 0 hold one)."""
+    from reverse_selective_ssm_b200 import synthetic as S
+    case = S.make_case(0)
+    assert case.B == 1
+    cb = bench.cpu_baseline(case)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and "[0]" in cb["sample"]
