@@ -384,7 +384,7 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   if (osplit) {
     r2l::TcGemm gm{};
     gm.A = (const bf16*)y; gm.lda = E; gm.B = (const bf16*)w->out_proj_w; gm.ldb = E;
-    gm.C = nullptr; gm.ldc = d; gm.c_fp32 = true; gm.keep_partials = true;
+    gm.C = nullptr; gm.ldc = d; gm.c_fp32 = true; gm.keep_partials = true; gm.kept_splits = p.osplits;
     gm.M = (int)M; gm.N = d; gm.K = E; gm.len = len; gm.L = L; gm.err = err;
     gm.partial = (float*)(ws + p.osplit); gm.partial_bytes = p.osplit_bytes;
     if (r2l::tc_gemm(gm, st) != cudaSuccess) return R2L_ERR_CUDA;

@@ -159,7 +159,7 @@ cudaError_t launch(const TcGemm& g, cudaStream_t st) {
   int splits = 1;
   if constexpr (std::is_same<TOut, float>::value) {
     if (g.keep_partials) {
-      const int sp = tc_gemm_kept_splits(g.M, g.N, g.K);
+      const int sp = g.kept_splits;
       const size_t need = (size_t)sp * num_m * Cfg::BM * g.N * sizeof(float);
       if (BN != 256 || MB != 1 || sp < 1 || !g.partial || g.partial_bytes < need) return cudaErrorInvalidValue;
       splits = sp;

@@ -26,10 +26,13 @@ struct TcGemm {
   unsigned* err;           // device status word (timeout flag)
   float* partial;          // optional scratch for split-K partial sums (fp32 C only), or null
   size_t partial_bytes;
-  // keep_partials (fp32 C only): run on 128 × 256 tiles with tc_gemm_kept_splits
-  // splits and leave the partial sums in `partial` as [splits][Mp][N], Mp = M
-  // rounded up to 128, for the caller to add in split order; C is not written.
+  // keep_partials (fp32 C only): run on 128 × 256 tiles with kept_splits (≥ 1,
+  // normally tc_gemm_kept_splits of the shape, decided by the caller so that it
+  // and the code adding the slices agree) K splits and leave the partial sums
+  // in `partial` as [kept_splits][Mp][N], Mp = M rounded up to 128, for the
+  // caller to add in split order; C is not written.
   bool keep_partials;
+  int kept_splits;
 };
 
 // Streaming multiprocessors of the current device (148 on B200).
