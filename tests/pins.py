@@ -324,8 +324,9 @@ def pin_right_context_only(O):
 
 
 def pin_ragged_isolation(O):
-    """A sequence in a right-padded batch equals the same sequence alone; the
-    padding (NaN) is never read and is returned unchanged."""
+    """A sequence in a right-padded batch equals the same sequence alone, and
+    equals the independently written forward block through the flip (C3, C7);
+    the padding (NaN) is never read and is returned unchanged."""
     rng = RNG(13)
     w = tiny_weights(rng)
     B, L, d = 3, 10, w["W_in"].shape[1]
@@ -337,22 +338,37 @@ def pin_ragged_isolation(O):
     for b, n in enumerate(lengths):
         alone = O.sidecar_sequence(h[b, :n], w, 0.9) if n > 0 else h[b, :0]
         assert np.array_equal(out[b, :n], alone), f"sequence {b} differs from running alone"
+        if n > 0:
+            want = h[b, :n] + np.tanh(0.9) * forward_mamba_block_l2r(h[b, :n][::-1].copy(), w)[::-1]
+            _close(out[b, :n], want, 1e-11, f"sequence {b} against the forward block through the flip")
         assert np.all(np.isnan(out[b, n:])), f"padding of sequence {b} was written"
         assert np.all(np.isfinite(out[b, :n]))
 
 
 def pin_stack_composition(O):
-    """Hooks compose: the stack equals applying the hooks one by one with the
-    hidden state rounded to the storage dtype in between."""
+    """Hooks compose in order, each with its own weights and gate: the stack
+    (fp64 between hooks) on a ragged batch equals the hooks applied one after
+    another through the independently written forward block and the flip (C3);
+    and with bf16 storage each hook's output is rounded before the next hook
+    reads it."""
     rng = RNG(14)
     ws = [tiny_weights(rng) for _ in range(3)]
     ss = [0.3, -0.7, 0.5]
-    h = O.round_to_bf16(rng.normal(size=(2, 6, ws[0]["W_in"].shape[1])))
-    cur = h
+    lengths = [6, 4]
+    h = rng.normal(size=(2, 6, ws[0]["W_in"].shape[1]))
+    h[1, 4:] = np.nan
+    got = O.sidecar_stack(h, ws, ss, lengths=lengths)
+    for b, n in enumerate(lengths):
+        cur = h[b, :n].copy()
+        for w, s in zip(ws, ss):
+            cur = cur + np.tanh(s) * forward_mamba_block_l2r(cur[::-1].copy(), w)[::-1]
+        _close(got[b, :n], cur, 1e-10, f"stack of 3 hooks, sequence {b}")
+        assert np.all(np.isnan(got[b, n:])), f"padding of sequence {b} was written"
+    hb = O.round_to_bf16(rng.normal(size=(2, 6, ws[0]["W_in"].shape[1])))
+    cur = hb
     for w, s in zip(ws, ss):
         cur = O.round_to_bf16(O.sidecar_forward(cur, w, s))
-    got = O.sidecar_stack(h, ws, ss, out_dtype="bf16")
-    assert np.array_equal(got, cur)
+    assert np.array_equal(O.sidecar_stack(hb, ws, ss, out_dtype="bf16"), cur)
 
 
 def pin_l2r_direction(O):

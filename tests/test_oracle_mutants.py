@@ -85,6 +85,20 @@ def _silu_as_sigmoid(v):
     return 1.0 / (1.0 + np.exp(-v))
 
 
+def _stack_reversed(h, weights_list, s_list, lengths=None, out_dtype="f64", batch_indices=None):
+    cur = np.asarray(h, dtype=np.float64)
+    for w, s in zip(reversed(weights_list), reversed(s_list)):
+        cur = R.sidecar_forward(cur, w, s, lengths, out_dtype, batch_indices)
+    return cur
+
+
+def _stack_gates_rotated(h, weights_list, s_list, lengths=None, out_dtype="f64", batch_indices=None):
+    cur = np.asarray(h, dtype=np.float64)
+    for w, s in zip(weights_list, list(s_list[1:]) + list(s_list[:1])):
+        cur = R.sidecar_forward(cur, w, s, lengths, out_dtype, batch_indices)
+    return cur
+
+
 MUTANTS = {
     "conv taps reversed": ("anticausal_conv_silu", _conv_taps_reversed),
     "conv causal direction": ("anticausal_conv_silu", _conv_causal),
@@ -102,6 +116,8 @@ MUTANTS = {
     "dt drops bias": ("dt_softplus", _dt_no_bias),
     "softplus replaced by exp": ("softplus", _softplus_as_exp),
     "silu replaced by sigmoid": ("silu", _silu_as_sigmoid),
+    "stack applies the hooks in reverse order": ("sidecar_stack", _stack_reversed),
+    "stack pairs the gates with the wrong hooks": ("sidecar_stack", _stack_gates_rotated),
 }
 
 
