@@ -363,10 +363,12 @@ def sidecar_forward_train(hidden: torch.Tensor, weights, dims: Dims, s: float, l
 
 def sidecar_backward(hidden: torch.Tensor, weights, dims: Dims, s: float, dh_out: torch.Tensor,
                      grads: Dict[str, Optional[torch.Tensor]], lengths=None, workspace: Optional[torch.Tensor] = None,
-                     stream=None, check: bool = True):
+                     stream=None, check: bool = True, dh: Optional[torch.Tensor] = None,
+                     ds: Optional[torch.Tensor] = None):
     """r2l_sidecar_backward: returns (dh [B, L, d] fp32, ds (a 1-element fp32
     device tensor)); grads (from alloc_grads) receives every parameter's
-    gradient."""
+    gradient.  dh and ds may be given (fp32 [B, L, d] and at least 4 floats,
+    caller-owned); they are allocated here otherwise."""
     lib = load()
     B, L = hidden.shape[0], hidden.shape[1]
     if workspace is None:
@@ -376,8 +378,10 @@ def sidecar_backward(hidden: torch.Tensor, weights, dims: Dims, s: float, dh_out
     g = Grads()
     for key, field in _WMAP:
         setattr(g, field, _ptr(grads.get(key)))
-    dh = torch.empty(dh_out.shape, dtype=torch.float32, device=hidden.device)
-    ds = torch.zeros(4, dtype=torch.float32, device=hidden.device)
+    if dh is None:
+        dh = torch.empty(dh_out.shape, dtype=torch.float32, device=hidden.device)
+    if ds is None:
+        ds = torch.zeros(4, dtype=torch.float32, device=hidden.device)
     st = lib.r2l_sidecar_backward(_ptr(hidden), ctypes.byref(w), ctypes.byref(dims), float(s), B, L, _ptr(lengths),
                                   _ptr(dh_out), _ptr(dh), _ptr(ds), ctypes.byref(g), _ptr(workspace),
                                   workspace.numel(), _stream_ptr(stream))
