@@ -1,11 +1,11 @@
 """The separate conv + SiLU kernel (batches below one 128-row tile per SM, where
 x_proj runs on its own, unsplit or split along K) against the oracle of
 "Bifocal Diffusion Language Models" (arXiv 2606.27732v1, §3.4 steps ❶–❷), at
-three batch sizes: 9600, 3200 and 600 tokens (16 tokens per conv thread at the
-first two, 8 at the last).  Lengths end part-way through a thread's tokens;
+four batch sizes: 9600, 3200, 600 and 128 tokens (16 tokens per conv thread at
+the first two, 8 at the others).  Lengths end part-way through a thread's tokens;
 u, Δr, C, y, o and ĥ are compared, in both directions,
-and padding rows of h must stay untouched.  At 600 tokens out_proj also runs
-split along K, its partial sums added by the LayerNorm kernel."""
+and padding rows of h must stay untouched.  At 600 and 128 tokens out_proj
+also runs split along K, its partial sums added by the LayerNorm kernel."""
 import numpy as np
 import pytest
 import torch
@@ -20,11 +20,13 @@ pytestmark = pytest.mark.gpu
 
 # (B, L, lengths, sequences checked in full), all below the 18,944 rows where the
 # fused conv/x_proj kernel takes over; x_proj runs unsplit at 9600 rows (75
-# tiles) and split along K at 3200 and 600
+# tiles) and split along K at 3200, 600 and 128; out_proj runs split along K
+# into the LayerNorm kernel at 600 rows (3 slices) and 128 (8 slices)
 CASES = {
     "b8_l1200": (8, 1200, [1200, 1199, 1, 0, 1185, 1200, 17, 1200], (1, 6)),
     "b4_l800": (4, 800, [800, 793, 9, 800], (1, 2)),
     "b2_l300": (2, 300, [300, 299], (0, 1)),
+    "b1_l128": (1, 128, [121], (0,)),
 }
 
 
