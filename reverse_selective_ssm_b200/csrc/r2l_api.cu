@@ -42,6 +42,7 @@ struct Plan {
   size_t status, len, aflags, xz, u, dbc, dr, dt, y, o, carry, xsplit, xsplit_bytes, osplit, osplit_bytes, total;
   int chunk_tokens;  // scan chunk length (bf16 path)
   int osplits;       // out_proj K splits left to the LayerNorm kernel (0: o stored by the GEMM)
+  bool ragged = false;  // the caller gave per-sequence lengths (set by the entry point)
   long long M;
   int E, d, R, N, ldd;
   size_t act;
@@ -207,9 +208,10 @@ r2l_status check_a_log_hooks(const r2l_weights* w, int n, int E, unsigned* flags
 template <typename T, typename TC>
 r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long long M, int N, int K,
                 const int* len, int L, unsigned* err, cudaStream_t st, bf16* c2 = nullptr, int ldc2 = 0,
-                int c2_cols = 0, float* partial = nullptr, size_t partial_bytes = 0) {
+                int c2_cols = 0, float* partial = nullptr, size_t partial_bytes = 0, bool ragged = false) {
   if constexpr (std::is_same<T, bf16>::value) {
     r2l::TcGemm g{};
+    g.ragged = ragged;
     g.A = A; g.lda = lda; g.B = W; g.ldb = ldw; g.C = C; g.ldc = ldc;
     g.c_fp32 = std::is_same<TC, float>::value;
     g.C2 = c2; g.ldc2 = ldc2; g.c2_cols = c2_cols;
@@ -287,7 +289,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
   // a1: [x | z] = h · W_inᵀ
   R2L_TRY(prof->mark(R2L_STAGE_IN_PROJ, st));
   prof->launches++;
-  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st));
+  R2L_TRY(proj(hidden, d, (const T*)w->in_proj_w, d, xz, 2 * E, M, 2 * E, d, len, L, err, st, nullptr, 0, 0, nullptr,
+               0, p.ragged));
   // a2: u = SiLU(anti-causal conv(x)); a3: [Δr | B | C] = u · W_xᵀ (fp32 out).
   // bf16 with an x_proj of 160 columns and at least one 128-row tile per SM:
   // one kernel does both (the conv runs in x_proj's operand producer and u
@@ -395,7 +398,8 @@ r2l_status run_layer(T* hidden, const r2l_weights* w, const Plan& p, float g, in
         return R2L_ERR_CUDA;
     }
   } else {
-    R2L_TRY(proj(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, err, st));
+    R2L_TRY(proj(y, E, (const T*)w->out_proj_w, E, o, d, M, d, E, len, L, err, st, nullptr, 0, 0, nullptr, 0,
+                 p.ragged));
   }
 
   if (dbg) {
@@ -442,6 +446,7 @@ r2l_status forward_impl(void* hidden, const r2l_weights* weights, const r2l_dims
                         Prof* prof = nullptr) {
   Plan p;
   R2L_TRY(check_call(hidden, dims, B, L, workspace, workspace_bytes, &p));
+  p.ragged = lengths != nullptr;
   R2L_TRY(check_weights(weights));
   if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
   const float g = (float)std::tanh((double)s);
@@ -517,6 +522,7 @@ r2l_status r2l_sidecar_stack(void* hidden, const r2l_weights* weights, const flo
   if (!weights || !s || n_hooks <= 0) return R2L_ERR_INVALID_ARG;
   Plan p;
   R2L_TRY(check_call(hidden, dims, B, L, workspace, workspace_bytes, &p));
+  p.ragged = lengths != nullptr;
   for (int k = 0; k < n_hooks; ++k) R2L_TRY(check_weights(&weights[k]));
   if (lengths && ((uintptr_t)lengths & 3u)) return R2L_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
@@ -810,6 +816,7 @@ r2l_status backward_impl(const void* hidden, const r2l_weights* w, const r2l_dim
   namespace K = r2l::bwd;
   BwdPlan q;
   if (!make_bwd_plan(dims, B, L, &q)) return R2L_ERR_INVALID_ARG;
+  q.f.ragged = lengths != nullptr;
   const Plan& p = q.f;
   char* ws = (char*)workspace;
   const long long M = p.M, Mp = q.Mp;
@@ -1006,6 +1013,7 @@ r2l_status r2l_sidecar_forward_train(const void* hidden, void* out, const r2l_we
   if (!aligned16(out)) return R2L_ERR_ALIGNMENT;
   BwdPlan q;
   make_bwd_plan(dims, B, L, &q);
+  q.f.ragged = lengths != nullptr;
   cudaStream_t st = (cudaStream_t)stream;
   // h⁺ is formed in `out` (a copy of h, updated in place on valid rows); h,
   // which the gradient reads again, stays as it is

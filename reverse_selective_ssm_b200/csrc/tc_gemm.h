@@ -33,6 +33,9 @@ struct TcGemm {
   // caller to add in split order; C is not written.
   bool keep_partials;
   int kept_splits;
+  // the rows come from sequences of different lengths (right-padded): 128-row
+  // tiles, which waste fewer padding rows at each sequence's end than 256-row ones
+  bool ragged;
 };
 
 // Streaming multiprocessors of the current device (148 on B200).
