@@ -225,8 +225,9 @@ r2l_status proj(const T* A, int lda, const T* W, int ldw, TC* C, int ldc, long l
 
 // LayerNorm + gated residual for bf16 rows of d <= 2048 (nv = ceil(d / 256)).
 // With ps (the out_proj partial sums of a small batch, `splits` slices of
-// `slice` floats) o is added up from them, and written to `o` only when
-// o_keep is set (the debug entry point).
+// `slice` floats) o is added up from them, and written to `o` when o_keep is
+// set (the layer always sets it: the gradient of a training forward and the
+// debug entry point read o back).
 template <int NV>
 r2l_status ln_bf16_nv(bool has_ln, unsigned blocks, cudaStream_t st, bf16* h, const bf16* o, const float* lw,
                       const float* lb, float g, int d, const int* len, int L, long long M, float* hhat,
