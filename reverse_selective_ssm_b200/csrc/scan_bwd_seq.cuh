@@ -324,14 +324,16 @@ __device__ __forceinline__ void qgstep(const QLane& l, QSmem& S, int r, const fl
   __syncwarp();
   {
     const int col = l.j + 16 * l.h;                     // the lane index
-    float t[16];
+    // a fixed pairwise tree, t[i] += t[i + w] for w = 8, 4, 2, 1, its adds
+    // taken two at a time as packed f32x2 (the same additions, the same bits)
+    float2 t[8];
 #pragma unroll
-    for (int ch = 0; ch < 16; ++ch) t[ch] = S.xb[l.w][ch][col];
+    for (int ch = 0; ch < 8; ++ch) t[ch] = make_float2(S.xb[l.w][2 * ch][col], S.xb[l.w][2 * ch + 1][col]);
 #pragma unroll
-    for (int w = 8; w >= 1; w >>= 1)                    // a fixed pairwise tree
+    for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
-      for (int i = 0; i < w; ++i) t[i] += t[i + w];
-    S.red[l.w][r][col] = t[0];
+      for (int i = 0; i < w; ++i) t[i] = __fadd2_rn(t[i], t[i + w]);
+    S.red[l.w][r][col] = t[0].x + t[0].y;
   }
   // the gradients (both halves of a channel hold the same sums) go over the
   // row's staged scalars, which no later step reads
