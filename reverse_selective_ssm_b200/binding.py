@@ -380,8 +380,12 @@ def sidecar_backward(hidden: torch.Tensor, weights, dims: Dims, s: float, dh_out
         setattr(g, field, _ptr(grads.get(key)))
     if dh is None:
         dh = torch.empty(dh_out.shape, dtype=torch.float32, device=hidden.device)
+    elif dh.dtype != torch.float32 or dh.shape != dh_out.shape:
+        raise ValueError("dh must be fp32 and shaped like dh_out")
     if ds is None:
         ds = torch.zeros(4, dtype=torch.float32, device=hidden.device)
+    elif ds.dtype != torch.float32 or ds.numel() < 4:
+        raise ValueError("ds must be fp32 with at least 4 elements")
     st = lib.r2l_sidecar_backward(_ptr(hidden), ctypes.byref(w), ctypes.byref(dims), float(s), B, L, _ptr(lengths),
                                   _ptr(dh_out), _ptr(dh), _ptr(ds), ctypes.byref(g), _ptr(workspace),
                                   workspace.numel(), _stream_ptr(stream))
